@@ -1,0 +1,5 @@
+"""fp64 CPU oracle for the HyLRA decode path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package.  The product path never does.
+"""

@@ -1,0 +1,94 @@
+"""Pins for the oracle's overlap matrix and DP policy (CPU only)."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import hylra_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_similarity_hand_worked():
+    g = _load("similarity_3layer.json")
+    M = O.similarity_matrix(np.array(g["topk"]))
+    assert M.tolist() == g["M"]
+
+
+def test_similarity_identical_and_disjoint():
+    a = np.array([[[0, 1, 2, 3]], [[3, 2, 1, 0]], [[4, 5, 6, 7]]])
+    M = O.similarity_matrix(a)
+    assert M[1, 0] == 1.0 and M[2, 0] == 0.0 and M[2, 1] == 0.0
+    assert np.all(np.diag(M) == 1.0)
+    assert np.all(np.triu(M, 1) == 0.0)
+
+
+def test_similarity_padding_is_ignored():
+    a = np.array([[[0, 1, -1, -1]], [[1, 5, -1, -1]]])
+    M = O.similarity_matrix(a)
+    assert M[1, 0] == 0.5 and M[1, 1] == 1.0
+
+
+def _dyadic_matrix(L, rng, denom=64):
+    M = np.zeros((L, L))
+    for t in range(L):
+        for s in range(t):
+            M[t, s] = rng.integers(0, denom + 1) / denom
+        M[t, t] = 1.0
+    return M
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("theta", [0.0, 0.25, 0.5, 0.8, 1.0])
+def test_dp_matches_bruteforce(L, theta):
+    rng = np.random.default_rng(L * 100 + int(theta * 100))
+    for _ in range(25):
+        M = _dyadic_matrix(L, rng)
+        assert O.dp_policy(M, theta) == O.dp_policy_bruteforce(M, theta)
+
+
+def test_dp_hand_worked():
+    g = _load("dp_4layer.json")
+    M = np.array(g["M"])
+    for case in g["cases"]:
+        pol, R, S = O.dp_policy(M, case["theta"])
+        assert list(pol) == case["policy"]
+        assert R == case["resets"]
+        assert S == case["sim"]
+
+
+def test_dp_closed_forms():
+    rng = np.random.default_rng(7)
+    for L in (4, 9, 16, 32):
+        M = _dyadic_matrix(L, rng)
+        # theta >= 1: no similarity can exceed it -> every layer resets
+        pol, R, S = O.dp_policy(M, 1.0)
+        assert pol == (1,) * L and R == L and S == 0.0
+        # theta below every entry: one reset; the best source is layer 0 or a
+        # later reset, but a single reset already minimises -> sim = sum M[j][0]
+        pol, R, S = O.dp_policy(M, -1.0)
+        assert R == 1 and pol == (1,) + (0,) * (L - 1)
+        assert S == sum(M[j, 0] for j in range(1, L))
+
+
+def test_dp_resets_monotone_in_theta():
+    rng = np.random.default_rng(11)
+    M = _dyadic_matrix(12, rng)
+    last = 0
+    for theta in np.linspace(-0.1, 1.0, 23):
+        _, R, _ = O.dp_policy(M, theta)
+        assert R >= last
+        last = R
+
+
+def test_dp_strict_threshold():
+    M = np.array([[1.0, 0.0], [0.5, 1.0]])
+    assert O.dp_policy(M, 0.5)[0] == (1, 1)     # 0.5 does not exceed 0.5
+    assert O.dp_policy(M, 0.4999)[0] == (1, 0)
