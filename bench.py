@@ -1,0 +1,528 @@
+"""HyLRA decode-attention benchmark (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one decode step of the whole hot path: every layer of the model,
+a reset layer running full attention + block scoring + top-k, a reuse layer
+attending over the blocks the most recent reset layer selected, under the
+policy the DP derives from a profiling run (all layers full) of the same
+synthetic workload.  Inputs are resident in HBM before timing starts; each
+step streams more bytes than the 126 MB L2 holds.
+
+value      = device time per hybrid decode step (us), max over ranks
+e2e        = the same step through the C-ABI host-buffer entry point
+             (q copied host->device, outputs device->host, inside the timing)
+roofline   = the full (reset-layer) kernel: K+V bytes of one layer per launch
+             over its average duration in the all-full step
+cpu_baseline / --impl reference = the fp64 oracle on the host cores
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_sparsity_b200 import build as hbuild  # noqa: E402
+from kv_cache_sparsity_b200 import workloads as W  # noqa: E402
+
+METRIC = ("decode-attention µs/step & KV HBM GB/s vs ~8 TB/s; HyLRA vs full speedup")
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- helpers
+
+def workload_desc(w: W.Workload) -> str:
+    lens = (f"context {w.seqlens[0]}" if len(set(w.seqlens)) == 1
+            else f"ragged contexts {min(w.seqlens)}..{max(w.seqlens)} (sum {w.total_tokens})")
+    pol = "DP policy theta=%g" % w.theta if w.policy is None else "fixed policy"
+    return (f"{w.name}: batch {w.batch}, {w.layers} layers, {w.num_q_heads} q / "
+            f"{w.num_kv_heads} KV heads, head_dim {w.head_dim}, {w.dtype} K/V, {lens}, "
+            f"block 128, top-k {w.topk}, {pol}, {'packed' if w.packed else 'dense'} layout")
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel_tag: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken
+    on the current kernel source (null otherwise)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    src = b""
+    for fn in ("hylra_kernels.cuh", "hylra_device.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_sparsity_b200", "csrc", fn), "rb") as f:
+            src += f.read()
+    sha = hashlib.sha256(src).hexdigest()[:16]
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != sha:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the GPU works."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        busy = [r for r in rows if _num(r[4]) and _num(r[4]) > 0] or rows
+        sm = [_num(r[1]) for r in busy if _num(r[1])]
+        smax = [_num(r[2]) for r in rows if _num(r[2])]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in busy for i in range(4) if "Active" in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(busy)}
+
+
+def _num(x):
+    try:
+        return float(x)
+    except ValueError:
+        return None
+
+
+# ----------------------------------------------------------------- our arm
+
+class Model:
+    """All layers of one synthetic workload resident on this GPU."""
+
+    def __init__(self, w: W.Workload, H, resident_layers: int):
+        self.w, self.H = w, H
+        dev = "cuda"
+        self.seqlens = torch.tensor(w.seqlens, dtype=torch.int32, device=dev)
+        self.offs = (torch.tensor(W.seq_offsets(w)[:-1], dtype=torch.int64, device=dev)
+                     if w.packed else None)
+        dtype = H.BF16 if w.dtype == "bf16" else H.FP32
+        if w.packed:
+            self.shape = H.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.topk,
+                                      w.max_seqlen, dtype=dtype, total_tokens=w.total_tokens,
+                                      seq_offsets=self.offs)
+        else:
+            self.shape = H.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.topk,
+                                      w.max_seqlen, dtype=dtype, kv_capacity=w.max_seqlen)
+        self.ws = torch.empty(H.workspace_bytes(self.shape), dtype=torch.uint8, device=dev)
+        H.workspace_init(self.ws)
+        self.resident = resident_layers
+        self.q, self.K, self.V = [], [], []
+        for l in range(w.layers):
+            q, K, V = W.layer_inputs(w, l, device=dev)
+            self.q.append(q)
+            if l < resident_layers:
+                self.K.append(K)
+                self.V.append(V)
+            else:
+                del K, V
+        torch.cuda.synchronize()
+        self.Ks = [self.K[l % resident_layers] for l in range(w.layers)]
+        self.Vs = [self.V[l % resident_layers] for l in range(w.layers)]
+        self.outs = [torch.empty(w.batch, w.num_q_heads, w.head_dim, device=dev)
+                     for _ in range(w.layers)]
+        self.topk = torch.full((w.layers, w.batch, w.num_kv_heads, w.topk), -1,
+                               dtype=torch.int32, device=dev)
+
+    def step(self, policy, stream=None):
+        self.H.decode_step(self.shape, policy, self.q, self.Ks, self.Vs, self.seqlens,
+                           self.outs, self.topk, self.ws, stream=stream)
+
+    def graph(self, policy):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step(policy)  # warm (one-time host setup outside capture)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.step(policy, stream=torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        return g
+
+
+def derive_policy(m: Model, H):
+    """Profiling run (every layer full) -> overlap matrix -> DP policy."""
+    w = m.w
+    if w.policy is not None:
+        return tuple(w.policy), None
+    allfull = (1,) * w.layers
+    m.step(allfull)
+    torch.cuda.synchronize()
+    tk = m.topk.cpu().numpy().reshape(w.layers, w.batch * w.num_kv_heads, w.topk)
+    M = H.similarity(tk)
+    pol, R, S = H.dp_policy(M, w.theta)
+    return pol, M
+
+
+def timed_replays(g, steps, dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    return e0.elapsed_time(e1) / steps
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
+    """Through hylra_decode_step_host: q from pinned host memory, outputs back."""
+    w = m.w
+    q_host = torch.stack([q.cpu() for q in m.q]).pin_memory()
+    q_dev = torch.empty_like(q_host, device="cuda")
+    out_dev = torch.empty(w.layers, w.batch, w.num_q_heads, w.head_dim, device="cuda")
+    out_host = torch.empty(out_dev.shape, dtype=torch.float32).pin_memory()
+    tk_dev = torch.full((w.layers, w.batch, w.num_kv_heads, w.topk), -1, dtype=torch.int32,
+                        device="cuda")
+    tk_host = torch.empty(tk_dev.shape, dtype=torch.int32).pin_memory()
+
+    def one():
+        H.decode_step_host(m.shape, policy, q_host, q_dev, m.Ks, m.Vs, m.seqlens, out_dev,
+                           out_host, tk_dev, tk_host, m.ws)
+
+    for _ in range(warmup):
+        one()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * 4 + tk_host.numel() * 4
+    return ms, h2d, d2h
+
+
+def oracle_sample(w: W.Workload, m: Model, policy, heads=(0,), reps=1):
+    """Time the fp64 oracle on a bounded sample of one decode step: all
+    layers under ``policy`` for the KV heads ``heads`` of every sequence.
+    Returns (seconds per full step scaled to all heads, sample text, threads)."""
+    from oracle import hylra_oracle as O
+    r = w.group
+    data = []
+    for l in range(w.layers):
+        q = m.q[l].double().cpu().numpy()
+        K, V = m.Ks[l], m.Vs[l]
+        per_b = []
+        for b in range(w.batch):
+            kb = W.per_sequence(w, K, b)
+            vb = W.per_sequence(w, V, b)
+            per_b.append((q[b][[g for h in heads for g in range(h * r, (h + 1) * r)]],
+                          kb[list(heads)].double().cpu().numpy(),
+                          vb[list(heads)].double().cpu().numpy()))
+        data.append(per_b)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        current = [None] * w.batch
+        for l in range(w.layers):
+            for b in range(w.batch):
+                qb, kb, vb = data[l][b]
+                n = w.seqlens[b]
+                if policy[l]:
+                    _, _, current[b] = O.full_layer(qb, kb, vb, n, w.topk)
+                else:
+                    O.reuse_attention(qb, kb, vb, n, current[b])
+    dt = (time.perf_counter() - t0) / reps
+    scale = w.num_kv_heads / len(heads)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    sample = (f"{reps} decode step(s) of all {w.layers} layers under the bench policy for "
+              f"KV head(s) {list(heads)} of {w.num_kv_heads} of every sequence, scaled x{scale:g}")
+    return dt * scale, sample, threads
+
+
+def run_ours(args, rank, world, dist_on):
+    from kv_cache_sparsity_b200 import hylra as H
+    hbuild.build()
+    H.load()
+    w = W.config(args.config)
+    free = torch.cuda.mem_get_info()[0]
+    per_layer = w.kv_bytes_per_layer()  # K and V bytes of one layer
+    resident = w.layers
+    if per_layer * w.layers > free * 0.85:
+        resident = max(1, int(free * 0.85 // per_layer))
+    m = Model(w, H, resident)
+    policy, M = derive_policy(m, H)
+    allfull = (1,) * w.layers
+    R = sum(policy)
+    g_h = m.graph(policy)
+    g_f = m.graph(allfull)
+    for _ in range(args.warmup):
+        g_h.replay()
+        g_f.replay()
+    torch.cuda.synchronize()
+    assert H.read_status(m.ws) == 0, "device status set during warm-up"
+
+    uuid = str(getattr(torch.cuda.get_device_properties(0), "uuid", ""))
+    if uuid and not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    clk = ClockSampler(uuid)
+    clk.start()
+    ms_h = timed_replays(g_h, args.steps, dist_on)
+    ms_f = timed_replays(g_f, args.steps, dist_on)
+    # keep the GPU busy long enough for the sampler when the timed region is short
+    t_end = time.time() + max(0.0, 0.6 - (ms_h + ms_f) * args.steps / 1000.0)
+    while time.time() < t_end:
+        g_h.replay()
+        torch.cuda.synchronize()
+    clocks = clk.stop()
+    ms_h = max_over_ranks(ms_h, dist_on)
+    ms_f = max_over_ranks(ms_f, dist_on)
+    status = H.read_status(m.ws)
+
+    e2e_ms, h2d, d2h = e2e_step_time(m, H, policy, max(3, args.steps // 4), args.warmup,
+                                     dist_on)
+    e2e_ms = max_over_ranks(e2e_ms, dist_on)
+    del g_h, g_f
+
+    full_b = w.kv_bytes_per_layer()
+    reuse_b = w.kv_bytes_reuse_layer()
+    step_bytes = R * full_b + (w.layers - R) * reuse_b
+    us_h = ms_h * 1000.0
+    kv_gbs = step_bytes / (ms_h * 1e-3) / 1e9
+    full_launch_us = ms_f * 1000.0 / w.layers
+    achieved = full_b / (full_launch_us * 1e-6) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    line = {
+        "metric": METRIC,
+        "value": round(us_h, 3),
+        "unit": "us/step",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_h, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
+        "config": {
+            "workload": workload_desc(w),
+            "policy": "".join("R" if x else "U" for x in policy),
+            "resets": R,
+            "resident_layer_caches": m.resident,
+            "l2": "inputs larger than L2: a step streams %.2f GB" % (step_bytes / 1e9),
+            "replicas": "each rank runs its own copy of the workload" if world > 1 else None,
+        },
+        "kv_bytes_per_step": step_bytes,
+        "kv_gbs": round(kv_gbs, 1),
+        "kv_frac_of_8tbs": round(kv_gbs / NOMINAL_HBM_GBS, 4),
+        "full_us_per_step": round(ms_f * 1000.0, 3),
+        "speedup_vs_full": round(ms_f / ms_h, 4),
+        "sequences_per_s_all_ranks": round(world * w.batch / (ms_h * 1e-3), 1),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode_bf16_kernel<full> (reset layer)",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": ncu_traffic("full_kernel", w.name),
+            "algorithmic_bytes_per_launch": full_b,
+            "avg_launch_us": round(full_launch_us, 3),
+        },
+        "e2e": {"value": round(e2e_ms * 1000.0, 3), "unit": "us/step",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": w.layers * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, sample, threads = oracle_sample(w, m, policy, heads=(0,), reps=1)
+        line["cpu_baseline"] = {"value": round(sec * 1e6, 1), "unit": "us/step",
+                                "cores": threads, "kind": "oracle", "sample": sample}
+    return line
+
+
+# ----------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The fp64 oracle, as it stands, on the host cores (no GPU needed)."""
+    from oracle import hylra_oracle as O
+    w = W.config(args.config)
+    heads = (0,)  # bounded sample: one KV head of every sequence, scaled to all heads
+
+    class _M:
+        pass
+
+    m = _M()
+    m.q, m.Ks, m.Vs = [], [], []
+    for l in range(w.layers):
+        q, K, V = W.layer_inputs(w, l, device="cpu")
+        m.q.append(q)
+        m.Ks.append(K)
+        m.Vs.append(V)
+    # policy: the oracle's own profiling + DP on this sample (every layer full)
+    if w.policy is not None:
+        policy = tuple(w.policy)
+    else:
+        sets = []
+        for l in range(w.layers):
+            per = []
+            for b in range(w.batch):
+                kb = W.per_sequence(w, m.Ks[l], b).double().numpy()
+                vb = W.per_sequence(w, m.Vs[l], b).double().numpy()
+                _, _, tk = O.full_layer(m.q[l][b].double().numpy(), kb, vb, w.seqlens[b],
+                                        w.topk)
+                per.extend(list(tk))
+            sets.append(per)
+        M = O.similarity_matrix(np.array(sets))
+        policy, _, _ = O.dp_policy(M, w.theta)
+    times = []
+    for _ in range(args.warmup):
+        oracle_sample(w, m, policy, heads=heads, reps=1)
+    sample = ""
+    threads = 1
+    for _ in range(args.steps):
+        sec, sample, threads = oracle_sample(w, m, policy, heads=heads, reps=1)
+        times.append(sec)
+    us = statistics.mean(times) * 1e6
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(us, 1),
+        "unit": "us/step",
+        "n_gpus": 0,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(us / 1000.0, 3),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
+        "config": {"workload": workload_desc(w),
+                   "policy": "".join("R" if x else "U" for x in policy)},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="llama8b_32k", choices=W.CONFIG_NAMES)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    line = run_ours(args, rank, world, dist_on)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -1,0 +1,188 @@
+/*
+ * hylra.h - C ABI of the HyLRA decode-attention library (B200, sm_100a).
+ *
+ * Method: "HyLRA: Hybrid Layer Reuse Attention for Efficient Long-Context
+ * Inference" (gist.science technical summary of arXiv 2602.00777), cited as
+ * "HyLRA summary" with its section numbers.
+ *
+ *   §2.3 Hybrid Inference Strategy: during decoding, a sensitive ("reset")
+ *        layer runs standard full attention and extracts top-k indices that
+ *        are passed forward; a tolerant ("reuse") layer reuses the indices of
+ *        the preceding reset layer and restricts attention to that subset of
+ *        the KV cache.                     -> hylra_decode_full, hylra_decode_reuse,
+ *                                             hylra_decode_step
+ *   §2.4 Block-level Sparsity: selection works on fixed 128-token blocks.
+ *   §2.2 Offline policy: a lower-triangular overlap matrix M of top-k indices
+ *        between source and target layers, and a dynamic program over states
+ *        (i, j) with reset jumps and vertical moves gated by theta.
+ *                                          -> hylra_similarity, hylra_dp_policy
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Every call returns an int status: HYLRA_OK (0) or a negative
+ *    hylra_error_t.  Bad arguments are detected on the host before anything
+ *    is launched; nothing is written in that case.
+ *  * Device entry points are asynchronous on the caller's stream.  They never
+ *    allocate, never synchronise and keep no state between calls; the caller
+ *    owns every buffer.  Data problems found on the device (a sequence length
+ *    beyond the cache, a block index out of range, a duplicate index) never
+ *    trap: the kernel skips the offending work and sets a bit in the status
+ *    word of the workspace, read with hylra_read_status.
+ *  * Shapes: B sequences, Hq query heads, Hkv KV heads (r = Hq / Hkv in
+ *    1..8; q-head g reads KV head g / r), head_dim d = 128, block = 128 tokens.
+ *    n_b = seqlens[b], NB_b = ceil(n_b / 128), k' = min(k, NB_b).
+ *  * q: [B][Hq][d] (bf16 or fp32, see dtype), out: [B][Hq][d] fp32.
+ *  * K, V: dense [B][Hkv][kv_capacity][d] (kv_capacity > 0), or packed
+ *    [Hkv][total_tokens][d] with sequence b at rows seq_offsets[b] ..
+ *    seq_offsets[b] + n_b - 1 of every KV-head plane (kv_capacity == 0).
+ *    Device pointers must be 16-byte aligned.
+ *  * top-k indices: int32 [B][Hkv][k], in rank order (largest block
+ *    attention mass first, lower block index first among equal fp32 scores);
+ *    slots k'..k-1 hold -1.
+ *  * One workspace may be used by one stream at a time.  It must be zeroed
+ *    once (hylra_workspace_init) before its first use; every call leaves it
+ *    ready for the next one.
+ */
+#ifndef HYLRA_H_
+#define HYLRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* hylra_stream_t;
+
+#define HYLRA_BLOCK_TOKENS 128
+#define HYLRA_HEAD_DIM 128
+#define HYLRA_MAX_GROUP 8          /* largest Hq / Hkv                      */
+#define HYLRA_MAX_BATCH 1024
+#define HYLRA_MAX_TOPK 1024
+#define HYLRA_MAX_SEQLEN 262144    /* 2048 blocks per sequence              */
+
+typedef enum {
+  HYLRA_OK = 0,
+  HYLRA_ERR_INVALID = -1,      /* null pointer, bad size, misaligned pointer   */
+  HYLRA_ERR_UNSUPPORTED = -2,  /* d != 128, block != 128, r > 8, limits above  */
+  HYLRA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed            */
+  HYLRA_ERR_WORKSPACE = -4,    /* workspace smaller than hylra_workspace_bytes */
+  HYLRA_ERR_INFEASIBLE = -5    /* no policy satisfies the constraints          */
+} hylra_error_t;
+
+typedef enum { HYLRA_BF16 = 0, HYLRA_FP32 = 1 } hylra_dtype_t;
+
+/* Bits of the device status word (hylra_read_status). */
+#define HYLRA_STATUS_BAD_SEQLEN 0x1u   /* n_b < 0, > max_seqlen, or beyond the cache: sequence skipped */
+#define HYLRA_STATUS_BAD_INDEX 0x2u    /* reuse index outside [0, NB_b) (and not -1): block skipped    */
+#define HYLRA_STATUS_DUP_INDEX 0x4u    /* a block index appears twice in one reuse list               */
+#define HYLRA_STATUS_NONFINITE 0x8u    /* a non-finite block score was met (treated as 0)             */
+#define HYLRA_STATUS_TIMEOUT 0x10u     /* a bounded wait inside a kernel gave up                      */
+
+typedef struct hylra_shape {
+  int32_t batch;         /* B, 1..HYLRA_MAX_BATCH                                        */
+  int32_t num_q_heads;   /* Hq                                                           */
+  int32_t num_kv_heads;  /* Hkv; Hq % Hkv == 0 and Hq / Hkv <= HYLRA_MAX_GROUP          */
+  int32_t head_dim;      /* must be 128                                                   */
+  int32_t block_size;    /* must be 128 (HyLRA summary §2.4)                              */
+  int32_t topk;          /* k, 1..HYLRA_MAX_TOPK                                          */
+  int32_t dtype;         /* hylra_dtype_t of q, K and V                                   */
+  int32_t max_seqlen;    /* upper bound on every seqlens[b]; sizes the workspace          */
+  int64_t kv_capacity;   /* dense: rows per (b, KV head) plane (>= max_seqlen); 0: packed */
+  int64_t total_tokens;  /* packed: rows per KV-head plane; ignored when dense           */
+  const int64_t* seq_offsets; /* packed: device int64 [B]; ignored when dense            */
+} hylra_shape_t;
+
+/* Bytes of workspace the decode calls need for this shape on the current
+ * device (it depends on the device's SM count).  Host only. */
+int hylra_workspace_bytes(const hylra_shape_t* shape, size_t* bytes);
+
+/* Zero a workspace (async cudaMemsetAsync on stream).  Needed once. */
+int hylra_workspace_init(void* workspace, size_t bytes, hylra_stream_t stream);
+
+/* Reset layer (HyLRA summary §2.3 "Sensitive Layers"): full single-query
+ * GQA attention over every cached token, plus the per-KV-head top-k of the
+ * 128-token blocks ranked by attention probability mass (summed over the r
+ * q-heads of the KV head).  seqlens: device int32 [B].  out: device fp32
+ * [B][Hq][d].  topk_out: device int32 [B][Hkv][k].  A sequence with n_b == 0
+ * gets a zero output and all -1 indices. */
+int hylra_decode_full(const hylra_shape_t* shape, const void* q, const void* K,
+                      const void* V, const int32_t* seqlens, float* out,
+                      int32_t* topk_out, void* workspace, size_t workspace_bytes,
+                      hylra_stream_t stream);
+
+/* Reuse layer (HyLRA summary §2.3 "Tolerant Layers"): attention restricted
+ * to the blocks listed in topk_in (device int32 [B][Hkv][k], as written by
+ * hylra_decode_full of an earlier layer), softmax renormalised over those
+ * tokens.  Only slots 0..k'-1 are read; -1 entries are skipped; an empty
+ * selection gives a zero output.  seqlens masks a partial last block. */
+int hylra_decode_reuse(const hylra_shape_t* shape, const void* q, const void* K,
+                       const void* V, const int32_t* seqlens, const int32_t* topk_in,
+                       float* out, void* workspace, size_t workspace_bytes,
+                       hylra_stream_t stream);
+
+/* One decode step over num_layers layers (HyLRA summary §2.3): layer l runs
+ * hylra_decode_full when policy[l] == 1 (writing topk + l*B*Hkv*k) and
+ * hylra_decode_reuse when policy[l] == 0 (reading the slot of the most recent
+ * reset layer).  policy[0] must be 1.  q, K, V, out: HOST arrays of
+ * num_layers DEVICE pointers.  topk: device int32 [num_layers][B][Hkv][k];
+ * slots of reuse layers are left untouched.  Capturable in a CUDA graph. */
+int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers,
+                      const uint8_t* policy, const void* const* q,
+                      const void* const* K, const void* const* V,
+                      const int32_t* seqlens, float* const* out, int32_t* topk,
+                      void* workspace, size_t workspace_bytes, hylra_stream_t stream);
+
+/* The same step with the per-step inputs and outputs in HOST memory:
+ * q_host [num_layers][B][Hq][d] is copied to q_dev (same shape, device) and,
+ * after the step, out_dev [num_layers][B][Hq][d] fp32 to out_host and
+ * topk_dev [num_layers][B][Hkv][k] to topk_host (either host pointer may be
+ * NULL to skip that copy).  Host buffers should be pinned for asynchronous
+ * copies.  Returns after enqueueing; synchronise the stream before reading
+ * the host outputs. */
+int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers,
+                           const uint8_t* policy, const void* q_host, void* q_dev,
+                           const void* const* K, const void* const* V,
+                           const int32_t* seqlens, float* out_dev, float* out_host,
+                           int32_t* topk_dev, int32_t* topk_host, void* workspace,
+                           size_t workspace_bytes, hylra_stream_t stream);
+
+/* Overlap matrix (HyLRA summary §2.2 "Similarity Matrix Construction").
+ * topk: HOST int32 [num_layers][num_sets][k] index sets from a profiling run
+ * in which every layer is a reset layer (num_sets = profiled steps x B x Hkv),
+ * -1 padded.  M: HOST double [num_layers][num_layers], row = target layer t,
+ * column = source layer s <= t: M[t][s] = sum_u |I_s(u) & I_t(u)| /
+ * sum_u |I_t(u)| (pooled overlap ratio).  Diagonal 1 (0 for a layer with no
+ * valid sets); upper triangle 0.  Synchronous. */
+int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k,
+                     const int32_t* topk, double* M);
+
+/* Policy (HyLRA summary §2.2 "Dynamic Programming").  States (i, j): layer j
+ * uses the indices of reset layer i; layer 0 is a reset.  Reset jump
+ * (i, j) -> (j+1, j+1); vertical move (i, j) -> (i, j+1) allowed when
+ * M[j+1][i] > theta (strict), adding M[j+1][i] to the cumulative similarity.
+ * Optimum: fewest resets, then largest cumulative similarity (summed in layer
+ * order), then the lexicographically smallest policy with reuse < reset.
+ * policy: HOST uint8 [num_layers] (1 = reset, 0 = reuse).  num_resets and
+ * cum_similarity may be NULL.  Synchronous. */
+int hylra_dp_policy(int32_t num_layers, const double* M, double theta,
+                    uint8_t* policy, int32_t* num_resets, double* cum_similarity);
+
+/* Copy the workspace status word to *status (synchronises the stream); when
+ * clear != 0 the word is reset to 0 afterwards. */
+int hylra_read_status(void* workspace, uint32_t* status, int clear,
+                      hylra_stream_t stream);
+
+/* Static string for a hylra_error_t value. */
+const char* hylra_strerror(int err);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int hylra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYLRA_H_ */

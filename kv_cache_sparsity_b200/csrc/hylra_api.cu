@@ -1,0 +1,336 @@
+// hylra_api.cu - C ABI entry points of the decode kernels (see include/hylra.h).
+//
+// Host side only: argument validation, workspace layout, TMA descriptor
+// encoding and kernel launches.  The kernels live in hylra_kernels.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "hylra.h"
+#include "hylra_kernels.cuh"
+
+using namespace hylra;
+
+namespace {
+
+constexpr size_t kSmemBF16 = sizeof(SmemBF16) + 1024;  // + alignment slack
+static_assert(kSmemBF16 <= 232448, "bf16 kernel shared memory exceeds 227 KB");
+
+struct Layout {
+  size_t status, tickets, partials, bstat, total;
+  int G, nbmax, nbh, nslots;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int sm_count(int* G) {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  *G = n;
+  return HYLRA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(const hylra_shape_t* s) {
+  if (!s) return HYLRA_ERR_INVALID;
+  if (s->head_dim != HYLRA_HEAD_DIM || s->block_size != HYLRA_BLOCK_TOKENS)
+    return HYLRA_ERR_UNSUPPORTED;
+  if (s->batch < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1) return HYLRA_ERR_INVALID;
+  if (s->num_q_heads % s->num_kv_heads != 0) return HYLRA_ERR_INVALID;
+  if (s->num_q_heads / s->num_kv_heads > HYLRA_MAX_GROUP) return HYLRA_ERR_UNSUPPORTED;
+  if (s->batch > HYLRA_MAX_BATCH) return HYLRA_ERR_UNSUPPORTED;
+  if (s->topk < 1) return HYLRA_ERR_INVALID;
+  if (s->topk > HYLRA_MAX_TOPK) return HYLRA_ERR_UNSUPPORTED;
+  if (s->dtype != HYLRA_BF16 && s->dtype != HYLRA_FP32) return HYLRA_ERR_INVALID;
+  if (s->max_seqlen < 0) return HYLRA_ERR_INVALID;
+  if (s->max_seqlen > HYLRA_MAX_SEQLEN) return HYLRA_ERR_UNSUPPORTED;
+  if (s->kv_capacity < 0) return HYLRA_ERR_INVALID;
+  long long rows;
+  if (s->kv_capacity > 0) {
+    if (s->kv_capacity < s->max_seqlen) return HYLRA_ERR_INVALID;
+    rows = (long long)s->batch * s->num_kv_heads * s->kv_capacity;
+  } else {
+    if (s->total_tokens < 0 || s->seq_offsets == nullptr) return HYLRA_ERR_INVALID;
+    if (!aligned(s->seq_offsets, 8)) return HYLRA_ERR_INVALID;
+    rows = (long long)s->num_kv_heads * s->total_tokens;
+  }
+  if (rows > INT_MAX - 2 * HYLRA_BLOCK_TOKENS) return HYLRA_ERR_UNSUPPORTED;
+  const long long nbmax = (s->max_seqlen + HYLRA_BLOCK_TOKENS - 1) / HYLRA_BLOCK_TOKENS;
+  if ((long long)s->batch * s->num_kv_heads * std::max(1LL, nbmax) > INT_MAX / 4)
+    return HYLRA_ERR_UNSUPPORTED;
+  return HYLRA_OK;
+}
+
+Layout make_layout(const hylra_shape_t* s, int G) {
+  Layout L{};
+  const int r = s->num_q_heads / s->num_kv_heads;
+  L.G = G;
+  L.nbmax = std::max(1, (s->max_seqlen + BLK - 1) / BLK);
+  L.nbh = s->batch * s->num_kv_heads;
+  L.nslots = G + L.nbh;
+  size_t off = 0;
+  L.status = off;
+  off += 256;
+  L.tickets = off;
+  off = align_up(off + (size_t)L.nbh * 4, 256);
+  L.partials = off;
+  off = align_up(off + (size_t)L.nslots * SLOT_FLOATS * 4, 256);
+  L.bstat = off;
+  off = align_up(off + (size_t)L.nbh * L.nbmax * 2 * r * 4, 256);
+  L.total = off;
+  return L;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [rows][128] bf16 view with 64x128 boxes and 128-byte swizzle.
+int make_tmap(CUtensorMap* tm, const void* base, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return HYLRA_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)std::max(1LL, rows)};
+  cuuint64_t strides[1] = {(cuuint64_t)HD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)BLK};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r =
+      fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HYLRA_OK : HYLRA_ERR_CUDA;
+}
+
+// Opt the bf16 kernels in to their dynamic shared memory once per device.
+int prepare_bf16_kernels() {
+  static std::mutex mu;
+  static std::vector<char> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)done.size() <= dev) done.resize(dev + 1, 0);
+  if (done[dev]) return HYLRA_OK;
+  if (cudaFuncSetAttribute(decode_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBF16) != cudaSuccess ||
+      cudaFuncSetAttribute(decode_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBF16) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  done[dev] = 1;
+  return HYLRA_OK;
+}
+
+int check_layer_ptrs(const hylra_shape_t* s, const void* q, const void* K, const void* V,
+                     const float* out) {
+  if (!q || !K || !V || !out) return HYLRA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
+    return HYLRA_ERR_INVALID;
+  (void)s;
+  return HYLRA_OK;
+}
+
+int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, const void* V,
+           const int32_t* seqlens, const int32_t* topk_in, float* out, int32_t* topk_out,
+           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if ((rc = check_layer_ptrs(s, q, K, V, out))) return rc;
+  if (!seqlens || !ws || !aligned(seqlens, 4) || !aligned(ws, 256)) return HYLRA_ERR_INVALID;
+  if (full && (!topk_out || !aligned(topk_out, 4))) return HYLRA_ERR_INVALID;
+  if (!full && (!topk_in || !aligned(topk_in, 4))) return HYLRA_ERR_INVALID;
+  int G = 0;
+  if ((rc = sm_count(&G))) return rc;
+  const Layout L = make_layout(s, G);
+  if (ws_bytes < L.total) return HYLRA_ERR_WORKSPACE;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  Params p{};
+  p.q = q;
+  p.K = K;
+  p.V = V;
+  p.seqlens = seqlens;
+  p.seq_off = s->kv_capacity > 0 ? nullptr : s->seq_offsets;
+  p.topk_in = topk_in;
+  p.out = out;
+  p.topk_out = topk_out;
+  p.status = reinterpret_cast<uint32_t*>(w + L.status);
+  p.tickets = reinterpret_cast<uint32_t*>(w + L.tickets);
+  p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.bstat = reinterpret_cast<float*>(w + L.bstat);
+  p.cap = s->kv_capacity;
+  p.total = s->kv_capacity > 0 ? 0 : s->total_tokens;
+  p.B = s->batch;
+  p.Hq = s->num_q_heads;
+  p.Hkv = s->num_kv_heads;
+  p.r = s->num_q_heads / s->num_kv_heads;
+  p.k = s->topk;
+  p.max_seqlen = s->max_seqlen;
+  p.nbmax = L.nbmax;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
+
+  if (s->dtype == HYLRA_BF16) {
+    if ((rc = prepare_bf16_kernels())) return rc;
+    const long long rows = s->kv_capacity > 0
+                               ? (long long)s->batch * s->num_kv_heads * s->kv_capacity
+                               : (long long)s->num_kv_heads * s->total_tokens;
+    CUtensorMap tmK, tmV;
+    if ((rc = make_tmap(&tmK, K, rows))) return rc;
+    if ((rc = make_tmap(&tmV, V, rows))) return rc;
+    if (full)
+      decode_bf16_kernel<true><<<G, NTHR_BF16, kSmemBF16, stream>>>(tmK, tmV, p);
+    else
+      decode_bf16_kernel<false><<<G, NTHR_BF16, kSmemBF16, stream>>>(tmK, tmV, p);
+  } else {
+    if (full)
+      decode_f32_kernel<true><<<G, NTHR_F32, 0, stream>>>(p);
+    else
+      decode_f32_kernel<false><<<G, NTHR_F32, 0, stream>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
+}
+
+size_t elem_size(const hylra_shape_t* s) { return s->dtype == HYLRA_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+int hylra_version(void) { return 100; }
+
+const char* hylra_strerror(int err) {
+  switch (err) {
+    case HYLRA_OK: return "ok";
+    case HYLRA_ERR_INVALID: return "invalid argument";
+    case HYLRA_ERR_UNSUPPORTED: return "unsupported shape or limit exceeded";
+    case HYLRA_ERR_CUDA: return "CUDA error";
+    case HYLRA_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown error";
+  }
+}
+
+int hylra_workspace_bytes(const hylra_shape_t* shape, size_t* bytes) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!bytes) return HYLRA_ERR_INVALID;
+  int G = 0;
+  if ((rc = sm_count(&G))) return rc;
+  *bytes = make_layout(shape, G).total;
+  return HYLRA_OK;
+}
+
+int hylra_workspace_init(void* workspace, size_t bytes, hylra_stream_t stream) {
+  if (!workspace) return HYLRA_ERR_INVALID;
+  return cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream) == cudaSuccess
+             ? HYLRA_OK
+             : HYLRA_ERR_CUDA;
+}
+
+int hylra_decode_full(const hylra_shape_t* shape, const void* q, const void* K, const void* V,
+                      const int32_t* seqlens, float* out, int32_t* topk_out, void* workspace,
+                      size_t workspace_bytes, hylra_stream_t stream) {
+  return launch(shape, true, q, K, V, seqlens, nullptr, out, topk_out, workspace,
+                workspace_bytes, (cudaStream_t)stream);
+}
+
+int hylra_decode_reuse(const hylra_shape_t* shape, const void* q, const void* K, const void* V,
+                       const int32_t* seqlens, const int32_t* topk_in, float* out,
+                       void* workspace, size_t workspace_bytes, hylra_stream_t stream) {
+  return launch(shape, false, q, K, V, seqlens, topk_in, out, nullptr, workspace,
+                workspace_bytes, (cudaStream_t)stream);
+}
+
+int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,
+                      const void* const* q, const void* const* K, const void* const* V,
+                      const int32_t* seqlens, float* const* out, int32_t* topk, void* workspace,
+                      size_t workspace_bytes, hylra_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (num_layers < 1 || !policy || !q || !K || !V || !out || !topk) return HYLRA_ERR_INVALID;
+  if (policy[0] != 1) return HYLRA_ERR_INVALID;
+  for (int l = 0; l < num_layers; ++l) {
+    if (policy[l] > 1) return HYLRA_ERR_INVALID;
+    if ((rc = check_layer_ptrs(shape, q[l], K[l], V[l], out[l]))) return rc;
+  }
+  const size_t per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
+  int last_reset = 0;
+  for (int l = 0; l < num_layers; ++l) {
+    if (policy[l]) {
+      last_reset = l;
+      rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
+                  workspace, workspace_bytes, (cudaStream_t)stream);
+    } else {
+      rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
+                  nullptr, workspace, workspace_bytes, (cudaStream_t)stream);
+    }
+    if (rc) return rc;
+  }
+  return HYLRA_OK;
+}
+
+int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,
+                           const void* q_host, void* q_dev, const void* const* K,
+                           const void* const* V, const int32_t* seqlens, float* out_dev,
+                           float* out_host, int32_t* topk_dev, int32_t* topk_host,
+                           void* workspace, size_t workspace_bytes, hylra_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (num_layers < 1 || !q_host || !q_dev || !out_dev || !topk_dev || !K || !V)
+    return HYLRA_ERR_INVALID;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t q_layer = (size_t)shape->batch * shape->num_q_heads * HD;
+  const size_t q_bytes = q_layer * elem_size(shape) * num_layers;
+  const size_t out_bytes = q_layer * sizeof(float) * num_layers;
+  const size_t topk_bytes =
+      (size_t)shape->batch * shape->num_kv_heads * shape->topk * sizeof(int32_t) * num_layers;
+  std::vector<const void*> qp(num_layers);
+  std::vector<float*> op(num_layers);
+  for (int l = 0; l < num_layers; ++l) {
+    qp[l] = static_cast<const uint8_t*>(q_dev) + l * q_layer * elem_size(shape);
+    op[l] = out_dev + l * q_layer;
+  }
+  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  rc = hylra_decode_step(shape, num_layers, policy, qp.data(), K, V, seqlens, op.data(), topk_dev,
+                         workspace, workspace_bytes, stream);
+  if (rc) return rc;
+  if (out_host &&
+      cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  if (topk_host &&
+      cudaMemcpyAsync(topk_host, topk_dev, topk_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return HYLRA_OK;
+}
+
+int hylra_read_status(void* workspace, uint32_t* status, int clear, hylra_stream_t stream) {
+  if (!workspace || !status) return HYLRA_ERR_INVALID;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HYLRA_ERR_CUDA;
+  *status = v;
+  if (clear && cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return HYLRA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,926 @@
+// hylra_kernels.cuh - HyLRA decode-attention kernels for sm_100a.
+//
+// "HyLRA: Hybrid Layer Reuse Attention for Efficient Long-Context Inference"
+// (gist.science technical summary of arXiv 2602.00777):
+//   §2.3 Hybrid Inference Strategy - reset layers: full attention + top-k
+//        extraction; reuse layers: attention restricted to the reused subset.
+//   §2.4 Block-level Sparsity - 128-token blocks, regular coalesced access.
+//
+// Design (one persistent CTA per SM, static "stream-K" split of the work):
+//   * A unit of work is one 128-token block of one (sequence b, KV head h):
+//     every block of the cache on a reset layer, the k' reused blocks on a
+//     reuse layer.  Units are laid out (b, h, j)-major and CTA c takes the
+//     contiguous range [c*T/G, (c+1)*T/G), so the load is balanced to one
+//     block whatever the batch raggedness.  A CTA's range crosses (b, h)
+//     boundaries; each maximal run of one (b, h) is a "segment".
+//   * bf16 kernel: warp 0 issues TMA tile loads (128-byte swizzle, L2
+//     evict-first) of K and V blocks (64 KB per stage, 3 stages) plus the
+//     GQA group's q rows into shared memory; four consumer warps take 32
+//     tokens each.  Q.K^T runs as S^T = K Q^T on bf16 mma.sync (M = tokens,
+//     N = the r <= 8 q-heads), the softmax is online in the log2 domain with
+//     an fp32 running max and sum per warp, P^T moves from the accumulator
+//     layout to the B-operand layout with movmatrix, and O^T = V^T P^T
+//     accumulates in fp32 registers.
+//   * Reset layers also record, per block and q-head, the block's local max
+//     and probability sum (relative to that max): the exact ingredients of
+//     the block's attention mass once the global max and sum are known.
+//   * At a segment end the four warps' states are merged (LSE) into a partial
+//     in the workspace; the last CTA to finish a (b, h) (an atomic ticket, no
+//     spinning) merges all partials into the output and, on reset layers,
+//     turns the block records into fp32 block masses and selects the top-k
+//     (radix select on the fp32 bit patterns, index order among equals).
+//   * fp32 inputs (small cases) take a CUDA-core kernel with the same work
+//     split, block records, merge and selection.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "hylra.h"
+#include "hylra_device.cuh"
+
+namespace hylra {
+
+constexpr int BLK = HYLRA_BLOCK_TOKENS;  // tokens per block
+constexpr int HD = HYLRA_HEAD_DIM;       // head dimension
+constexpr int GMAX = HYLRA_MAX_GROUP;    // q-heads per KV head, padded MMA N
+constexpr int NCW = 4;                   // consumer warps
+constexpr int NCONS = NCW * 32;          // consumer threads
+constexpr int NTHR_BF16 = NCONS + 32;    // + one producer warp
+constexpr int NTHR_F32 = NCONS;
+constexpr int NSTAGE = 3;
+constexpr int BOX_BYTES = 64 * 2 * BLK;       // 64 bf16 columns x 128 rows
+constexpr int STAGE_BYTES = 4 * BOX_BYTES;    // K[:, 0:64], K[:, 64:128], V.., V..
+constexpr int QSLOT_BYTES = GMAX * HD * 2;
+constexpr int SLOT_FLOATS = GMAX * HD + 2 * GMAX;  // partial: O[8][128], m[8], Z[8]
+constexpr int MAX_NB = HYLRA_MAX_SEQLEN / BLK;
+constexpr int BAR_CONS = 1;  // named barrier of the consumer threads
+
+struct Params {
+  const void* q;
+  const void* K;  // read directly by the fp32 kernel
+  const void* V;
+  const int32_t* seqlens;
+  const int64_t* seq_off;
+  const int32_t* topk_in;
+  float* out;
+  int32_t* topk_out;
+  uint32_t* status;
+  uint32_t* tickets;
+  float* partials;
+  float* bstat;
+  long long cap;    // dense rows per (b, h) plane; 0 = packed layout
+  long long total;  // packed rows per KV-head plane
+  int B, Hq, Hkv, r, k, max_seqlen, nbmax;
+  float scale_log2;  // log2(e) / sqrt(d)
+};
+
+struct StageMeta {
+  int b, h, blk, nvalid, flags, seg_slot, first_slot, ncontrib, nb, pad0, pad1, pad2;
+};
+constexpr int F_SEG_START = 1;
+constexpr int F_SEG_END = 2;
+
+// A stage description only ever comes from describe_unit; this re-checks the
+// fields that address global memory so that a consumer that gave up waiting
+// (HYLRA_STATUS_TIMEOUT) can never write out of bounds.
+__device__ __forceinline__ bool meta_sane(const Params& p, const StageMeta& m) {
+  const int nslots = (int)gridDim.x + p.B * p.Hkv;
+  return m.b >= 0 && m.b < p.B && m.h >= 0 && m.h < p.Hkv && m.blk < p.nbmax && m.nb >= 0 &&
+         m.nb <= p.nbmax && m.seg_slot >= 0 && m.seg_slot < nslots && m.first_slot >= 0 &&
+         m.ncontrib >= 1 && m.first_slot + m.ncontrib <= nslots && m.nvalid <= BLK;
+}
+
+struct SmemCommon {
+  float comb_o[NCW][GMAX][HD];  // per-warp O at a segment end; top-k scratch in a merge
+  float comb_m[NCW][GMAX];
+  float comb_z[NCW][GMAX];
+  float mg[GMAX];
+  float zg[GMAX];
+  int prefix[HYLRA_MAX_BATCH + 1];  // units before sequence b (all heads)
+  int hist[256];
+  int misc[8];  // 0: last-CTA flag, 1: radix digit, 2: remaining, 3: list size, 4: abort
+  int warp_sums[NCW];
+};
+static_assert(sizeof(float) * NCW * GMAX * HD >= MAX_NB * 4 + HYLRA_MAX_TOPK * 8,
+              "top-k scratch must fit in the combine buffer");
+
+struct SmemBF16 {
+  uint8_t stage[NSTAGE][STAGE_BYTES];  // 1024-byte aligned (128-byte swizzle atoms)
+  uint8_t qslot[NSTAGE][QSLOT_BYTES];
+  float bst_s[NSTAGE][NCW][GMAX];
+  float bst_m[NSTAGE][NCW][GMAX];
+  int bst_cnt[NSTAGE];
+  StageMeta meta[NSTAGE];
+  alignas(8) uint64_t full_bar[NSTAGE];
+  alignas(8) uint64_t empty_bar[NSTAGE];
+  SmemCommon c;
+};
+
+struct SmemF32 {
+  float qs[GMAX][HD];
+  float bst_s[2][NCW][GMAX];
+  float bst_m[2][NCW][GMAX];
+  SmemCommon c;
+};
+
+// ------------------------------------------------------------ work layout
+
+// Sequence length after validation; an invalid length counts as empty.
+__device__ __forceinline__ int valid_seqlen(const Params& p, int b, bool report) {
+  const int n = p.seqlens[b];
+  bool bad = n < 0 || n > p.max_seqlen;
+  if (!bad) {
+    if (p.cap > 0) {
+      bad = (long long)n > p.cap;
+    } else {
+      const long long o = p.seq_off[b];
+      bad = o < 0 || o + n > p.total;
+    }
+  }
+  if (bad) {
+    if (report) atomicOr(p.status, HYLRA_STATUS_BAD_SEQLEN);
+    return 0;
+  }
+  return n;
+}
+
+__device__ __forceinline__ int units_of(const Params& p, int n, bool full) {
+  const int nb = (n + BLK - 1) / BLK;
+  return full ? nb : min(p.k, nb);
+}
+
+// First row of (b, h) in the 2-D [rows][d] view of K or V.
+__device__ __forceinline__ long long row_base(const Params& p, int b, int h) {
+  return p.cap > 0 ? ((long long)b * p.Hkv + h) * p.cap : (long long)h * p.total + p.seq_off[b];
+}
+
+// CTA that owns linear unit u when CTA c holds [floor(c*T/G), floor((c+1)*T/G));
+// with G <= T every such range is non-empty.
+__device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
+  return (int)(((u + 1) * G - 1) / T);
+}
+
+// prefix[b] = number of units of sequences 0..b-1 (all KV heads); warp 0.
+__device__ void build_prefix(const Params& p, SmemCommon& c, bool full) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const int per = (p.B + 31) / 32;
+  const int b0 = min(p.B, lane * per), b1 = min(p.B, b0 + per);
+  int local = 0;
+  for (int b = b0; b < b1; ++b)
+    local += units_of(p, valid_seqlen(p, b, blockIdx.x == 0), full) * p.Hkv;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  int run = incl - local;
+  for (int b = b0; b < b1; ++b) {
+    c.prefix[b] = run;
+    run += units_of(p, valid_seqlen(p, b, false), full) * p.Hkv;
+  }
+  if (lane == 31) c.prefix[p.B] = incl;
+}
+
+// Sequences without units still need an output: zeros (and -1 indices).
+template <bool FULL>
+__device__ void write_empty_outputs(const Params& p, const SmemCommon& c) {
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    if (c.prefix[b + 1] != c.prefix[b]) continue;
+    float* o = p.out + (size_t)b * p.Hq * HD;
+    for (int i = threadIdx.x; i < p.Hq * HD; i += blockDim.x) o[i] = 0.f;
+    if (FULL) {
+      int32_t* t = p.topk_out + (size_t)b * p.Hkv * p.k;
+      for (int i = threadIdx.x; i < p.Hkv * p.k; i += blockDim.x) t[i] = -1;
+    }
+  }
+}
+
+// Walks units (b, h, j) in linear order.
+struct UnitIter {
+  int b, h, j, U;
+  __device__ void seek(const SmemCommon& c, const Params& p, int u) {
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (c.prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    U = (c.prefix[b + 1] - c.prefix[b]) / p.Hkv;
+    const int off = u - c.prefix[b];
+    h = off / U;
+    j = off - h * U;
+  }
+  __device__ void advance(const SmemCommon& c, const Params& p) {
+    if (++j < U) return;
+    j = 0;
+    if (++h < p.Hkv) return;
+    h = 0;
+    do { ++b; } while (b < p.B && c.prefix[b + 1] == c.prefix[b]);
+    if (b < p.B) U = (c.prefix[b + 1] - c.prefix[b]) / p.Hkv;
+  }
+};
+
+// Everything a unit needs besides its data.
+template <bool FULL>
+__device__ __forceinline__ StageMeta describe_unit(const Params& p, const SmemCommon& c,
+                                                   const UnitIter& it, int i, int n, int T,
+                                                   int G, bool report) {
+  StageMeta m;
+  const int bh = it.b * p.Hkv + it.h;
+  const int seqlen = valid_seqlen(p, it.b, false);
+  const int nb = (seqlen + BLK - 1) / BLK;
+  int blk;
+  if (FULL) {
+    blk = it.j;
+  } else {
+    blk = p.topk_in[(size_t)bh * p.k + it.j];
+    if (blk < 0 || blk >= nb) {
+      if (blk != -1 && report) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
+      blk = -1;
+    }
+  }
+  const int start = c.prefix[it.b] + it.h * it.U;
+  const int cf = owner_cta(start, T, G);
+  const int cl = owner_cta((long long)start + it.U - 1, T, G);
+  m.b = it.b;
+  m.h = it.h;
+  m.blk = blk;
+  m.nvalid = blk >= 0 ? min(BLK, seqlen - blk * BLK) : 0;
+  m.flags = ((i == 0 || it.j == 0) ? F_SEG_START : 0) | ((i == n - 1 || it.j == it.U - 1) ? F_SEG_END : 0);
+  m.seg_slot = (int)blockIdx.x + bh;
+  m.first_slot = cf + bh;
+  m.ncontrib = cl - cf + 1;
+  m.nb = nb;
+  m.pad0 = m.pad1 = m.pad2 = 0;
+  return m;
+}
+
+// ------------------------------------------------------------------ top-k
+
+// Top-k of the block scores keys[0..nb) (fp32 bit patterns of non-negative
+// scores, so unsigned order is numeric order): rank order, score descending,
+// lower block index first among equal scores; slots k'..k-1 get -1.
+// Called by the NCONS consumer threads (ct = 0..NCONS-1).
+__device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int ct) {
+  uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
+  uint2* list = reinterpret_cast<uint2*>(reinterpret_cast<char*>(&c.comb_o[0][0][0]) + MAX_NB * 4);
+  int32_t* dst = p.topk_out + (size_t)bh * p.k;
+  const int kp = min(p.k, nb);
+  const int lane = ct & 31, wid = ct >> 5;
+
+  // Radix select of the kp-th largest key, 8 bits per pass.
+  uint32_t prefix = 0;
+  int remain = kp;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    c.hist[ct] = 0;
+    c.hist[ct + NCONS] = 0;
+    if (ct == 0) c.misc[3] = 0;
+    named_bar_sync(BAR_CONS, NCONS);
+    for (int beta = ct; beta < nb; beta += NCONS) {
+      const uint32_t key = keys[beta];
+      const bool match = pass == 0 || ((key ^ prefix) >> (shift + 8)) == 0u;
+      if (match) atomicAdd(&c.hist[(key >> shift) & 255u], 1);
+    }
+    named_bar_sync(BAR_CONS, NCONS);
+    if (wid == 0) {
+      int cnt[8];
+      int local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = c.hist[255 - 8 * lane - i];
+        local += cnt[i];
+      }
+      int incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const int excl = incl - local;
+      if (excl < remain && remain <= incl) {
+        int acc = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (acc + cnt[i] >= remain) {
+            c.misc[1] = 255 - 8 * lane - i;
+            c.misc[2] = remain - acc;
+            break;
+          }
+          acc += cnt[i];
+        }
+      }
+    }
+    named_bar_sync(BAR_CONS, NCONS);
+    prefix |= (uint32_t)c.misc[1] << shift;
+    remain = c.misc[2];
+  }
+  const uint32_t tau = prefix;  // the kp-th largest score; take `remain` of its copies
+
+  // Keep every key above tau and the lowest-index `remain` keys equal to it.
+  const int per = (nb + NCONS - 1) / NCONS;
+  const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
+  int eq = 0;
+  for (int beta = b0; beta < b1; ++beta) eq += keys[beta] == tau;
+  int incl = eq;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) c.warp_sums[wid] = incl;
+  named_bar_sync(BAR_CONS, NCONS);
+  int before = incl - eq;
+  for (int w = 0; w < wid; ++w) before += c.warp_sums[w];
+  for (int beta = b0; beta < b1; ++beta) {
+    const uint32_t key = keys[beta];
+    bool sel = key > tau;
+    if (key == tau) {
+      sel = before < remain;
+      ++before;
+    }
+    if (sel) {
+      const int pos = atomicAdd(&c.misc[3], 1);
+      if (pos < kp) list[pos] = make_uint2(key, (uint32_t)beta);  // exactly kp are selected
+    }
+  }
+  named_bar_sync(BAR_CONS, NCONS);
+  for (int e = ct; e < kp; e += NCONS) {
+    const uint2 me = list[e];
+    int rank = 0;
+    for (int j = 0; j < kp; ++j) {
+      const uint2 o = list[j];
+      rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+    }
+    dst[rank] = (int32_t)me.y;
+  }
+  for (int slot = kp + ct; slot < p.k; slot += NCONS) dst[slot] = -1;
+}
+
+// ---------------------------------------------------------------- merging
+
+// The last CTA of (b, h): LSE-merge every contributor's partial into out;
+// on reset layers also score the blocks and select the top-k.
+template <bool FULL>
+__device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
+  const int bh = m.b * p.Hkv + m.h;
+  const int d = ct;
+  for (int g = 0; g < p.r; ++g) {
+    float M = -INFINITY;
+    for (int j = 0; j < m.ncontrib; ++j)
+      M = fmaxf(M, __ldcg(p.partials + (size_t)(m.first_slot + j) * SLOT_FLOATS + GMAX * HD + g));
+    float Z = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int j = 0; j < m.ncontrib; ++j) {
+        const float* sl = p.partials + (size_t)(m.first_slot + j) * SLOT_FLOATS;
+        const float mj = __ldcg(sl + GMAX * HD + g);
+        if (mj == -INFINITY) continue;
+        const float f = exp2f(mj - M);
+        Z += __ldcg(sl + GMAX * HD + GMAX + g) * f;
+        O += __ldcg(sl + g * HD + d) * f;
+      }
+    }
+    p.out[((size_t)m.b * p.Hq + (size_t)m.h * p.r + g) * HD + d] = Z > 0.f ? O / Z : 0.f;
+    if (ct == 0) {
+      c.mg[g] = M;
+      c.zg[g] = Z;
+    }
+  }
+  if (FULL) {
+    named_bar_sync(BAR_CONS, NCONS);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
+    bool nonfinite = false;
+    for (int beta = ct; beta < m.nb; beta += NCONS) {
+      const float* bs = p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * p.r);
+      float score = 0.f;
+      for (int g = 0; g < p.r; ++g) {
+        const float s = __ldcg(bs + 2 * g), mb = __ldcg(bs + 2 * g + 1);
+        if (c.zg[g] > 0.f && mb != -INFINITY) score += s * exp2f(mb - c.mg[g]) / c.zg[g];
+      }
+      uint32_t key = 0u;
+      if (isfinite(score)) {
+        if (score > 0.f) key = __float_as_uint(score);
+      } else {
+        nonfinite = true;
+      }
+      keys[beta] = key;
+    }
+    if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
+    named_bar_sync(BAR_CONS, NCONS);
+    topk_select(p, c, bh, m.nb, ct);
+  }
+  if (!FULL) {
+    // a reused list naming one block twice counts that block twice: flag it
+    const int kp = min(p.k, m.nb);
+    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+    bool dup = false;
+    for (int e = ct; e < kp; e += NCONS) {
+      const int32_t v = idx[e];
+      if (v < 0) continue;
+      for (int j = 0; j < e; ++j) dup |= idx[j] == v;
+    }
+    if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
+  }
+  if (ct == 0) p.tickets[bh] = 0u;  // ready for the next launch
+  named_bar_sync(BAR_CONS, NCONS);
+}
+
+// Segment end: comb_* hold the NCW warps' (m, Z, O).  Merge them into this
+// CTA's partial, publish it, and merge (b, h) if this CTA finished it last.
+template <bool FULL>
+__device__ void publish_segment(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
+  const int d = ct;
+  const bool sane = meta_sane(p, m);
+  float* slot = p.partials + (size_t)(sane ? m.seg_slot : 0) * SLOT_FLOATS;
+  for (int g = 0; g < p.r && sane; ++g) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) M = fmaxf(M, c.comb_m[w][g]);
+    float O = 0.f, Z = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float mw = c.comb_m[w][g];
+        if (mw == -INFINITY) continue;
+        const float f = exp2f(mw - M);
+        O += c.comb_o[w][g][d] * f;
+        Z += c.comb_z[w][g] * f;
+      }
+    }
+    slot[g * HD + d] = O;
+    if (d == 0) {
+      slot[GMAX * HD + g] = M;
+      slot[GMAX * HD + GMAX + g] = Z;
+    }
+  }
+  __threadfence();
+  named_bar_sync(BAR_CONS, NCONS);
+  if (ct == 0) {
+    c.misc[0] = 0;
+    if (sane) {
+      const uint32_t old = atomic_add_acq_rel_gpu(p.tickets + m.b * p.Hkv + m.h, 1u);
+      c.misc[0] = (old == (uint32_t)(m.ncontrib - 1)) ? 1 : 0;
+    }
+  }
+  named_bar_sync(BAR_CONS, NCONS);
+  if (c.misc[0]) {
+    __threadfence();
+    merge_bh<FULL>(p, c, m, ct);
+  }
+}
+
+// Block record (local max, sum relative to it) of the NCW warps' shares of a
+// block, for head g: one (sum, max) pair relative to the block's own max.
+__device__ __forceinline__ void combine_block_record(const float (*bs)[GMAX],
+                                                     const float (*bm)[GMAX], int g, float* dst) {
+  float mm = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, bm[w][g]);
+  float ss = 0.f;
+  if (mm != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+      const float mw = bm[w][g];
+      if (mw != -INFINITY) ss += bs[w][g] * exp2f(mw - mm);
+    }
+  }
+  dst[0] = ss;
+  dst[1] = mm;
+}
+
+// ------------------------------------------------------------ bf16 kernel
+
+template <bool FULL>
+__global__ void __launch_bounds__(NTHR_BF16, 1)
+    decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemBF16& sm = *reinterpret_cast<SmemBF16*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  SmemCommon& c = sm.c;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&sm.full_bar[s], 1);
+      mbar_init(&sm.empty_bar[s], NCW);
+      sm.bst_cnt[s] = 0;
+      StageMeta z{};
+      z.blk = -1;
+      z.ncontrib = 1;
+      sm.meta[s] = z;
+    }
+    c.misc[4] = 0;
+    fence_mbar_init();
+  }
+  if (tid == 32) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  build_prefix(p, c, FULL);
+  __syncthreads();
+  // Work split over G = min(grid, T) CTAs so that every working CTA owns at
+  // least one unit (the contributor count of a (b, h) relies on it).
+  const int T = c.prefix[p.B];
+  const int G = T > 0 ? min((int)gridDim.x, T) : 1;
+  const bool works = (int)blockIdx.x < G;
+  const int lo = works ? (int)((long long)blockIdx.x * T / G) : 0;
+  const int hi = works ? (int)((long long)(blockIdx.x + 1) * T / G) : 0;
+  const int n = hi - lo;
+  write_empty_outputs<FULL>(p, c);
+  volatile int* abort_flag = &c.misc[4];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0 || n <= 0) return;
+    UnitIter it;
+    it.seek(c, p, lo);
+    const uint64_t pol = l2_evict_first_policy();
+    const uint8_t* qbase = static_cast<const uint8_t*>(p.q);
+    const uint32_t qbytes = (uint32_t)(p.r * HD * 2);
+    for (int i = 0; i < n; ++i) {
+      const int s = i % NSTAGE;
+      const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
+      mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
+      const StageMeta m = describe_unit<FULL>(p, c, it, i, n, T, G, true);
+      sm.meta[s] = m;
+      const bool seg_start = (m.flags & F_SEG_START) != 0;
+      uint32_t bytes = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? (uint32_t)STAGE_BYTES : 0u);
+      if (*abort_flag) bytes = 0;
+      if (bytes) {
+        mbar_arrive_expect_tx(&sm.full_bar[s], bytes);
+        if (seg_start)
+          bulk_load(sm.qslot[s], qbase + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD * 2, qbytes,
+                    &sm.full_bar[s]);
+        if (m.blk >= 0) {
+          const int row = (int)(row_base(p, m.b, m.h) + (long long)m.blk * BLK);
+          uint8_t* st = sm.stage[s];
+          tma_load_2d(st, &tmK, 0, row, &sm.full_bar[s], pol);
+          tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.full_bar[s], pol);
+          tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.full_bar[s], pol);
+          tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.full_bar[s], pol);
+        }
+      } else {
+        mbar_arrive(&sm.full_bar[s]);
+      }
+      it.advance(c, p);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;
+  const int ct = tid - 32;
+  const int g4 = lane >> 2, c4 = lane & 3;
+  float o[8][4];
+  float m_run[2], z_run[2];
+  uint32_t qf[8][2];
+#pragma unroll
+  for (int dm = 0; dm < 8; ++dm)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[dm][e] = 0.f;
+  m_run[0] = m_run[1] = -INFINITY;
+  z_run[0] = z_run[1] = 0.f;
+#pragma unroll
+  for (int kt = 0; kt < 8; ++kt) qf[kt][0] = qf[kt][1] = 0u;
+
+  for (int i = 0; i < n; ++i) {
+    const int s = i % NSTAGE;
+    const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
+    mbar_wait_bounded(&sm.full_bar[s], ph, abort_flag);
+    const StageMeta m = sm.meta[s];
+    if (m.flags & F_SEG_START) {
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[dm][e] = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      z_run[0] = z_run[1] = 0.f;
+      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm.qslot[s]);
+#pragma unroll
+      for (int kt = 0; kt < 8; ++kt) {
+        // B operand of S^T = K Q^T: (k = d pair 2*c4 [+8], n = q-head g4)
+        qf[kt][0] = g4 < p.r ? qs[(g4 * HD + kt * 16 + 2 * c4) >> 1] : 0u;
+        qf[kt][1] = g4 < p.r ? qs[(g4 * HD + kt * 16 + 8 + 2 * c4) >> 1] : 0u;
+      }
+    }
+    if (m.blk >= 0) {
+      const uint32_t kbase = smem_u32(sm.stage[s]);
+      const uint32_t vbase = kbase + 2 * BOX_BYTES;
+      const int tokw = cw * 32;
+      const bool partial = m.nvalid < BLK;
+      float x[2][4];
+      // ---- S^T = K Q^T for this warp's 32 tokens (two m16 tiles)
+      {
+        float acc[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt) {
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const int row = tokw + mt * 16 + (lane & 7) + (mi & 1) * 8;
+            const int ch = 2 * kt + (mi >> 1);
+            const uint32_t addr =
+                kbase + (ch >> 3) * BOX_BYTES + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, qf[kt][0], qf[kt][1]);
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = acc[mt][e] * p.scale_log2;
+            if (partial) {
+              const int tok = tokw + mt * 16 + g4 + ((e & 2) ? 8 : 0);
+              if (tok >= m.nvalid) v = -INFINITY;
+            }
+            x[mt][e] = v;
+          }
+      }
+      if (partial) {
+        // rows past the sequence end may hold anything (even NaN): zero V
+        for (int idx = lane; idx < 32 * 16; idx += 32) {
+          const int row = tokw + (idx >> 4);
+          if (row < m.nvalid) continue;
+          const int ch = idx & 15;
+          uint8_t* ptr = sm.stage[s] + 2 * BOX_BYTES + (ch >> 3) * BOX_BYTES + row * 128 + (ch & 7) * 16;
+          *reinterpret_cast<uint4*>(ptr) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      // ---- block-local max and sums for heads 2*c4 (A) and 2*c4+1 (B)
+      float mxA = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+      float mxB = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, off));
+        mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, off));
+      }
+      const float msA = mxA == -INFINITY ? 0.f : mxA;
+      const float msB = mxB == -INFINITY ? 0.f : mxB;
+      float pr[2][4];
+      float sA = 0.f, sB = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        pr[mt][0] = ex2_approx(x[mt][0] - msA);
+        pr[mt][1] = ex2_approx(x[mt][1] - msB);
+        pr[mt][2] = ex2_approx(x[mt][2] - msA);
+        pr[mt][3] = ex2_approx(x[mt][3] - msB);
+        sA += pr[mt][0] + pr[mt][2];
+        sB += pr[mt][1] + pr[mt][3];
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        sA += __shfl_xor_sync(0xffffffffu, sA, off);
+        sB += __shfl_xor_sync(0xffffffffu, sB, off);
+      }
+      if (FULL && g4 == 0) {
+        sm.bst_s[s][cw][2 * c4] = sA;
+        sm.bst_s[s][cw][2 * c4 + 1] = sB;
+        sm.bst_m[s][cw][2 * c4] = mxA;
+        sm.bst_m[s][cw][2 * c4 + 1] = mxB;
+      }
+      // ---- online softmax update
+      const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
+      float alA = 1.f, beA = 0.f, alB = 1.f, beB = 0.f;
+      if (mnA != -INFINITY) {
+        alA = ex2_approx(m_run[0] - mnA);
+        beA = ex2_approx(mxA - mnA);
+      }
+      if (mnB != -INFINITY) {
+        alB = ex2_approx(m_run[1] - mnB);
+        beB = ex2_approx(mxB - mnB);
+      }
+      z_run[0] = z_run[0] * alA + sA * beA;
+      z_run[1] = z_run[1] * alB + sB * beB;
+      m_run[0] = mnA;
+      m_run[1] = mnB;
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        o[dm][0] *= alA;
+        o[dm][1] *= alB;
+        o[dm][2] *= alA;
+        o[dm][3] *= alB;
+      }
+      // ---- P^T to the B-operand layout, then O^T += V^T P^T
+      uint32_t pb[2][2];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        pb[mt][0] = movmatrix_trans(pack_bf16x2(pr[mt][0] * beA, pr[mt][1] * beB));
+        pb[mt][1] = movmatrix_trans(pack_bf16x2(pr[mt][2] * beA, pr[mt][3] * beB));
+      }
+      const int mi = lane >> 3;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int dm = 0; dm < 8; ++dm) {
+          const int row = tokw + mt * 16 + (lane & 7) + (mi >> 1) * 8;
+          const int ch = 2 * dm + (mi & 1);
+          const uint32_t addr =
+              vbase + (ch >> 3) * BOX_BYTES + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(addr, a0, a1, a2, a3);
+          mma_bf16_16816(o[dm], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+        }
+      }
+    }
+    if (FULL && m.blk >= 0) {
+      // the last warp to finish this block merges the four shares
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(&sm.bst_cnt[s], 1) == NCW - 1;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence_block();
+        if (lane < p.r && meta_sane(p, m)) {
+          float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
+          float rec[2];
+          combine_block_record(sm.bst_s[s], sm.bst_m[s], lane, rec);
+          dst[0] = rec[0];
+          dst[1] = rec[1];
+        }
+        if (lane == 0) sm.bst_cnt[s] = 0;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
+
+    if (m.flags & F_SEG_END) {
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        const int d0 = dm * 16 + g4;
+        c.comb_o[cw][2 * c4][d0] = o[dm][0];
+        c.comb_o[cw][2 * c4 + 1][d0] = o[dm][1];
+        c.comb_o[cw][2 * c4][d0 + 8] = o[dm][2];
+        c.comb_o[cw][2 * c4 + 1][d0 + 8] = o[dm][3];
+      }
+      if (g4 == 0) {
+        c.comb_m[cw][2 * c4] = m_run[0];
+        c.comb_m[cw][2 * c4 + 1] = m_run[1];
+        c.comb_z[cw][2 * c4] = z_run[0];
+        c.comb_z[cw][2 * c4 + 1] = z_run[1];
+      }
+      named_bar_sync(BAR_CONS, NCONS);
+      publish_segment<FULL>(p, c, m, ct);
+    }
+  }
+  if (*abort_flag && ct == 0) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------ fp32 kernel
+
+template <bool FULL>
+__global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_constant__ Params p) {
+  __shared__ SmemF32 sm;
+  SmemCommon& c = sm.c;
+  const int ct = threadIdx.x, cw = ct >> 5, lane = ct & 31;
+  build_prefix(p, c, FULL);
+  __syncthreads();
+  // Work split over G = min(grid, T) CTAs so that every working CTA owns at
+  // least one unit (the contributor count of a (b, h) relies on it).
+  const int T = c.prefix[p.B];
+  const int G = T > 0 ? min((int)gridDim.x, T) : 1;
+  const bool works = (int)blockIdx.x < G;
+  const int lo = works ? (int)((long long)blockIdx.x * T / G) : 0;
+  const int hi = works ? (int)((long long)(blockIdx.x + 1) * T / G) : 0;
+  const int n = hi - lo;
+  write_empty_outputs<FULL>(p, c);
+  if (n <= 0) return;
+
+  const float* Kf = static_cast<const float*>(p.K);
+  const float* Vf = static_cast<const float*>(p.V);
+  float o[GMAX][4], m_run[GMAX], z_run[GMAX];
+  UnitIter it;
+  it.seek(c, p, lo);
+  for (int i = 0; i < n; ++i) {
+    const StageMeta m = describe_unit<FULL>(p, c, it, i, n, T, G, ct == 0);
+    it.advance(c, p);
+    if (m.flags & F_SEG_START) {
+      const float* qg = static_cast<const float*>(p.q) + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD;
+      for (int e = ct; e < p.r * HD; e += NTHR_F32) sm.qs[e / HD][e % HD] = qg[e];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        m_run[g] = -INFINITY;
+        z_run[g] = 0.f;
+        o[g][0] = o[g][1] = o[g][2] = o[g][3] = 0.f;
+      }
+      named_bar_sync(BAR_CONS, NCONS);
+    }
+    if (m.blk >= 0) {
+      const long long row0 = row_base(p, m.b, m.h) + (long long)m.blk * BLK + cw * 32;
+      const int t = cw * 32 + lane;
+      const bool valid = t < m.nvalid;
+      float acc[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) acc[g] = 0.f;
+      if (valid) {
+        const float4* kr = reinterpret_cast<const float4*>(Kf + (size_t)(row0 + lane) * HD);
+        for (int d4 = 0; d4 < HD / 4; ++d4) {
+          const float4 kv = kr[d4];
+#pragma unroll
+          for (int g = 0; g < GMAX; ++g) {
+            if (g < p.r) {
+              acc[g] = fmaf(kv.x, sm.qs[g][4 * d4], acc[g]);
+              acc[g] = fmaf(kv.y, sm.qs[g][4 * d4 + 1], acc[g]);
+              acc[g] = fmaf(kv.z, sm.qs[g][4 * d4 + 2], acc[g]);
+              acc[g] = fmaf(kv.w, sm.qs[g][4 * d4 + 3], acc[g]);
+            }
+          }
+        }
+      }
+      float pr[GMAX], be[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (g >= p.r) {
+          pr[g] = 0.f;
+          be[g] = 0.f;
+          continue;
+        }
+        const float xg = valid ? acc[g] * p.scale_log2 : -INFINITY;
+        float mx = xg;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float ms = mx == -INFINITY ? 0.f : mx;
+        const float pv = ex2_approx(xg - ms);
+        float sum = pv;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (FULL && lane == 0) {
+          sm.bst_s[i & 1][cw][g] = sum;
+          sm.bst_m[i & 1][cw][g] = mx;
+        }
+        const float mn = fmaxf(m_run[g], mx);
+        float al = 1.f, b = 0.f;
+        if (mn != -INFINITY) {
+          al = ex2_approx(m_run[g] - mn);
+          b = ex2_approx(mx - mn);
+        }
+        z_run[g] = z_run[g] * al + sum * b;
+        m_run[g] = mn;
+        o[g][0] *= al;
+        o[g][1] *= al;
+        o[g][2] *= al;
+        o[g][3] *= al;
+        pr[g] = pv * b;
+        be[g] = b;
+      }
+      const int nv = max(0, min(32, m.nvalid - cw * 32));
+      for (int tt = 0; tt < nv; ++tt) {
+        const float4 v = reinterpret_cast<const float4*>(Vf + (size_t)(row0 + tt) * HD)[lane];
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          if (g < p.r) {
+            const float pt = __shfl_sync(0xffffffffu, pr[g], tt);
+            o[g][0] = fmaf(pt, v.x, o[g][0]);
+            o[g][1] = fmaf(pt, v.y, o[g][1]);
+            o[g][2] = fmaf(pt, v.z, o[g][2]);
+            o[g][3] = fmaf(pt, v.w, o[g][3]);
+          }
+        }
+      }
+      (void)be;
+    }
+    if (FULL && m.blk >= 0) {
+      named_bar_sync(BAR_CONS, NCONS);
+      if (cw == 0 && lane < p.r && meta_sane(p, m)) {
+        float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
+        float rec[2];
+        combine_block_record(sm.bst_s[i & 1], sm.bst_m[i & 1], lane, rec);
+        dst[0] = rec[0];
+        dst[1] = rec[1];
+      }
+    }
+    if (m.flags & F_SEG_END) {
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (g < p.r) {
+          c.comb_o[cw][g][lane * 4 + 0] = o[g][0];
+          c.comb_o[cw][g][lane * 4 + 1] = o[g][1];
+          c.comb_o[cw][g][lane * 4 + 2] = o[g][2];
+          c.comb_o[cw][g][lane * 4 + 3] = o[g][3];
+          if (lane == 0) {
+            c.comb_m[cw][g] = m_run[g];
+            c.comb_z[cw][g] = z_run[g];
+          }
+        }
+      }
+      named_bar_sync(BAR_CONS, NCONS);
+      publish_segment<FULL>(p, c, m, ct);
+    }
+  }
+}
+
+}  // namespace hylra

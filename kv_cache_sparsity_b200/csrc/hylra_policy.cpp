@@ -1,0 +1,149 @@
+// hylra_policy.cpp - offline policy of HyLRA on the host (see include/hylra.h).
+//
+// "HyLRA: Hybrid Layer Reuse Attention for Efficient Long-Context Inference"
+// (gist.science technical summary of arXiv 2602.00777), §2.2 "Offline Policy
+// Optimization via Dynamic Programming":
+//   * the overlap matrix M of top-k indices between a source and a target
+//     layer (lower-triangular), from a profiling run with every layer full;
+//   * the policy: a path over states (i, j) - layer j reuses the indices of
+//     reset layer i - with reset jumps (j, j) and vertical moves (i, j) ->
+//     (i, j+1) allowed while the similarity exceeds theta; fewest full
+//     attention layers first, then the largest cumulative similarity.
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "hylra.h"
+
+namespace {
+
+// Sorted distinct valid (>= 0) entries of one k-long index list.
+std::vector<int32_t> index_set(const int32_t* list, int k) {
+  std::vector<int32_t> v;
+  v.reserve(k);
+  for (int i = 0; i < k; ++i)
+    if (list[i] >= 0) v.push_back(list[i]);
+  std::sort(v.begin(), v.end());
+  v.erase(std::unique(v.begin(), v.end()), v.end());
+  return v;
+}
+
+long long intersection_size(const std::vector<int32_t>& a, const std::vector<int32_t>& b) {
+  long long n = 0;
+  size_t i = 0, j = 0;
+  while (i < a.size() && j < b.size()) {
+    if (a[i] < b[j]) {
+      ++i;
+    } else if (b[j] < a[i]) {
+      ++j;
+    } else {
+      ++n;
+      ++i;
+      ++j;
+    }
+  }
+  return n;
+}
+
+// Best way found so far to reach "layer i is a reset": resets, cumulative
+// similarity and the policy of layers 0..i.
+struct Path {
+  bool valid = false;
+  int resets = 0;
+  double sim = 0.0;
+  std::vector<uint8_t> policy;
+};
+
+// Preference between two complete-or-equal-length paths: fewer resets, then
+// more similarity, then the lexicographically smaller policy (reuse < reset).
+bool preferred(int r1, double s1, const std::vector<uint8_t>& p1, const Path& b) {
+  if (!b.valid) return true;
+  if (r1 != b.resets) return r1 < b.resets;
+  if (s1 != b.sim) return s1 > b.sim;
+  return p1 < b.policy;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k, const int32_t* topk,
+                     double* M) {
+  if (num_layers < 1 || num_sets < 0 || k < 1 || !M || (num_sets > 0 && !topk))
+    return HYLRA_ERR_INVALID;
+  const int L = num_layers, S = num_sets;
+  std::vector<std::vector<int32_t>> sets((size_t)L * S);
+  for (int l = 0; l < L; ++l)
+    for (int u = 0; u < S; ++u)
+      sets[(size_t)l * S + u] = index_set(topk + ((size_t)l * S + u) * k, k);
+  for (int t = 0; t < L; ++t) {
+    for (int s = 0; s < L; ++s) {
+      double v = 0.0;
+      if (s <= t) {
+        long long inter = 0, total = 0;
+        for (int u = 0; u < S; ++u) {
+          const auto& target = sets[(size_t)t * S + u];
+          total += (long long)target.size();
+          inter += intersection_size(sets[(size_t)s * S + u], target);
+        }
+        v = total ? (double)inter / (double)total : 0.0;
+      }
+      M[(size_t)t * L + s] = v;
+    }
+  }
+  return HYLRA_OK;
+}
+
+int hylra_dp_policy(int32_t num_layers, const double* M, double theta, uint8_t* policy,
+                    int32_t* num_resets, double* cum_similarity) {
+  if (num_layers < 1 || !M || !policy || std::isnan(theta)) return HYLRA_ERR_INVALID;
+  const int L = num_layers;
+  // reset[i]: best path whose layer i is a reset.  Every candidate for
+  // reset[j+1] comes from a state (i, j) with i <= j, so visiting i in
+  // increasing order settles reset[i] before it is extended.
+  std::vector<Path> reset(L);
+  reset[0].valid = true;
+  reset[0].resets = 1;
+  reset[0].sim = 0.0;
+  reset[0].policy.assign(1, 1);
+  Path best;
+  for (int i = 0; i < L; ++i) {
+    const Path& from = reset[i];
+    if (!from.valid) continue;
+    std::vector<uint8_t> pol = from.policy;  // policy of layers 0..j
+    double sim = from.sim;
+    for (int j = i;; ++j) {
+      // at state (i, j)
+      if (j == L - 1) {
+        if (preferred(from.resets, sim, pol, best)) {
+          best.valid = true;
+          best.resets = from.resets;
+          best.sim = sim;
+          best.policy = pol;
+        }
+        break;
+      }
+      // reset jump to (j+1, j+1)
+      pol.push_back(1);
+      if (preferred(from.resets + 1, sim, pol, reset[j + 1])) {
+        Path& to = reset[j + 1];
+        to.valid = true;
+        to.resets = from.resets + 1;
+        to.sim = sim;
+        to.policy = pol;
+      }
+      pol.pop_back();
+      // vertical move to (i, j+1), only while the similarity exceeds theta
+      const double mv = M[(size_t)(j + 1) * L + i];
+      if (!(mv > theta)) break;
+      sim += mv;
+      pol.push_back(0);
+    }
+  }
+  for (int l = 0; l < L; ++l) policy[l] = best.policy[l];
+  if (num_resets) *num_resets = best.resets;
+  if (cum_similarity) *cum_similarity = best.sim;
+  return HYLRA_OK;
+}
+
+}  // extern "C"

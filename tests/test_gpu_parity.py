@@ -1,0 +1,334 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle on
+the same seeded inputs, at sizes that span several work units and a ragged
+tail, plus the edge cases of the method."""
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_sparsity_b200 import build as hbuild
+from kv_cache_sparsity_b200 import hylra as H
+from kv_cache_sparsity_b200 import workloads as W
+from oracle import hylra_oracle as O
+
+import hylra_testlib as T
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    hbuild.build()
+    H.load()
+
+
+def _layer(w, layer=0):
+    q, K, V = W.layer_inputs(w, layer, device="cpu")
+    return q.cuda(), K.cuda(), V.cuda()
+
+
+def _full_and_check(w, layer=0, kv_capacity=None, inputs=None):
+    run = T.Runner(w, kv_capacity=kv_capacity)
+    q, K, V = inputs if inputs is not None else _layer(w, layer)
+    out, tk = run.full(q, K, V)
+    assert run.status() == 0
+    out, tk = out.cpu().numpy(), tk.cpu().numpy()
+    swaps = 0
+    for b in range(w.batch):
+        o_ref, S32, tk_ref = T.oracle_full(w, q, K, V, b)
+        T.check_out(out[b], o_ref, w.dtype, f"{w.name} b={b}")
+        for h in range(w.num_kv_heads):
+            swaps += T.check_topk(tk[b, h], tk_ref[h], S32[h], f"{w.name} b={b} h={h}")
+    return run, (q, K, V), out, tk, swaps
+
+
+CASES = [
+    W.custom("b1_h8_2_n4096", seqlens=(4096,), num_q_heads=8, num_kv_heads=2, topk=8),
+    W.custom("b3_dense_ragged", batch=3, seqlens=(1000, 128, 1), num_q_heads=8, num_kv_heads=2,
+             topk=4, seed=3),
+    W.custom("packed_ragged", batch=4, seqlens=(300, 2048, 129, 5000), num_q_heads=32,
+             num_kv_heads=8, topk=16, packed=True, seed=4),
+    W.custom("group1", seqlens=(2000,), num_q_heads=4, num_kv_heads=4, topk=6, seed=5),
+    W.custom("group2", seqlens=(3000,), num_q_heads=8, num_kv_heads=4, topk=6, seed=6),
+    W.custom("group8", seqlens=(2500,), num_q_heads=16, num_kv_heads=2, topk=6, seed=7),
+    W.custom("iid_bf16", seqlens=(6000,), num_q_heads=8, num_kv_heads=2, topk=8,
+             structure="iid", seed=8),
+    W.custom("many_heads", batch=2, seqlens=(9000, 7000), num_q_heads=64, num_kv_heads=16,
+             topk=12, seed=9),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_full_layer_matches_oracle(w):
+    _full_and_check(w)
+
+
+def test_tiny_fp32_config_step_matches_oracle():
+    """The small fp32 configuration: 4 layers, fixed policy [R, U, U, R]."""
+    w = W.config("tiny")
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    topk = torch.full((w.layers, w.batch, w.num_kv_heads, w.topk), -7, dtype=torch.int32,
+                      device="cuda")
+    outs = [run.new_out() for _ in range(w.layers)]
+    H.decode_step(run.shape, w.policy, [l[0] for l in layers], [l[1] for l in layers],
+                  [l[2] for l in layers], run.seqlens, outs, topk, run.ws)
+    assert run.status() == 0
+    np_layers = [(q.double().cpu().numpy(), K.double().cpu().numpy(), V.double().cpu().numpy())
+                 for q, K, V in layers]
+    o_ref, tk_ref = O.decode_step(w.policy, np_layers, w.seqlens, w.topk)
+    tk = topk.cpu().numpy()
+    for l in range(w.layers):
+        T.check_out(outs[l].cpu().numpy()[0], o_ref[l][0], "fp32", f"tiny layer {l}")
+        if w.policy[l]:
+            _, S32, _ = T.oracle_full(w, *layers[l], 0)
+            for h in range(w.num_kv_heads):
+                assert T.check_topk(tk[l, 0, h], tk_ref[l][0, h], S32[h], f"tiny l={l}") == 0
+
+
+def test_fp32_ragged_packed():
+    w = W.custom("fp32_packed", batch=3, seqlens=(777, 130, 2049), num_q_heads=6, num_kv_heads=2,
+                 topk=5, dtype="fp32", packed=True, structure="iid", seed=11)
+    _full_and_check(w)
+
+
+def test_dense_tail_rows_may_hold_nan():
+    """Rows past n_b in a dense cache are not part of the sequence: even NaN
+    there must not reach the output."""
+    w = W.custom("nan_tail", batch=2, seqlens=(1000, 300), num_q_heads=8, num_kv_heads=2, topk=4,
+                 seed=12)
+    q, K, V = _layer(w)
+    K = K.clone()
+    V = V.clone()
+    for b, n in enumerate(w.seqlens):
+        K[b, :, n:] = float("nan")
+        V[b, :, n:] = float("nan")
+    _full_and_check(w, inputs=(q, K, V))
+    run = T.Runner(w)
+    idx = torch.tensor([[[7, 0, 3, -1], [7, 1, -1, -1]], [[2, 0, 1, -1], [0, 2, -1, -1]]],
+                       dtype=torch.int32, device="cuda")
+    out = run.reuse(q, K, V, idx).cpu().numpy()
+    assert run.status() == 0
+    for b in range(2):
+        ref = T.oracle_reuse(w, q, K, V, b, idx[b].cpu().numpy())
+        T.check_out(out[b], ref, "bf16", f"nan_tail reuse b={b}")
+
+
+def test_capacity_larger_than_longest_sequence():
+    w = W.custom("cap", batch=2, seqlens=(640, 1500), num_q_heads=8, num_kv_heads=2, topk=4,
+                 seed=13)
+    q, K, V = _layer(w)
+    cap = 2048
+    K2 = torch.zeros(2, 2, cap, 128, dtype=K.dtype, device="cuda")
+    V2 = torch.zeros_like(K2)
+    K2[:, :, :K.shape[2]] = K
+    V2[:, :, :V.shape[2]] = V
+    _full_and_check(w, kv_capacity=cap, inputs=(q, K2, V2))
+
+
+@pytest.mark.parametrize("w", CASES[:3] + [W.custom("fp32r", seqlens=(1500, 4000), batch=2,
+                                                    dtype="fp32", structure="iid", seed=14)],
+                         ids=lambda w: w.name)
+def test_reuse_layer_matches_oracle(w):
+    """Reuse with the indices the full kernel produced for another layer."""
+    run = T.Runner(w)
+    q0, K0, V0 = _layer(w, 0)
+    q1, K1, V1 = _layer(w, 1)
+    _, tk = run.full(q0, K0, V0)
+    out = run.reuse(q1, K1, V1, tk).cpu().numpy()
+    assert run.status() == 0
+    tkn = tk.cpu().numpy()
+    for b in range(w.batch):
+        ref = T.oracle_reuse(w, q1, K1, V1, b, tkn[b])
+        T.check_out(out[b], ref, w.dtype, f"{w.name} reuse b={b}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_reuse_with_every_block_equals_full(dtype):
+    w = W.custom("allblocks", batch=2, seqlens=(1300, 700), num_q_heads=8, num_kv_heads=2,
+                 topk=11, dtype=dtype, seed=15)
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    out_f, _ = run.full(q, K, V)
+    nb = [(n + 127) // 128 for n in w.seqlens]
+    idx = torch.full((2, 2, 11), -1, dtype=torch.int32)
+    for b in range(2):
+        for h in range(2):
+            idx[b, h, :nb[b]] = torch.randperm(nb[b])
+    out_r = run.reuse(q, K, V, idx.cuda())
+    assert run.status() == 0
+    tol = 2e-3 if dtype == "bf16" else 1e-5
+    assert torch.allclose(out_r, out_f, atol=tol, rtol=0)
+
+
+def test_reuse_skips_minus_one_and_flags_bad_indices():
+    w = W.custom("badidx", batch=1, seqlens=(1000,), num_q_heads=8, num_kv_heads=2, topk=4,
+                 seed=16)
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    idx = torch.tensor([[[3, -1, 99, 5], [-5, 2, -1, -1]]], dtype=torch.int32, device="cuda")
+    out = run.reuse(q, K, V, idx).cpu().numpy()
+    st = run.status()
+    assert st & H.STATUS_BAD_INDEX
+    ref = T.oracle_reuse(w, q, K, V, 0, np.array([[3, -1, -1, 5], [-1, 2, -1, -1]]))
+    T.check_out(out[0], ref, "bf16", "badidx")
+
+
+def test_reuse_flags_duplicate_indices():
+    w = W.custom("dupidx", batch=1, seqlens=(1000,), num_q_heads=8, num_kv_heads=2, topk=4,
+                 seed=24)
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    idx = torch.tensor([[[3, 1, 3, -1], [0, 1, 2, 4]]], dtype=torch.int32, device="cuda")
+    run.reuse(q, K, V, idx)
+    assert run.status() & H.STATUS_DUP_INDEX
+    idx = torch.tensor([[[3, 1, 2, -1], [0, 1, 2, 4]]], dtype=torch.int32, device="cuda")
+    run.reuse(q, K, V, idx)
+    assert run.status() == 0
+
+
+def test_reuse_empty_selection_gives_zero():
+    w = W.custom("empty_sel", batch=1, seqlens=(500,), num_q_heads=8, num_kv_heads=2, topk=3,
+                 seed=17)
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    idx = torch.full((1, 2, 3), -1, dtype=torch.int32, device="cuda")
+    out = run.reuse(q, K, V, idx)
+    assert run.status() == 0
+    assert torch.all(out == 0)
+
+
+def test_empty_sequence_and_k_beyond_blocks():
+    w = W.custom("edge", batch=3, seqlens=(0, 200, 1), num_q_heads=8, num_kv_heads=2, topk=4,
+                 seed=18)
+    run, (q, K, V), out, tk, _ = _full_and_check(w)
+    assert np.all(out[0] == 0) and np.all(tk[0] == -1)
+    assert np.all(tk[1, :, 2:] == -1) and np.all(tk[2, :, 1:] == -1) and np.all(tk[2, :, 0] == 0)
+
+
+def test_equal_scores_pick_lowest_indices():
+    """All keys zero: every logit equal, every full block the same mass, the
+    partial last block less; ranks follow block index (lower first)."""
+    w = W.custom("ties", batch=1, seqlens=(128 * 9 + 50,), num_q_heads=8, num_kv_heads=2, topk=6,
+                 seed=19)
+    q, K, V = _layer(w)
+    K = torch.zeros_like(K)
+    _, _, _, tk, _ = _full_and_check(w, inputs=(q, K, V))
+    assert np.all(tk[0] == np.arange(6))
+
+
+def test_invalid_seqlen_is_flagged_not_faulted():
+    w = W.custom("badlen", batch=2, seqlens=(300, 300), num_q_heads=8, num_kv_heads=2, topk=3,
+                 seed=20)
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    run.seqlens[1] = 5000  # beyond the cache
+    out, tk = run.full(q, K, V)
+    st = run.status()
+    assert st & H.STATUS_BAD_SEQLEN
+    assert torch.all(out[1] == 0) and torch.all(tk[1] == -1)
+    ref, _, tk_ref = T.oracle_full(w, q, K, V, 0)
+    T.check_out(out[0].cpu().numpy(), ref, "bf16", "badlen b=0")
+
+
+def test_step_hybrid_matches_oracle_walk():
+    w = W.custom("step", batch=2, layers=6, seqlens=(3000, 1700), num_q_heads=8, num_kv_heads=2,
+                 topk=5, seed=21)
+    policy = (1, 0, 0, 1, 0, 1)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    topk = torch.full((w.layers, 2, 2, 5), -7, dtype=torch.int32, device="cuda")
+    outs = [run.new_out() for _ in range(w.layers)]
+    H.decode_step(run.shape, policy, [l[0] for l in layers], [l[1] for l in layers],
+                  [l[2] for l in layers], run.seqlens, outs, topk, run.ws)
+    assert run.status() == 0
+    np_layers = []
+    for q, K, V in layers:
+        np_layers.append((q.double().cpu().numpy(), K.double().cpu().numpy(),
+                          V.double().cpu().numpy()))
+    o_ref, tk_ref = O.decode_step(policy, np_layers, w.seqlens, w.topk)
+    tk = topk.cpu().numpy()
+    for l in range(w.layers):
+        T.check_out(outs[l].cpu().numpy(), o_ref[l], "bf16", f"step layer {l}")
+        if policy[l]:
+            assert np.array_equal(tk[l], tk_ref[l]), f"layer {l}"
+        else:
+            assert np.all(tk[l] == -7)   # reuse layers leave their slot untouched
+
+
+def test_step_in_cuda_graph_matches_eager():
+    w = W.custom("graph", batch=1, layers=4, seqlens=(4096,), num_q_heads=8, num_kv_heads=2,
+                 topk=8, seed=22)
+    policy = (1, 0, 1, 0)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    topk = torch.full((4, 1, 2, 8), -1, dtype=torch.int32, device="cuda")
+    outs = [run.new_out() for _ in range(4)]
+    args = ([l[0] for l in layers], [l[1] for l in layers], [l[2] for l in layers])
+    H.decode_step(run.shape, policy, *args, run.seqlens, outs, topk, run.ws)
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    eager_tk = topk.clone()
+    for o in outs:
+        o.fill_(float("nan"))
+    topk.fill_(-1)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        H.decode_step(run.shape, policy, *args, run.seqlens, outs, topk, run.ws,
+                      stream=torch.cuda.current_stream())
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs, eager):
+        assert torch.equal(a, b)
+    assert torch.equal(topk, eager_tk)
+    assert run.status() == 0
+
+
+def test_step_host_buffers_match_device_step():
+    w = W.custom("hoststep", batch=2, layers=3, seqlens=(2000, 900), num_q_heads=8,
+                 num_kv_heads=2, topk=4, seed=23)
+    policy = (1, 0, 1)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    q_host = torch.stack([l[0].cpu() for l in layers]).pin_memory()
+    q_dev = torch.empty_like(q_host, device="cuda")
+    out_dev = torch.empty(3, 2, 8, 128, dtype=torch.float32, device="cuda")
+    out_host = torch.empty(3, 2, 8, 128, dtype=torch.float32).pin_memory()
+    tk_dev = torch.full((3, 2, 2, 4), -1, dtype=torch.int32, device="cuda")
+    tk_host = torch.empty(3, 2, 2, 4, dtype=torch.int32).pin_memory()
+    H.decode_step_host(run.shape, policy, q_host, q_dev, [l[1] for l in layers],
+                       [l[2] for l in layers], run.seqlens, out_dev, out_host, tk_dev, tk_host,
+                       run.ws)
+    torch.cuda.synchronize()
+    outs = [run.new_out() for _ in range(3)]
+    tk2 = torch.full((3, 2, 2, 4), -1, dtype=torch.int32, device="cuda")
+    H.decode_step(run.shape, policy, [l[0] for l in layers], [l[1] for l in layers],
+                  [l[2] for l in layers], run.seqlens, outs, tk2, run.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, torch.stack([o.cpu() for o in outs]))
+    assert torch.equal(tk_host[0], tk2[0].cpu()) and torch.equal(tk_host[2], tk2[2].cpu())
+    assert run.status() == 0
+
+
+def test_repeated_calls_are_deterministic():
+    w = CASES[2]
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    o1, t1 = run.full(q, K, V)
+    o2, t2 = run.full(q, K, V)
+    assert torch.equal(o1, o2) and torch.equal(t1, t2)
+    assert run.status() == 0
+
+
+def test_workspace_too_small_is_rejected():
+    w = CASES[0]
+    run = T.Runner(w)
+    q, K, V = _layer(w)
+    small = run.ws[:256]
+    with pytest.raises(H.HylraError) as e:
+        H.decode_full(run.shape, q, K, V, run.seqlens, run.new_out(), run.new_topk(), small)
+    assert e.value.code == -4

@@ -1,0 +1,147 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol of
+include/hylra.h, validates arguments on the host, and its host-side policy
+functions (overlap matrix, DP) agree bit for bit with the oracle."""
+
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from kv_cache_sparsity_b200 import build as hbuild
+from kv_cache_sparsity_b200 import hylra as H
+from oracle import hylra_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return H.load()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(hylra_\w+)\s*\(", text,
+                                    re.MULTILINE))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"hylra_decode_full", "hylra_decode_reuse", "hylra_similarity",
+            "hylra_dp_policy"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+    assert set(H.EXPORTS) <= names
+
+
+def test_version_and_strerror(lib):
+    assert H.version() == 100
+    assert H.strerror(0) == "ok"
+    assert "workspace" in H.strerror(-4)
+
+
+def _shape(**kw):
+    base = dict(batch=1, num_q_heads=32, num_kv_heads=8, topk=16, max_seqlen=4096,
+                kv_capacity=4096)
+    base.update(kw)
+    return H.make_shape(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), -2), (dict(block_size=64), -2), (dict(num_q_heads=30), -1),
+    (dict(num_q_heads=80, num_kv_heads=8), -2), (dict(topk=0), -1), (dict(topk=5000), -2),
+    (dict(max_seqlen=-1), -1), (dict(max_seqlen=300000, kv_capacity=300000), -2),
+    (dict(kv_capacity=100), -1), (dict(batch=0), -1), (dict(batch=2000), -2),
+    (dict(dtype=7), -1), (dict(kv_capacity=0, total_tokens=100), -1),
+])
+def test_shape_validation_before_any_device_call(lib, kw, code):
+    n = ctypes.c_size_t(0)
+    rc = lib.hylra_workspace_bytes(ctypes.byref(_shape(**kw)), ctypes.byref(n))
+    assert rc == code
+
+
+def test_null_pointers_rejected(lib):
+    sh = _shape()
+    rc = lib.hylra_decode_full(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None)
+    assert rc == -1
+    rc = lib.hylra_dp_policy(0, None, 0.5, None, None, None)
+    assert rc == -1
+
+
+def test_step_rejects_leading_reuse_before_launch(lib):
+    sh = _shape()
+    pol = (ctypes.c_uint8 * 2)(0, 1)
+    fake = (ctypes.c_void_p * 2)(16, 16)
+    rc = lib.hylra_decode_step(ctypes.byref(sh), 2, pol, fake, fake, fake, 16, fake, 16, 256,
+                               1 << 20, None)
+    assert rc == -1
+
+
+# ------------------------------------------------------- host policy parity
+
+def test_similarity_golden(lib):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "similarity_3layer.json")))
+    M = H.similarity(np.array(g["topk"]))
+    assert M.tolist() == g["M"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_similarity_matches_oracle_bitwise(lib, seed):
+    rng = np.random.default_rng(seed)
+    L, S, k = int(rng.integers(1, 12)), int(rng.integers(1, 20)), int(rng.integers(1, 9))
+    nb = int(rng.integers(k, 3 * k + 2))
+    topk = np.full((L, S, k), -1, dtype=np.int32)
+    for l in range(L):
+        for u in range(S):
+            kp = int(rng.integers(0, k + 1)) if seed % 2 else k
+            topk[l, u, :kp] = rng.permutation(nb)[:kp]
+    M = H.similarity(topk)
+    Mo = O.similarity_matrix(topk)
+    assert M.tobytes() == Mo.tobytes()
+
+
+def _dyadic(L, rng, denom=64):
+    M = np.zeros((L, L))
+    for t in range(L):
+        M[t, :t] = rng.integers(0, denom + 1, size=t) / denom
+        M[t, t] = 1.0
+    return M
+
+
+@pytest.mark.parametrize("L", [1, 2, 4, 7, 8])
+def test_dp_matches_oracle_and_bruteforce(lib, L):
+    rng = np.random.default_rng(100 + L)
+    for trial in range(30):
+        M = _dyadic(L, rng)
+        theta = float(rng.choice([0.0, 0.3, 0.5, 0.75, 0.8, 1.0, -1.0]))
+        got = H.dp_policy(M, theta)
+        assert got == O.dp_policy(M, theta)
+        assert got == O.dp_policy_bruteforce(M, theta)
+
+
+def test_dp_matches_oracle_long(lib):
+    rng = np.random.default_rng(5)
+    for L in (16, 32, 64):
+        M = _dyadic(L, rng, denom=16)
+        for theta in (0.5, 0.8, 0.9):
+            assert H.dp_policy(M, theta) == O.dp_policy(M, theta)
+
+
+def test_dp_golden(lib):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "dp_4layer.json")))
+    for case in g["cases"]:
+        pol, R, S = H.dp_policy(np.array(g["M"]), case["theta"])
+        assert list(pol) == case["policy"] and R == case["resets"] and S == case["sim"]
+
+
+def test_dp_rejects_nan_theta(lib):
+    with pytest.raises(H.HylraError):
+        H.dp_policy(np.eye(3), float("nan"))
