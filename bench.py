@@ -132,7 +132,7 @@ class ClockSampler:
         sm = [_num(r[1]) for r in busy if _num(r[1])]
         smax = [_num(r[2]) for r in rows if _num(r[2])]
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in busy for i in range(4) if "Active" in r[5 + i]})
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
                 "samples": len(busy)}
@@ -346,7 +346,8 @@ def run_ours(args, rank, world, dist_on):
     ms_h = timed_replays(g_h, args.steps, dist_on)
     ms_f = timed_replays(g_f, args.steps, dist_on)
     # keep the GPU busy long enough for the sampler when the timed region is short
-    t_end = time.time() + max(0.0, 0.6 - (ms_h + ms_f) * args.steps / 1000.0)
+    fill = 0.0 if args.no_clock_fill else 0.6
+    t_end = time.time() + max(0.0, fill - (ms_h + ms_f) * args.steps / 1000.0)
     while time.time() < t_end:
         g_h.replay()
         torch.cuda.synchronize()
@@ -496,6 +497,8 @@ def main():
     ap.add_argument("--config", default="llama8b_32k", choices=W.CONFIG_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clock-fill", action="store_true",
+                    help="skip the extra busy window for the clock sampler (profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

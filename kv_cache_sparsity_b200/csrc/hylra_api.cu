@@ -35,7 +35,7 @@ int sm_count(int* G) {
   if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  *G = n;
+  *G = std::min(n, MAX_CTAS);
   return HYLRA_OK;
 }
 
@@ -147,9 +147,14 @@ int check_layer_ptrs(const hylra_shape_t* s, const void* q, const void* K, const
   return HYLRA_OK;
 }
 
+// pdl: launch as a programmatic dependent of the preceding kernel in the
+// stream (used between the layers of one decode step): the kernel's prologue
+// and its K/V streaming may overlap the preceding kernel's tail; everything
+// the preceding kernel writes is touched only after griddepcontrol.wait.
 int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, const void* V,
            const int32_t* seqlens, const int32_t* topk_in, float* out, int32_t* topk_out,
-           void* ws, size_t ws_bytes, cudaStream_t stream) {
+           void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl = false,
+           bool idx_from_prev = true) {
   int rc = check_shape(s);
   if (rc) return rc;
   if ((rc = check_layer_ptrs(s, q, K, V, out))) return rc;
@@ -184,6 +189,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.k = s->topk;
   p.max_seqlen = s->max_seqlen;
   p.nbmax = L.nbmax;
+  p.idx_wait = idx_from_prev ? 1 : 0;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
 
   if (s->dtype == HYLRA_BF16) {
@@ -194,15 +200,24 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     CUtensorMap tmK, tmV;
     if ((rc = make_tmap(&tmK, K, rows))) return rc;
     if ((rc = make_tmap(&tmV, V, rows))) return rc;
-    if (full)
-      decode_bf16_kernel<true><<<G, NTHR_BF16, kSmemBF16, stream>>>(tmK, tmV, p);
-    else
-      decode_bf16_kernel<false><<<G, NTHR_BF16, kSmemBF16, stream>>>(tmK, tmV, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(NTHR_BF16);
+    cfg.dynamicSmemBytes = kSmemBF16;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = full ? cudaLaunchKernelEx(&cfg, decode_bf16_kernel<true>, tmK, tmV, p)
+                               : cudaLaunchKernelEx(&cfg, decode_bf16_kernel<false>, tmK, tmV, p);
+    if (e != cudaSuccess) return HYLRA_ERR_CUDA;
   } else {
     if (full)
-      decode_f32_kernel<true><<<G, NTHR_F32, 0, stream>>>(p);
+      decode_f32_kernel<true><<<G, NT_F32, 0, stream>>>(p);
     else
-      decode_f32_kernel<false><<<G, NTHR_F32, 0, stream>>>(p);
+      decode_f32_kernel<false><<<G, NT_F32, 0, stream>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
 }
@@ -275,10 +290,11 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint
     if (policy[l]) {
       last_reset = l;
       rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
-                  workspace, workspace_bytes, (cudaStream_t)stream);
+                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0);
     } else {
       rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
-                  nullptr, workspace, workspace_bytes, (cudaStream_t)stream);
+                  nullptr, workspace, workspace_bytes, (cudaStream_t)stream, l > 0,
+                  last_reset == l - 1);
     }
     if (rc) return rc;
   }
@@ -319,6 +335,15 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
     return HYLRA_ERR_CUDA;
   return HYLRA_OK;
 }
+
+#ifdef HYLRA_TRACE
+// Trace builds only: device buffer of TRACE_PER_CTA uint64 per CTA (or NULL).
+int hylra_trace_set(void* buf) {
+  unsigned long long* p = static_cast<unsigned long long*>(buf);
+  return cudaMemcpyToSymbol(g_hylra_trace, &p, sizeof(p)) == cudaSuccess ? HYLRA_OK
+                                                                          : HYLRA_ERR_CUDA;
+}
+#endif
 
 int hylra_read_status(void* workspace, uint32_t* status, int clear, hylra_stream_t stream) {
   if (!workspace || !status) return HYLRA_ERR_INVALID;

@@ -164,3 +164,20 @@ __device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t
 }
 
 }  // namespace hylra
+
+namespace hylra {
+
+// ------------------------------------------- programmatic dependent launch
+// Wait until the preceding kernel in the stream (launched as this kernel's
+// programmatic primary) has completed and its writes are visible.  A no-op
+// when the kernel was launched without the programmatic attribute.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream to begin launching.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace hylra

@@ -15,7 +15,7 @@
 //     boundaries; each maximal run of one (b, h) is a "segment".
 //   * bf16 kernel: warp 0 issues TMA tile loads (128-byte swizzle, L2
 //     evict-first) of K and V blocks (64 KB per stage, 3 stages) plus the
-//     GQA group's q rows into shared memory; four consumer warps take 32
+//     GQA group's q rows into shared memory; eight consumer warps take 16
 //     tokens each.  Q.K^T runs as S^T = K Q^T on bf16 mma.sync (M = tokens,
 //     N = the r <= 8 q-heads), the softmax is online in the log2 domain with
 //     an fp32 running max and sum per warp, P^T moves from the accumulator
@@ -44,17 +44,40 @@ namespace hylra {
 constexpr int BLK = HYLRA_BLOCK_TOKENS;  // tokens per block
 constexpr int HD = HYLRA_HEAD_DIM;       // head dimension
 constexpr int GMAX = HYLRA_MAX_GROUP;    // q-heads per KV head, padded MMA N
-constexpr int NCW = 4;                   // consumer warps
-constexpr int NCONS = NCW * 32;          // consumer threads
-constexpr int NTHR_BF16 = NCONS + 32;    // + one producer warp
-constexpr int NTHR_F32 = NCONS;
+constexpr int NW_BF16 = 8;               // consumer warps of the bf16 kernel (16 tokens each)
+constexpr int NT_BF16 = NW_BF16 * 32;    // consumer threads of the bf16 kernel
+constexpr int NTHR_BF16 = NT_BF16 + 32;  // + one producer warp
+constexpr int NW_F32 = 4;                // warps of the fp32 kernel (32 tokens each)
+constexpr int NT_F32 = NW_F32 * 32;
+constexpr int NWMAX = 8;
+constexpr int NCOMB = 4;                 // per-warp states merged at a segment end
 constexpr int NSTAGE = 3;
 constexpr int BOX_BYTES = 64 * 2 * BLK;       // 64 bf16 columns x 128 rows
 constexpr int STAGE_BYTES = 4 * BOX_BYTES;    // K[:, 0:64], K[:, 64:128], V.., V..
 constexpr int QSLOT_BYTES = GMAX * HD * 2;
 constexpr int SLOT_FLOATS = GMAX * HD + 2 * GMAX;  // partial: O[8][128], m[8], Z[8]
 constexpr int MAX_NB = HYLRA_MAX_SEQLEN / BLK;
-constexpr int BAR_CONS = 1;  // named barrier of the consumer threads
+constexpr int BAR_CONS = 1;     // named barrier of the consumer threads
+constexpr int MAX_CTAS = 256;   // grid limit (a merge stages one entry per contributing CTA)
+constexpr int MAX_SEGS = 8;     // segments a CTA queues before taking their tickets
+
+// Optional timeline tracing (compile with -DHYLRA_TRACE; off by default and
+// then free): per CTA, the producer and the first consumer thread append
+// (event code, %globaltimer) pairs to a device buffer set by the host.
+#ifdef HYLRA_TRACE
+__device__ unsigned long long* g_hylra_trace = nullptr;
+constexpr int TRACE_PER_CTA = 512;
+__device__ __forceinline__ void trace_event(int& n, int base, int code) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  if (g_hylra_trace && n < 255)
+    g_hylra_trace[(size_t)blockIdx.x * TRACE_PER_CTA + base + n] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
+  ++n;
+}
+#define HYLRA_TRACE_EV(n, base, code) trace_event(n, base, code)
+#else
+#define HYLRA_TRACE_EV(n, base, code) ((void)0)
+#endif
 
 struct Params {
   const void* q;
@@ -72,6 +95,7 @@ struct Params {
   long long cap;    // dense rows per (b, h) plane; 0 = packed layout
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
+  int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
   float scale_log2;  // log2(e) / sqrt(d)
 };
 
@@ -92,35 +116,43 @@ __device__ __forceinline__ bool meta_sane(const Params& p, const StageMeta& m) {
 }
 
 struct SmemCommon {
-  float comb_o[NCW][GMAX][HD];  // per-warp O at a segment end; top-k scratch in a merge
-  float comb_m[NCW][GMAX];
-  float comb_z[NCW][GMAX];
+  float comb_o[NCOMB][GMAX][HD];  // warp states at a segment end; merge/top-k scratch
+  float comb_m[NWMAX][GMAX];
+  float comb_z[NWMAX][GMAX];
   float mg[GMAX];
   float zg[GMAX];
+  float cf[NCOMB][GMAX];  // segment-end scale factors
   int prefix[HYLRA_MAX_BATCH + 1];  // units before sequence b (all heads)
   int hist[256];
-  int misc[8];  // 0: last-CTA flag, 1: radix digit, 2: remaining, 3: list size, 4: abort
-  int warp_sums[NCW];
+  int misc[8];  // 1: radix digit, 2: remaining, 3: list size, 4: abort
+  int warp_sums[NWMAX];
+  StageMeta segs[MAX_SEGS];  // segments whose partial is stored but not yet ticketed
+  int seg_last[MAX_SEGS];
+  int nseg;
+  int trace_n;  // trace builds: events recorded by consumer thread 0
 };
-static_assert(sizeof(float) * NCW * GMAX * HD >= MAX_NB * 4 + HYLRA_MAX_TOPK * 8,
+static_assert(sizeof(float) * NCOMB * GMAX * HD >= MAX_NB * 4 + HYLRA_MAX_TOPK * 8,
               "top-k scratch must fit in the combine buffer");
+static_assert(sizeof(float) * NCOMB * GMAX * HD >= 2 * MAX_CTAS * GMAX * 4,
+              "merge staging must fit in the combine buffer");
 
 struct SmemBF16 {
   uint8_t stage[NSTAGE][STAGE_BYTES];  // 1024-byte aligned (128-byte swizzle atoms)
   uint8_t qslot[NSTAGE][QSLOT_BYTES];
-  float bst_s[NSTAGE][NCW][GMAX];
-  float bst_m[NSTAGE][NCW][GMAX];
+  float bst_s[NSTAGE][NW_BF16][GMAX];
+  float bst_m[NSTAGE][NW_BF16][GMAX];
   int bst_cnt[NSTAGE];
   StageMeta meta[NSTAGE];
-  alignas(8) uint64_t full_bar[NSTAGE];
+  alignas(8) uint64_t fullK_bar[NSTAGE];  // q rows (segment start) + K tile landed
+  alignas(8) uint64_t fullV_bar[NSTAGE];  // V tile landed
   alignas(8) uint64_t empty_bar[NSTAGE];
   SmemCommon c;
 };
 
 struct SmemF32 {
   float qs[GMAX][HD];
-  float bst_s[2][NCW][GMAX];
-  float bst_m[2][NCW][GMAX];
+  float bst_s[2][NW_F32][GMAX];
+  float bst_m[2][NW_F32][GMAX];
   SmemCommon c;
 };
 
@@ -189,6 +221,7 @@ template <bool FULL>
 __device__ void write_empty_outputs(const Params& p, const SmemCommon& c) {
   for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
     if (c.prefix[b + 1] != c.prefix[b]) continue;
+    griddep_wait();  // outputs may be buffers the preceding kernel writes
     float* o = p.out + (size_t)b * p.Hq * HD;
     for (int i = threadIdx.x; i < p.Hq * HD; i += blockDim.x) o[i] = 0.f;
     if (FULL) {
@@ -223,24 +256,19 @@ struct UnitIter {
   }
 };
 
-// Everything a unit needs besides its data.
+// Everything a unit needs besides its data.  seqlen: the validated length of
+// sequence it.b; blk_raw: the unit's block (FULL) or its reused index entry.
 template <bool FULL>
 __device__ __forceinline__ StageMeta describe_unit(const Params& p, const SmemCommon& c,
                                                    const UnitIter& it, int i, int n, int T,
-                                                   int G, bool report) {
+                                                   int G, int seqlen, int blk_raw, bool report) {
   StageMeta m;
   const int bh = it.b * p.Hkv + it.h;
-  const int seqlen = valid_seqlen(p, it.b, false);
   const int nb = (seqlen + BLK - 1) / BLK;
-  int blk;
-  if (FULL) {
-    blk = it.j;
-  } else {
-    blk = p.topk_in[(size_t)bh * p.k + it.j];
-    if (blk < 0 || blk >= nb) {
-      if (blk != -1 && report) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
-      blk = -1;
-    }
+  int blk = blk_raw;
+  if (!FULL && (blk < 0 || blk >= nb)) {
+    if (blk != -1 && report) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
+    blk = -1;
   }
   const int start = c.prefix[it.b] + it.h * it.U;
   const int cf = owner_cta(start, T, G);
@@ -258,13 +286,19 @@ __device__ __forceinline__ StageMeta describe_unit(const Params& p, const SmemCo
   return m;
 }
 
+__device__ __forceinline__ int unit_index_entry(const Params& p, const UnitIter& it) {
+  return __ldcg(p.topk_in + ((size_t)it.b * p.Hkv + it.h) * p.k + it.j);
+}
+
 // ------------------------------------------------------------------ top-k
 
 // Top-k of the block scores keys[0..nb) (fp32 bit patterns of non-negative
 // scores, so unsigned order is numeric order): rank order, score descending,
 // lower block index first among equal scores; slots k'..k-1 get -1.
-// Called by the NCONS consumer threads (ct = 0..NCONS-1).
+// Called by the NT merge threads (ct = 0..NT-1).
+template <int NT>
 __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int ct) {
+  constexpr int NW = NT / 32;
   uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
   uint2* list = reinterpret_cast<uint2*>(reinterpret_cast<char*>(&c.comb_o[0][0][0]) + MAX_NB * 4);
   int32_t* dst = p.topk_out + (size_t)bh * p.k;
@@ -276,16 +310,20 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
   int remain = kp;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    c.hist[ct] = 0;
-    c.hist[ct + NCONS] = 0;
+    for (int i = ct; i < 256; i += NT) c.hist[i] = 0;
     if (ct == 0) c.misc[3] = 0;
-    named_bar_sync(BAR_CONS, NCONS);
-    for (int beta = ct; beta < nb; beta += NCONS) {
-      const uint32_t key = keys[beta];
-      const bool match = pass == 0 || ((key ^ prefix) >> (shift + 8)) == 0u;
-      if (match) atomicAdd(&c.hist[(key >> shift) & 255u], 1);
+    named_bar_sync(BAR_CONS, NT);
+    // one shared atomic per distinct digit per warp (scores of one head
+    // mostly share their top bits, so per-thread atomics would serialize)
+    for (int beta0 = 0; beta0 < nb; beta0 += NT) {
+      const int beta = beta0 + ct;
+      const uint32_t key = beta < nb ? keys[beta] : 0u;
+      const bool match = beta < nb && (pass == 0 || ((key ^ prefix) >> (shift + 8)) == 0u);
+      const uint32_t digit = match ? ((key >> shift) & 255u) : 256u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+      if (match && (__ffs(peers) - 1) == lane) atomicAdd(&c.hist[digit], __popc(peers));
     }
-    named_bar_sync(BAR_CONS, NCONS);
+    named_bar_sync(BAR_CONS, NT);
     if (wid == 0) {
       int cnt[8];
       int local = 0;
@@ -314,14 +352,14 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
         }
       }
     }
-    named_bar_sync(BAR_CONS, NCONS);
+    named_bar_sync(BAR_CONS, NT);
     prefix |= (uint32_t)c.misc[1] << shift;
     remain = c.misc[2];
   }
   const uint32_t tau = prefix;  // the kp-th largest score; take `remain` of its copies
 
   // Keep every key above tau and the lowest-index `remain` keys equal to it.
-  const int per = (nb + NCONS - 1) / NCONS;
+  const int per = (nb + NT - 1) / NT;
   const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
   int eq = 0;
   for (int beta = b0; beta < b1; ++beta) eq += keys[beta] == tau;
@@ -332,9 +370,11 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     if (lane >= off) incl += v;
   }
   if (lane == 31) c.warp_sums[wid] = incl;
-  named_bar_sync(BAR_CONS, NCONS);
+  named_bar_sync(BAR_CONS, NT);
   int before = incl - eq;
-  for (int w = 0; w < wid; ++w) before += c.warp_sums[w];
+#pragma unroll
+  for (int w = 0; w < NW; ++w)
+    if (w < wid) before += c.warp_sums[w];
   for (int beta = b0; beta < b1; ++beta) {
     const uint32_t key = keys[beta];
     bool sel = key > tau;
@@ -347,8 +387,8 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
       if (pos < kp) list[pos] = make_uint2(key, (uint32_t)beta);  // exactly kp are selected
     }
   }
-  named_bar_sync(BAR_CONS, NCONS);
-  for (int e = ct; e < kp; e += NCONS) {
+  named_bar_sync(BAR_CONS, NT);
+  for (int e = ct; e < kp; e += NT) {
     const uint2 me = list[e];
     int rank = 0;
     for (int j = 0; j < kp; ++j) {
@@ -357,49 +397,140 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     }
     dst[rank] = (int32_t)me.y;
   }
-  for (int slot = kp + ct; slot < p.k; slot += NCONS) dst[slot] = -1;
+  for (int slot = kp + ct; slot < p.k; slot += NT) dst[slot] = -1;
 }
 
 // ---------------------------------------------------------------- merging
 
 // The last CTA of (b, h): LSE-merge every contributor's partial into out;
-// on reset layers also score the blocks and select the top-k.
-template <bool FULL>
+// on reset layers also score the blocks and select the top-k.  Loads that do
+// not depend on one another are issued together: the merge sits on the
+// kernel's tail, so it is one L2 round trip plus shared-memory work.
+template <bool FULL, int NT>
 __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
+  constexpr int NW = NT / 32;
+  constexpr int OB = 24;  // contributors per batch of output-row loads
   const int bh = m.b * p.Hkv + m.h;
-  const int d = ct;
-  for (int g = 0; g < p.r; ++g) {
+  const int nc = m.ncontrib;
+  const int r = p.r;
+  const int lane = ct & 31, wid = ct >> 5;
+  float* fm = &c.comb_o[0][0][0];     // [nc][GMAX]: maxima, then scale factors
+  float* fz = fm + MAX_CTAS * GMAX;   // [nc][GMAX]: sums
+  const float* pbase = p.partials + (size_t)m.first_slot * SLOT_FLOATS;
+  const int kp = min(p.k, m.nb);
+  const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+  const int32_t my_idx = (!FULL && ct < kp) ? __ldcg(idx + ct) : -1;
+
+  // Output columns of this thread: pairs (g, 2 columns); r*64 pairs in all.
+  const int npairs = r * (HD / 2);
+  const int pr0 = ct;
+  const bool has0 = pr0 < npairs;
+  const int g0 = has0 ? pr0 / (HD / 2) : 0, col0 = 2 * (pr0 % (HD / 2));
+  float2 v0[OB];
+#pragma unroll
+  for (int u = 0; u < OB; ++u) {
+    v0[u] = make_float2(0.f, 0.f);
+    if (has0 && u < nc)
+      v0[u] = __ldcg(reinterpret_cast<const float2*>(pbase + (size_t)u * SLOT_FLOATS + g0 * HD + col0));
+  }
+  // block records of the first block of this thread (reset layers)
+  float2 sv0[GMAX];
+#pragma unroll
+  for (int g = 0; g < GMAX; ++g) {
+    sv0[g] = make_float2(0.f, -INFINITY);
+    if (FULL && ct < m.nb && g < r)
+      sv0[g] = __ldcg(reinterpret_cast<const float2*>(
+          p.bstat + ((size_t)bh * p.nbmax + ct) * (2 * r) + 2 * g));
+  }
+  for (int e = ct; e < nc * r; e += NT) {
+    const int j = e / r, g = e - j * r;
+    const float* sl = pbase + (size_t)j * SLOT_FLOATS + GMAX * HD;
+    const float mv = __ldcg(sl + g), zv = __ldcg(sl + GMAX + g);
+    fm[j * GMAX + g] = mv;
+    fz[j * GMAX + g] = zv;
+  }
+  named_bar_sync(BAR_CONS, NT);
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 10 << 8);
+  // per head (one warp each): global max, global sum, per-contributor factor
+  for (int g = wid; g < r; g += NW) {
     float M = -INFINITY;
-    for (int j = 0; j < m.ncontrib; ++j)
-      M = fmaxf(M, __ldcg(p.partials + (size_t)(m.first_slot + j) * SLOT_FLOATS + GMAX * HD + g));
-    float Z = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int j = 0; j < m.ncontrib; ++j) {
-        const float* sl = p.partials + (size_t)(m.first_slot + j) * SLOT_FLOATS;
-        const float mj = __ldcg(sl + GMAX * HD + g);
-        if (mj == -INFINITY) continue;
-        const float f = exp2f(mj - M);
-        Z += __ldcg(sl + GMAX * HD + GMAX + g) * f;
-        O += __ldcg(sl + g * HD + d) * f;
-      }
+    for (int j = lane; j < nc; j += 32) M = fmaxf(M, fm[j * GMAX + g]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float Z = 0.f;
+    for (int j = lane; j < nc; j += 32) {
+      const float mj = fm[j * GMAX + g];
+      const float f = (M == -INFINITY || mj == -INFINITY) ? 0.f : exp2f(mj - M);
+      Z += fz[j * GMAX + g] * f;
+      fm[j * GMAX + g] = f;
     }
-    p.out[((size_t)m.b * p.Hq + (size_t)m.h * p.r + g) * HD + d] = Z > 0.f ? O / Z : 0.f;
-    if (ct == 0) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+    if (lane == 0) {
       c.mg[g] = M;
       c.zg[g] = Z;
     }
   }
+  named_bar_sync(BAR_CONS, NT);
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 11 << 8);
+  // output rows
+  for (int pr = ct; pr < npairs; pr += NT) {
+    const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
+    float2 acc = make_float2(0.f, 0.f);
+    int j = 0;
+    if (pr == pr0) {
+#pragma unroll
+      for (int u = 0; u < OB; ++u) {
+        if (u < nc) {
+          const float f = fm[u * GMAX + g];
+          acc.x = fmaf(v0[u].x, f, acc.x);
+          acc.y = fmaf(v0[u].y, f, acc.y);
+        }
+      }
+      j = OB;
+    }
+    for (; j < nc; j += OB) {
+      float2 v[OB];
+#pragma unroll
+      for (int u = 0; u < OB; ++u)
+        v[u] = (j + u < nc) ? __ldcg(reinterpret_cast<const float2*>(
+                                  pbase + (size_t)(j + u) * SLOT_FLOATS + g * HD + col))
+                            : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < OB; ++u) {
+        if (j + u < nc) {
+          const float f = fm[(j + u) * GMAX + g];
+          acc.x = fmaf(v[u].x, f, acc.x);
+          acc.y = fmaf(v[u].y, f, acc.y);
+        }
+      }
+    }
+    const float Z = c.zg[g];
+    float2 o = make_float2(0.f, 0.f);
+    if (Z > 0.f) o = make_float2(acc.x / Z, acc.y / Z);
+    *reinterpret_cast<float2*>(p.out + ((size_t)m.b * p.Hq + (size_t)m.h * r + g) * HD + col) = o;
+  }
   if (FULL) {
-    named_bar_sync(BAR_CONS, NCONS);
+    named_bar_sync(BAR_CONS, NT);  // factors (comb_o) no longer needed
     uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
     bool nonfinite = false;
-    for (int beta = ct; beta < m.nb; beta += NCONS) {
-      const float* bs = p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * p.r);
-      float score = 0.f;
-      for (int g = 0; g < p.r; ++g) {
-        const float s = __ldcg(bs + 2 * g), mb = __ldcg(bs + 2 * g + 1);
-        if (c.zg[g] > 0.f && mb != -INFINITY) score += s * exp2f(mb - c.mg[g]) / c.zg[g];
+    for (int beta = ct; beta < m.nb; beta += NT) {
+      float2 sv[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (beta == ct) {
+          sv[g] = sv0[g];
+        } else {
+          sv[g] = g < r ? __ldcg(reinterpret_cast<const float2*>(
+                              p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * r) + 2 * g))
+                        : make_float2(0.f, -INFINITY);
+        }
       }
+      float score = 0.f;
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g)
+        if (g < r && c.zg[g] > 0.f && sv[g].y != -INFINITY)
+          score += sv[g].x * exp2f(sv[g].y - c.mg[g]) / c.zg[g];
       uint32_t key = 0u;
       if (isfinite(score)) {
         if (score > 0.f) key = __float_as_uint(score);
@@ -409,80 +540,104 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
       keys[beta] = key;
     }
     if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
-    named_bar_sync(BAR_CONS, NCONS);
-    topk_select(p, c, bh, m.nb, ct);
-  }
-  if (!FULL) {
+    named_bar_sync(BAR_CONS, NT);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 12 << 8);
+    topk_select<NT>(p, c, bh, m.nb, ct);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 13 << 8);
+  } else {
     // a reused list naming one block twice counts that block twice: flag it
-    const int kp = min(p.k, m.nb);
-    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+    named_bar_sync(BAR_CONS, NT);  // factors (comb_o) no longer needed
+    int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
+    for (int e = ct; e < kp; e += NT) sidx[e] = e == ct ? my_idx : __ldcg(idx + e);
+    named_bar_sync(BAR_CONS, NT);
     bool dup = false;
-    for (int e = ct; e < kp; e += NCONS) {
-      const int32_t v = idx[e];
+    for (int e = ct; e < kp; e += NT) {
+      const int32_t v = sidx[e];
       if (v < 0) continue;
-      for (int j = 0; j < e; ++j) dup |= idx[j] == v;
+      for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
     }
     if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
   }
   if (ct == 0) p.tickets[bh] = 0u;  // ready for the next launch
-  named_bar_sync(BAR_CONS, NCONS);
+  named_bar_sync(BAR_CONS, NT);
 }
 
-// Segment end: comb_* hold the NCW warps' (m, Z, O).  Merge them into this
-// CTA's partial, publish it, and merge (b, h) if this CTA finished it last.
-template <bool FULL>
-__device__ void publish_segment(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
-  const int d = ct;
+// Segment end: comb_*[0..NCOMB) hold partial states (m, Z, O) of this CTA's
+// share of (b, h).  Merge them and store the CTA's partial (no fence: the
+// ticket that makes it visible is taken later, in flush_segments), and queue
+// the segment.  Ends with a barrier (comb_* may be rewritten afterwards).
+template <int NT>
+__device__ void store_partial(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
   const bool sane = meta_sane(p, m);
   float* slot = p.partials + (size_t)(sane ? m.seg_slot : 0) * SLOT_FLOATS;
-  for (int g = 0; g < p.r && sane; ++g) {
+  if (sane && ct < p.r) {
+    const int g = ct;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NCW; ++w) M = fmaxf(M, c.comb_m[w][g]);
-    float O = 0.f, Z = 0.f;
-    if (M != -INFINITY) {
+    for (int w = 0; w < NCOMB; ++w) M = fmaxf(M, c.comb_m[w][g]);
+    float Z = 0.f;
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = c.comb_m[w][g];
-        if (mw == -INFINITY) continue;
-        const float f = exp2f(mw - M);
-        O += c.comb_o[w][g][d] * f;
-        Z += c.comb_z[w][g] * f;
-      }
+    for (int w = 0; w < NCOMB; ++w) {
+      const float mw = c.comb_m[w][g];
+      const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      c.cf[w][g] = f;
+      Z += c.comb_z[w][g] * f;
     }
-    slot[g * HD + d] = O;
-    if (d == 0) {
-      slot[GMAX * HD + g] = M;
-      slot[GMAX * HD + GMAX + g] = Z;
+    slot[GMAX * HD + g] = M;
+    slot[GMAX * HD + GMAX + g] = Z;
+  }
+  named_bar_sync(BAR_CONS, NT);
+  if (sane) {
+    for (int pr = ct; pr < p.r * HD; pr += NT) {
+      const int g = pr / HD, d = pr - g * HD;
+      float O = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCOMB; ++w) O = fmaf(c.comb_o[w][g][d], c.cf[w][g], O);
+      slot[g * HD + d] = O;
     }
+    if (ct == 0) c.segs[c.nseg++] = m;
   }
-  __threadfence();
-  named_bar_sync(BAR_CONS, NCONS);
-  if (ct == 0) {
-    c.misc[0] = 0;
-    if (sane) {
-      const uint32_t old = atomic_add_acq_rel_gpu(p.tickets + m.b * p.Hkv + m.h, 1u);
-      c.misc[0] = (old == (uint32_t)(m.ncontrib - 1)) ? 1 : 0;
-    }
-  }
-  named_bar_sync(BAR_CONS, NCONS);
-  if (c.misc[0]) {
-    __threadfence();
-    merge_bh<FULL>(p, c, m, ct);
-  }
+  named_bar_sync(BAR_CONS, NT);
 }
 
-// Block record (local max, sum relative to it) of the NCW warps' shares of a
-// block, for head g: one (sum, max) pair relative to the block's own max.
+// Make this CTA's stored partials visible, take one ticket per queued
+// segment, and merge every (b, h) this CTA finished last.
+template <bool FULL, int NT>
+__device__ void flush_segments(const Params& p, SmemCommon& c, int ct) {
+  __threadfence();
+  named_bar_sync(BAR_CONS, NT);
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 14 << 8);
+  const int ns = c.nseg;
+  if (ct < ns) {
+    const StageMeta& m = c.segs[ct];
+    const uint32_t old = atomic_add_acq_rel_gpu(p.tickets + m.b * p.Hkv + m.h, 1u);
+    c.seg_last[ct] = (old == (uint32_t)(m.ncontrib - 1)) ? 1 : 0;
+  }
+  named_bar_sync(BAR_CONS, NT);
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 15 << 8);
+  for (int k = 0; k < ns; ++k) {
+    if (c.seg_last[k]) {
+      __threadfence();
+      const StageMeta m = c.segs[k];
+      merge_bh<FULL, NT>(p, c, m, ct);
+    }
+  }
+  if (ct == 0) c.nseg = 0;
+  named_bar_sync(BAR_CONS, NT);
+}
+
+// Block record of one head g from the nw warps' shares of a block: the
+// block's own max and its probability sum relative to that max.
+template <int NW>
 __device__ __forceinline__ void combine_block_record(const float (*bs)[GMAX],
                                                      const float (*bm)[GMAX], int g, float* dst) {
   float mm = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, bm[w][g]);
+  for (int w = 0; w < NW; ++w) mm = fmaxf(mm, bm[w][g]);
   float ss = 0.f;
   if (mm != -INFINITY) {
 #pragma unroll
-    for (int w = 0; w < NCW; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const float mw = bm[w][g];
       if (mw != -INFINITY) ss += bs[w][g] * exp2f(mw - mm);
     }
@@ -505,8 +660,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&sm.full_bar[s], 1);
-      mbar_init(&sm.empty_bar[s], NCW);
+      mbar_init(&sm.fullK_bar[s], 1);
+      mbar_init(&sm.fullV_bar[s], 1);
+      mbar_init(&sm.empty_bar[s], NW_BF16);
       sm.bst_cnt[s] = 0;
       StageMeta z{};
       z.blk = -1;
@@ -514,6 +670,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       sm.meta[s] = z;
     }
     c.misc[4] = 0;
+    c.nseg = 0;
+    c.trace_n = 0;
     fence_mbar_init();
   }
   if (tid == 32) {
@@ -530,6 +688,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   const int lo = works ? (int)((long long)blockIdx.x * T / G) : 0;
   const int hi = works ? (int)((long long)(blockIdx.x + 1) * T / G) : 0;
   const int n = hi - lo;
+  // Programmatic launch: a thread lets the next kernel in the stream launch
+  // (griddep_launch_dependents) only once it has waited for the preceding
+  // kernel (griddep_wait) or will never touch anything a kernel writes; so
+  // when a kernel runs, every kernel before its predecessor has completed.
   write_empty_outputs<FULL>(p, c);
   volatile int* abort_flag = &c.misc[4];
 
@@ -541,40 +703,70 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     const uint64_t pol = l2_evict_first_policy();
     const uint8_t* qbase = static_cast<const uint8_t*>(p.q);
     const uint32_t qbytes = (uint32_t)(p.r * HD * 2);
+    // per-sequence values, reloaded only when the sequence changes
+    int cur_b = -1, seqlen = 0;
+    long long row0 = 0;
+    const long long hstride = p.cap > 0 ? p.cap : p.total;
+    // reused indices written by the preceding kernel: wait for it first
+    if (!FULL && p.idx_wait) griddep_wait();
+    griddep_launch_dependents();  // the producer writes nothing
+    int idx_cur = FULL ? 0 : unit_index_entry(p, it);
+    int tn = 0;
+    (void)tn;
     for (int i = 0; i < n; ++i) {
+      UnitIter nx = it;
+      nx.advance(c, p);
+      // reuse: fetch the next unit's index now, use it next iteration
+      const int idx_next = (!FULL && i + 1 < n) ? unit_index_entry(p, nx) : 0;
+      if (it.b != cur_b) {
+        cur_b = it.b;
+        seqlen = valid_seqlen(p, cur_b, false);
+        row0 = p.cap > 0 ? (long long)cur_b * p.Hkv * p.cap : p.seq_off[cur_b];
+      }
       const int s = i % NSTAGE;
       const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
       mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
-      const StageMeta m = describe_unit<FULL>(p, c, it, i, n, T, G, true);
+      HYLRA_TRACE_EV(tn, 256, (2 << 8) | (i & 0xff));
+      const StageMeta m =
+          describe_unit<FULL>(p, c, it, i, n, T, G, seqlen, FULL ? it.j : idx_cur, true);
       sm.meta[s] = m;
       const bool seg_start = (m.flags & F_SEG_START) != 0;
-      uint32_t bytes = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? (uint32_t)STAGE_BYTES : 0u);
-      if (*abort_flag) bytes = 0;
-      if (bytes) {
-        mbar_arrive_expect_tx(&sm.full_bar[s], bytes);
+      uint32_t bytesK = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? 2u * BOX_BYTES : 0u);
+      uint32_t bytesV = m.blk >= 0 ? 2u * BOX_BYTES : 0u;
+      if (*abort_flag) bytesK = bytesV = 0u;
+      const int row = (int)(row0 + (long long)m.h * hstride + (long long)m.blk * BLK);
+      uint8_t* st = sm.stage[s];
+      if (bytesK) {
+        mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
         if (seg_start)
           bulk_load(sm.qslot[s], qbase + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD * 2, qbytes,
-                    &sm.full_bar[s]);
+                    &sm.fullK_bar[s]);
         if (m.blk >= 0) {
-          const int row = (int)(row_base(p, m.b, m.h) + (long long)m.blk * BLK);
-          uint8_t* st = sm.stage[s];
-          tma_load_2d(st, &tmK, 0, row, &sm.full_bar[s], pol);
-          tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.full_bar[s], pol);
-          tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.full_bar[s], pol);
-          tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.full_bar[s], pol);
+          tma_load_2d(st, &tmK, 0, row, &sm.fullK_bar[s], pol);
+          tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.fullK_bar[s], pol);
         }
       } else {
-        mbar_arrive(&sm.full_bar[s]);
+        mbar_arrive(&sm.fullK_bar[s]);
       }
-      it.advance(c, p);
+      if (bytesV) {
+        mbar_arrive_expect_tx(&sm.fullV_bar[s], bytesV);
+        tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.fullV_bar[s], pol);
+        tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.fullV_bar[s], pol);
+      } else {
+        mbar_arrive(&sm.fullV_bar[s]);
+      }
+      it = nx;
+      idx_cur = idx_next;
     }
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;
+  const int cw = warp - 1;   // 0..7: tokens 16*cw .. 16*cw+15 of every block
   const int ct = tid - 32;
   const int g4 = lane >> 2, c4 = lane & 3;
+  const int tokw = cw * 16;
+  const int mi = lane >> 3;
   float o[8][4];
   float m_run[2], z_run[2];
   uint32_t qf[8][2];
@@ -586,11 +778,25 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   z_run[0] = z_run[1] = 0.f;
 #pragma unroll
   for (int kt = 0; kt < 8; ++kt) qf[kt][0] = qf[kt][1] = 0u;
+  // this lane's ldmatrix rows: K (non-transposed) and V (transposed) tiles
+  const int krow = tokw + (lane & 7) + (mi & 1) * 8, kchi = mi >> 1;
+  const int vrow = tokw + (lane & 7) + (mi >> 1) * 8, vchi = mi & 1;
+  const int xr = lane & 7;  // == krow & 7 == vrow & 7
+  bool waited = false;  // griddep_wait done (needed before the first global write)
+  auto ensure_waited = [&]() {
+    if (!waited) {
+      griddep_wait();
+      griddep_launch_dependents();
+      waited = true;
+    }
+  };
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 1 << 8);
 
   for (int i = 0; i < n; ++i) {
     const int s = i % NSTAGE;
     const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
-    mbar_wait_bounded(&sm.full_bar[s], ph, abort_flag);
+    mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, (3 << 8) | (i & 0xff));
     const StageMeta m = sm.meta[s];
     if (m.flags & F_SEG_START) {
 #pragma unroll
@@ -610,45 +816,34 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (m.blk >= 0) {
       const uint32_t kbase = smem_u32(sm.stage[s]);
       const uint32_t vbase = kbase + 2 * BOX_BYTES;
-      const int tokw = cw * 32;
       const bool partial = m.nvalid < BLK;
-      float x[2][4];
-      // ---- S^T = K Q^T for this warp's 32 tokens (two m16 tiles)
+      float x[4];
+      // ---- S^T = K Q^T for this warp's 16 tokens, two accumulation chains
       {
-        float acc[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-        const int mi = lane >> 3;
+        float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t kb = kbase + krow * 128;
 #pragma unroll
         for (int kt = 0; kt < 8; ++kt) {
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            const int row = tokw + mt * 16 + (lane & 7) + (mi & 1) * 8;
-            const int ch = 2 * kt + (mi >> 1);
-            const uint32_t addr =
-                kbase + (ch >> 3) * BOX_BYTES + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(addr, a0, a1, a2, a3);
-            mma_bf16_16816(acc[mt], a0, a1, a2, a3, qf[kt][0], qf[kt][1]);
-          }
+          const int ch = 2 * kt + kchi;
+          const uint32_t addr = kb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(addr, r0, r1, r2, r3);
+          mma_bf16_16816((kt & 1) ? a1 : a0, r0, r1, r2, r3, qf[kt][0], qf[kt][1]);
         }
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float v = acc[mt][e] * p.scale_log2;
-            if (partial) {
-              const int tok = tokw + mt * 16 + g4 + ((e & 2) ? 8 : 0);
-              if (tok >= m.nvalid) v = -INFINITY;
-            }
-            x[mt][e] = v;
+        for (int e = 0; e < 4; ++e) {
+          float v = (a0[e] + a1[e]) * p.scale_log2;
+          if (partial) {
+            const int tok = tokw + g4 + ((e & 2) ? 8 : 0);
+            if (tok >= m.nvalid) v = -INFINITY;
           }
+          x[e] = v;
+        }
       }
+      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);
       if (partial) {
         // rows past the sequence end may hold anything (even NaN): zero V
-        for (int idx = lane; idx < 32 * 16; idx += 32) {
+        for (int idx = lane; idx < 16 * 16; idx += 32) {
           const int row = tokw + (idx >> 4);
           if (row < m.nvalid) continue;
           const int ch = idx & 15;
@@ -659,8 +854,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         __syncwarp();
       }
       // ---- block-local max and sums for heads 2*c4 (A) and 2*c4+1 (B)
-      float mxA = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
-      float mxB = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+      float mxA = fmaxf(x[0], x[2]);
+      float mxB = fmaxf(x[1], x[3]);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, off));
@@ -668,17 +863,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       }
       const float msA = mxA == -INFINITY ? 0.f : mxA;
       const float msB = mxB == -INFINITY ? 0.f : mxB;
-      float pr[2][4];
-      float sA = 0.f, sB = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        pr[mt][0] = ex2_approx(x[mt][0] - msA);
-        pr[mt][1] = ex2_approx(x[mt][1] - msB);
-        pr[mt][2] = ex2_approx(x[mt][2] - msA);
-        pr[mt][3] = ex2_approx(x[mt][3] - msB);
-        sA += pr[mt][0] + pr[mt][2];
-        sB += pr[mt][1] + pr[mt][3];
-      }
+      const float p0 = ex2_approx(x[0] - msA), p1 = ex2_approx(x[1] - msB);
+      const float p2 = ex2_approx(x[2] - msA), p3 = ex2_approx(x[3] - msB);
+      float sA = p0 + p2, sB = p1 + p3;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         sA += __shfl_xor_sync(0xffffffffu, sA, off);
@@ -690,7 +877,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         sm.bst_m[s][cw][2 * c4] = mxA;
         sm.bst_m[s][cw][2 * c4 + 1] = mxB;
       }
-      // ---- online softmax update
+      // ---- online softmax update (rescale only when a running max moved)
       const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
       float alA = 1.f, beA = 0.f, alB = 1.f, beB = 0.f;
       if (mnA != -INFINITY) {
@@ -705,50 +892,46 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       z_run[1] = z_run[1] * alB + sB * beB;
       m_run[0] = mnA;
       m_run[1] = mnB;
-#pragma unroll
-      for (int dm = 0; dm < 8; ++dm) {
-        o[dm][0] *= alA;
-        o[dm][1] *= alB;
-        o[dm][2] *= alA;
-        o[dm][3] *= alB;
-      }
-      // ---- P^T to the B-operand layout, then O^T += V^T P^T
-      uint32_t pb[2][2];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        pb[mt][0] = movmatrix_trans(pack_bf16x2(pr[mt][0] * beA, pr[mt][1] * beB));
-        pb[mt][1] = movmatrix_trans(pack_bf16x2(pr[mt][2] * beA, pr[mt][3] * beB));
-      }
-      const int mi = lane >> 3;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+      if (__any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
 #pragma unroll
         for (int dm = 0; dm < 8; ++dm) {
-          const int row = tokw + mt * 16 + (lane & 7) + (mi >> 1) * 8;
-          const int ch = 2 * dm + (mi & 1);
-          const uint32_t addr =
-              vbase + (ch >> 3) * BOX_BYTES + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(addr, a0, a1, a2, a3);
-          mma_bf16_16816(o[dm], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+          o[dm][0] *= alA;
+          o[dm][1] *= alB;
+          o[dm][2] *= alA;
+          o[dm][3] *= alB;
         }
       }
+      // ---- P^T to the B-operand layout, then O^T += V^T P^T
+      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0 * beA, p1 * beB));
+      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2 * beA, p3 * beB));
+      const uint32_t vb = vbase + vrow * 128;
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        const int ch = 2 * dm + vchi;
+        const uint32_t addr = vb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_trans(addr, r0, r1, r2, r3);
+        mma_bf16_16816(o[dm], r0, r1, r2, r3, pb0, pb1);
+      }
+    } else {
+      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);  // keep the phase in step
     }
     if (FULL && m.blk >= 0) {
-      // the last warp to finish this block merges the four shares
+      // the last warp to finish this block merges the eight shares
       __syncwarp();
       int last = 0;
       if (lane == 0) {
         __threadfence_block();
-        last = atomicAdd(&sm.bst_cnt[s], 1) == NCW - 1;
+        last = atomicAdd(&sm.bst_cnt[s], 1) == NW_BF16 - 1;
       }
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence_block();
+        ensure_waited();
         if (lane < p.r && meta_sane(p, m)) {
           float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
           float rec[2];
-          combine_block_record(sm.bst_s[s], sm.bst_m[s], lane, rec);
+          combine_block_record<NW_BF16>(sm.bst_s[s], sm.bst_m[s], lane, rec);
           dst[0] = rec[0];
           dst[1] = rec[1];
         }
@@ -756,41 +939,83 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       }
     }
     __syncwarp();
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, (4 << 8) | (i & 0xff));
     if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
 
     if (m.flags & F_SEG_END) {
+      if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
+      ensure_waited();
+      // eight warp states -> four (pairwise), then publish
+      if (cw >= NCOMB) {
+        const int w = cw - NCOMB;
 #pragma unroll
-      for (int dm = 0; dm < 8; ++dm) {
-        const int d0 = dm * 16 + g4;
-        c.comb_o[cw][2 * c4][d0] = o[dm][0];
-        c.comb_o[cw][2 * c4 + 1][d0] = o[dm][1];
-        c.comb_o[cw][2 * c4][d0 + 8] = o[dm][2];
-        c.comb_o[cw][2 * c4 + 1][d0 + 8] = o[dm][3];
+        for (int dm = 0; dm < 8; ++dm) {
+          const int d0 = dm * 16 + g4;
+          c.comb_o[w][2 * c4][d0] = o[dm][0];
+          c.comb_o[w][2 * c4 + 1][d0] = o[dm][1];
+          c.comb_o[w][2 * c4][d0 + 8] = o[dm][2];
+          c.comb_o[w][2 * c4 + 1][d0 + 8] = o[dm][3];
+        }
+        if (g4 == 0) {
+          c.comb_m[w][2 * c4] = m_run[0];
+          c.comb_m[w][2 * c4 + 1] = m_run[1];
+          c.comb_z[w][2 * c4] = z_run[0];
+          c.comb_z[w][2 * c4 + 1] = z_run[1];
+        }
       }
-      if (g4 == 0) {
-        c.comb_m[cw][2 * c4] = m_run[0];
-        c.comb_m[cw][2 * c4 + 1] = m_run[1];
-        c.comb_z[cw][2 * c4] = z_run[0];
-        c.comb_z[cw][2 * c4 + 1] = z_run[1];
+      named_bar_sync(BAR_CONS, NT_BF16);
+      if (cw < NCOMB) {
+        const float m2A = c.comb_m[cw][2 * c4], m2B = c.comb_m[cw][2 * c4 + 1];
+        const float z2A = c.comb_z[cw][2 * c4], z2B = c.comb_z[cw][2 * c4 + 1];
+        __syncwarp();
+        const float mnA = fmaxf(m_run[0], m2A), mnB = fmaxf(m_run[1], m2B);
+        const float fA = mnA == -INFINITY ? 0.f : ex2_approx(m_run[0] - mnA);
+        const float hA = mnA == -INFINITY ? 0.f : ex2_approx(m2A - mnA);
+        const float fB = mnB == -INFINITY ? 0.f : ex2_approx(m_run[1] - mnB);
+        const float hB = mnB == -INFINITY ? 0.f : ex2_approx(m2B - mnB);
+#pragma unroll
+        for (int dm = 0; dm < 8; ++dm) {
+          const int d0 = dm * 16 + g4;
+          float* a = &c.comb_o[cw][2 * c4][d0];
+          float* b = &c.comb_o[cw][2 * c4 + 1][d0];
+          a[0] = o[dm][0] * fA + a[0] * hA;
+          b[0] = o[dm][1] * fB + b[0] * hB;
+          a[8] = o[dm][2] * fA + a[8] * hA;
+          b[8] = o[dm][3] * fB + b[8] * hB;
+        }
+        if (g4 == 0) {
+          c.comb_m[cw][2 * c4] = mnA;
+          c.comb_m[cw][2 * c4 + 1] = mnB;
+          c.comb_z[cw][2 * c4] = z_run[0] * fA + z2A * hA;
+          c.comb_z[cw][2 * c4 + 1] = z_run[1] * fB + z2B * hB;
+        }
       }
-      named_bar_sync(BAR_CONS, NCONS);
-      publish_segment<FULL>(p, c, m, ct);
+      named_bar_sync(BAR_CONS, NT_BF16);
+      store_partial<NT_BF16>(p, c, m, ct);
+      if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 6 << 8);
+      if (c.nseg == MAX_SEGS) flush_segments<FULL, NT_BF16>(p, c, ct);
     }
   }
+  if (n > 0) {
+    ensure_waited();
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 7 << 8);
+    flush_segments<FULL, NT_BF16>(p, c, ct);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 8 << 8);
+  }
+  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 9 << 8);
   if (*abort_flag && ct == 0) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
 }
 
 // ------------------------------------------------------------ fp32 kernel
 
 template <bool FULL>
-__global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(NT_F32, 1) decode_f32_kernel(const __grid_constant__ Params p) {
   __shared__ SmemF32 sm;
   SmemCommon& c = sm.c;
   const int ct = threadIdx.x, cw = ct >> 5, lane = ct & 31;
+  if (ct == 0) c.nseg = 0;
   build_prefix(p, c, FULL);
   __syncthreads();
-  // Work split over G = min(grid, T) CTAs so that every working CTA owns at
-  // least one unit (the contributor count of a (b, h) relies on it).
   const int T = c.prefix[p.B];
   const int G = T > 0 ? min((int)gridDim.x, T) : 1;
   const bool works = (int)blockIdx.x < G;
@@ -799,6 +1024,8 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
   const int n = hi - lo;
   write_empty_outputs<FULL>(p, c);
   if (n <= 0) return;
+  griddep_wait();  // the CUDA-core path is for small cases: no early start
+  griddep_launch_dependents();
 
   const float* Kf = static_cast<const float*>(p.K);
   const float* Vf = static_cast<const float*>(p.V);
@@ -806,18 +1033,20 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
   UnitIter it;
   it.seek(c, p, lo);
   for (int i = 0; i < n; ++i) {
-    const StageMeta m = describe_unit<FULL>(p, c, it, i, n, T, G, ct == 0);
+    const int blk_raw = FULL ? it.j : unit_index_entry(p, it);
+    const StageMeta m = describe_unit<FULL>(p, c, it, i, n, T, G, valid_seqlen(p, it.b, false),
+                                            blk_raw, ct == 0);
     it.advance(c, p);
     if (m.flags & F_SEG_START) {
       const float* qg = static_cast<const float*>(p.q) + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD;
-      for (int e = ct; e < p.r * HD; e += NTHR_F32) sm.qs[e / HD][e % HD] = qg[e];
+      for (int e = ct; e < p.r * HD; e += NT_F32) sm.qs[e / HD][e % HD] = qg[e];
 #pragma unroll
       for (int g = 0; g < GMAX; ++g) {
         m_run[g] = -INFINITY;
         z_run[g] = 0.f;
         o[g][0] = o[g][1] = o[g][2] = o[g][3] = 0.f;
       }
-      named_bar_sync(BAR_CONS, NCONS);
+      named_bar_sync(BAR_CONS, NT_F32);
     }
     if (m.blk >= 0) {
       const long long row0 = row_base(p, m.b, m.h) + (long long)m.blk * BLK + cw * 32;
@@ -841,12 +1070,11 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
           }
         }
       }
-      float pr[GMAX], be[GMAX];
+      float pr[GMAX];
 #pragma unroll
       for (int g = 0; g < GMAX; ++g) {
         if (g >= p.r) {
           pr[g] = 0.f;
-          be[g] = 0.f;
           continue;
         }
         const float xg = valid ? acc[g] * p.scale_log2 : -INFINITY;
@@ -875,7 +1103,6 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
         o[g][2] *= al;
         o[g][3] *= al;
         pr[g] = pv * b;
-        be[g] = b;
       }
       const int nv = max(0, min(32, m.nvalid - cw * 32));
       for (int tt = 0; tt < nv; ++tt) {
@@ -891,14 +1118,13 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
           }
         }
       }
-      (void)be;
     }
     if (FULL && m.blk >= 0) {
-      named_bar_sync(BAR_CONS, NCONS);
+      named_bar_sync(BAR_CONS, NT_F32);
       if (cw == 0 && lane < p.r && meta_sane(p, m)) {
         float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
         float rec[2];
-        combine_block_record(sm.bst_s[i & 1], sm.bst_m[i & 1], lane, rec);
+        combine_block_record<NW_F32>(sm.bst_s[i & 1], sm.bst_m[i & 1], lane, rec);
         dst[0] = rec[0];
         dst[1] = rec[1];
       }
@@ -917,10 +1143,12 @@ __global__ void __launch_bounds__(NTHR_F32) decode_f32_kernel(const __grid_const
           }
         }
       }
-      named_bar_sync(BAR_CONS, NCONS);
-      publish_segment<FULL>(p, c, m, ct);
+      named_bar_sync(BAR_CONS, NT_F32);
+      store_partial<NT_F32>(p, c, m, ct);
+      if (c.nseg == MAX_SEGS) flush_segments<FULL, NT_F32>(p, c, ct);
     }
   }
+  flush_segments<FULL, NT_F32>(p, c, ct);
 }
 
 }  // namespace hylra

@@ -9,8 +9,9 @@ concrete as five named configurations.
 Structure of the keys ("salient" workloads).  Per (sequence b, KV head h):
 a unit direction u[b,h] shared by every layer; a salient set of 2k blocks
 shared by every layer with base amplitude A ~ U[2, 6]; a per-layer drift
-A_l = A + 0.15 * W_l, where W_l is a Gaussian random walk over layers (so the
-top-k sets of nearby layers overlap and the overlap decays with distance).
+A_l = A + DRIFT * W_l, where W_l is a Gaussian random walk over layers (so the
+top-k sets of nearby layers overlap and the overlap decays with distance;
+DRIFT = 0.7 gives the 32-layer workloads about 7 reset layers at theta = 0.8).
 K_l[b,h,t] = A_l[block(t)] * u[b,h] (salient blocks only) + N(0, 0.5^2);
 q_l[b,g] = sqrt(d) * u[b, g // r] + N(0, 1); V_l ~ N(0, 1).
 
@@ -29,6 +30,7 @@ import torch
 
 BLOCK = 128
 BASE_SEED = 20260203
+DRIFT = 0.7  # per-layer step of the salient amplitudes' random walk (nats)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -149,7 +151,7 @@ def _structure(w: Workload) -> _Structure:
             walk = torch.cumsum(torch.randn(w.layers, nsal, generator=g, dtype=torch.float64),
                                 dim=0)
             walk[0] = 0.0
-            amp[:, b, h, blocks] = base[None, :] + 0.15 * walk
+            amp[:, b, h, blocks] = base[None, :] + DRIFT * walk
     return _Structure(u.float(), amp.float())
 
 
