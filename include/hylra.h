@@ -170,6 +170,27 @@ int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k,
 int hylra_dp_policy(int32_t num_layers, const double* M, double theta,
                     uint8_t* policy, int32_t* num_resets, double* cum_similarity);
 
+/* hylra_decode_full without a caller-supplied workspace.  The paper has no
+ * counterpart: this exists for callers that cannot allocate device memory
+ * when they call (a process that reserved all free device memory up front,
+ * code that must not call cudaMalloc because it synchronises the device, or
+ * a binding with nowhere to keep a workspace alive).  It allocates nothing:
+ * its scratch is an 8 MiB array compiled into the library, present on every
+ * device that loads the library until the process exits.
+ *  - Same arguments, layouts and results as hylra_decode_full; shapes whose
+ *    workspace (hylra_workspace_bytes) exceeds 8 MiB return
+ *    HYLRA_ERR_WORKSPACE before anything is launched.
+ *  - status_out: optional DEVICE uint32 that receives the call's status word
+ *    (HYLRA_STATUS_* bits); NULL to skip.
+ *  - The first call on a device looks up the scratch's device address; make
+ *    that first call before any stream capture on that device.
+ *  - Every call on a device shares the one scratch array: calls that can
+ *    overlap on the GPU (other streams, other host threads) race; serialise
+ *    them, e.g. on one stream. */
+int hylra_decode_full_noalloc(const hylra_shape_t* shape, const void* q, const void* K,
+                              const void* V, const int32_t* seqlens, float* out,
+                              int32_t* topk_out, uint32_t* status_out, hylra_stream_t stream);
+
 /* Copy the workspace status word to *status (synchronises the stream); when
  * clear != 0 the word is reset to 0 afterwards. */
 int hylra_read_status(void* workspace, uint32_t* status, int clear,

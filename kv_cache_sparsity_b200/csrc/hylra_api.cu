@@ -358,4 +358,67 @@ int hylra_read_status(void* workspace, uint32_t* status, int clear, hylra_stream
   return HYLRA_OK;
 }
 
+// ------------------------------------------------ no-allocation entry point
+//
+// Some callers cannot hand the library a workspace: a serving process may
+// reserve all free device memory for itself up front, cudaMalloc/cudaFree
+// synchronise the device and are off limits inside latency-critical loops,
+// and a thin foreign-language binding may have nowhere to keep a buffer
+// alive between calls.  For them, hylra_decode_full_noalloc runs the reset
+// layer kernel on a scratch area compiled into this library.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+
+// Scratch of hylra_decode_full_noalloc.  It exists on every device that loads
+// the library, for the life of the process.  In host code this name is only
+// a host-side handle: its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the first call on a device must not be inside a stream capture).
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> addr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)addr.size() <= dev) addr.resize(dev + 1, nullptr);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HYLRA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return HYLRA_OK;
+}
+
+}  // namespace
+
+int hylra_decode_full_noalloc(const hylra_shape_t* shape, const void* q, const void* K,
+                              const void* V, const int32_t* seqlens, float* out,
+                              int32_t* topk_out, uint32_t* status_out, hylra_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  int G = 0;
+  if ((rc = sm_count(&G))) return rc;
+  const Layout L = make_layout(shape, G);
+  if (L.total > kNoAllocScratchBytes) return HYLRA_ERR_WORKSPACE;  // shape too large for it
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  // The scratch keeps whatever the previous call left: zero the status word
+  // and the per-(sequence, KV head) tickets, which must start at zero.
+  if (cudaMemsetAsync(scratch, 0, L.partials, st) != cudaSuccess) return HYLRA_ERR_CUDA;
+  rc = hylra_decode_full(shape, q, K, V, seqlens, out, topk_out, scratch, kNoAllocScratchBytes,
+                         stream);
+  if (rc) return rc;
+  if (status_out &&
+      cudaMemcpyAsync(status_out, static_cast<unsigned char*>(scratch) + L.status,
+                      sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return HYLRA_OK;
+}
+
 }  // extern "C"

@@ -40,7 +40,7 @@ ERRORS = {0: "HYLRA_OK", -1: "HYLRA_ERR_INVALID", -2: "HYLRA_ERR_UNSUPPORTED",
 EXPORTS = ("hylra_workspace_bytes", "hylra_workspace_init", "hylra_decode_full",
            "hylra_decode_reuse", "hylra_decode_step", "hylra_decode_step_host",
            "hylra_similarity", "hylra_dp_policy", "hylra_read_status", "hylra_strerror",
-           "hylra_version")
+           "hylra_version", "hylra_decode_full_noalloc")
 
 
 class HylraError(RuntimeError):
@@ -94,6 +94,7 @@ def load() -> ctypes.CDLL:
         "hylra_dp_policy": [I32, P, ctypes.c_double, P, ctypes.POINTER(I32),
                             ctypes.POINTER(ctypes.c_double)],
         "hylra_read_status": [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P],
+        "hylra_decode_full_noalloc": [SP, P, P, P, P, P, P, P, P],
         "hylra_strerror": [ctypes.c_int],
         "hylra_version": [],
     }
@@ -185,6 +186,15 @@ def decode_step_host(shape: Shape, policy: Sequence[int], q_host, q_dev, Ks, Vs,
                                          _ptr(topk_host), _ptr(ws),
                                          ws.numel() * ws.element_size(), _stream(stream)),
            "hylra_decode_step_host")
+
+
+def decode_full_noalloc(shape: Shape, q, K, V, seqlens, out, topk_out, status_out=None,
+                        stream=None):
+    """Reset layer on the library's built-in scratch (no workspace argument)."""
+    _check(load().hylra_decode_full_noalloc(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V),
+                                            _ptr(seqlens), _ptr(out), _ptr(topk_out),
+                                            _ptr(status_out), _stream(stream)),
+           "hylra_decode_full_noalloc")
 
 
 def read_status(ws, clear: bool = True, stream=None) -> int:
