@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from kv_cache_sparsity_b200 import build as hbuild  # noqa: E402
+from kv_cache_sparsity_b200 import dist as D  # noqa: E402
 from kv_cache_sparsity_b200 import workloads as W  # noqa: E402
 
 METRIC = ("decode-attention µs/step & KV HBM GB/s vs ~8 TB/s; HyLRA vs full speedup")
@@ -217,8 +218,7 @@ def derive_policy(m: Model, H):
 
 
 def timed_replays(g, steps, dist_on):
-    if dist_on:
-        torch.distributed.barrier()
+    D.barrier()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -227,17 +227,12 @@ def timed_replays(g, steps, dist_on):
         g.replay()
     e1.record(st)
     torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
+    D.barrier()
     return e0.elapsed_time(e1) / steps
 
 
 def max_over_ranks(x: float, dist_on: bool) -> float:
-    if not dist_on:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return D.max_over_ranks(x, device="cuda") if dist_on else x
 
 
 def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
@@ -257,8 +252,7 @@ def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
 
     for _ in range(warmup):
         one()
-    if dist_on:
-        torch.distributed.barrier()
+    D.barrier()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -267,8 +261,7 @@ def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
         one()
     e1.record(st)
     torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
+    D.barrier()
     ms = e0.elapsed_time(e1) / steps
     h2d = q_host.numel() * q_host.element_size()
     d2h = out_host.numel() * 4 + tk_host.numel() * 4
@@ -503,9 +496,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = D.rank_env()
 
     if args.impl == "reference":
         if rank == 0:
