@@ -22,6 +22,8 @@ namespace {
 
 constexpr size_t kSmemBF16 = sizeof(SmemBF16) + 1024;  // + alignment slack
 static_assert(kSmemBF16 <= 232448, "bf16 kernel shared memory exceeds 227 KB");
+static_assert(rc_smem_bytes(NST_MAX_RC) + 1024 <= 232448,
+              "cluster reuse kernel shared memory exceeds 227 KB");
 
 struct Layout {
   size_t status, tickets, partials, bstat, total;
@@ -138,6 +140,87 @@ int prepare_bf16_kernels() {
   return HYLRA_OK;
 }
 
+// Cluster reuse kernel: cluster size (CTAs per (b, h)), blocks per CTA and
+// pipeline stages.  The largest cluster size (<= 16, <= the blocks per head)
+// whose B*Hkv clusters the device can hold at once; 0 when none can.
+struct RCPlan {
+  int cs, upc, nst;
+  size_t smem;
+};
+
+RCPlan rc_plan_for(int cs, int kmax) {
+  RCPlan pl{};
+  pl.cs = cs;
+  pl.upc = (kmax + cs - 1) / cs;
+  pl.nst = std::min(pl.upc, NST_MAX_RC);
+  pl.smem = rc_smem_bytes(pl.nst) + 1024;
+  return pl;
+}
+
+// Clusters of this size and stage count the device can hold at once
+// (queried once per device).
+int rc_max_active(int cs, int nst) {
+  static std::mutex mu;
+  static std::vector<std::vector<int>> cache;  // [dev][cs * 4 + nst]: -1 unknown
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, std::vector<int>(17 * 4, -1));
+  int& v = cache[dev][cs * 4 + nst];
+  if (v < 0) {
+    v = 0;
+    if (cudaFuncSetAttribute(decode_reuse_cluster_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(rc_smem_bytes(NST_MAX_RC) + 1024)) == cudaSuccess &&
+        cudaFuncSetAttribute(decode_reuse_cluster_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs, 1);
+      cfg.blockDim = dim3(NTHR_BF16);
+      cfg.dynamicSmemBytes = rc_smem_bytes(nst) + 1024;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, decode_reuse_cluster_kernel, &cfg) == cudaSuccess)
+        v = n;
+    }
+    cudaGetLastError();  // a refused query leaves no error behind
+  }
+  return v;
+}
+
+// A small reuse layer (fewer blocks than SMs) is latency-bound: it takes at
+// most half the SMs so that, launched as a programmatic dependent, the next
+// layer's CTAs are resident and loading while this one finishes.  A large one
+// spreads over every SM.  Each CTA holds a whole SM (registers).
+bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
+  const int nbmax = std::max(1, (s->max_seqlen + BLK - 1) / BLK);
+  const int kmax = std::max(1, std::min(s->topk, nbmax));
+  const int nbh = s->batch * s->num_kv_heads;
+  if (nbh > 65535) return false;
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return false;
+  const bool small = (long long)nbh * kmax <= sms;
+  const int budget = small ? sms / 2 : sms;
+  const int cs_max = std::max(1, std::min(std::min(16, kmax), budget / std::max(1, nbh)));
+  for (int cs = cs_max; cs >= 1; --cs) {
+    const RCPlan pl = rc_plan_for(cs, kmax);
+    const int n = rc_max_active(cs, pl.nst);
+    if (n >= nbh || (cs == 1 && n > 0)) {
+      *out = pl;
+      return true;
+    }
+  }
+  return false;
+}
+
 int check_layer_ptrs(const hylra_shape_t* s, const void* q, const void* K, const void* V,
                      const float* out) {
   if (!q || !K || !V || !out) return HYLRA_ERR_INVALID;
@@ -154,7 +237,7 @@ int check_layer_ptrs(const hylra_shape_t* s, const void* q, const void* K, const
 int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, const void* V,
            const int32_t* seqlens, const int32_t* topk_in, float* out, int32_t* topk_out,
            void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl = false,
-           bool idx_from_prev = true) {
+           bool idx_from_prev = true, int trace_slot = 0) {
   int rc = check_shape(s);
   if (rc) return rc;
   if ((rc = check_layer_ptrs(s, q, K, V, out))) return rc;
@@ -190,6 +273,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.max_seqlen = s->max_seqlen;
   p.nbmax = L.nbmax;
   p.idx_wait = idx_from_prev ? 1 : 0;
+  p.trace_slot = trace_slot;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
 
   if (s->dtype == HYLRA_BF16) {
@@ -200,6 +284,32 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     CUtensorMap tmK, tmV;
     if ((rc = make_tmap(&tmK, K, rows))) return rc;
     if ((rc = make_tmap(&tmV, V, rows))) return rc;
+    if (!full) {
+      // reuse layers: one cluster per (b, h) when the device can schedule it
+      const int nbh = s->batch * s->num_kv_heads;
+      RCPlan pl{};
+      if (plan_reuse_cluster(s, &pl)) {
+        p.upc = pl.upc;
+        p.nst = pl.nst;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pl.cs, nbh);
+        cfg.blockDim = dim3(NTHR_BF16);
+        cfg.dynamicSmemBytes = pl.smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = pl.cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 2 : 1;
+        if (cudaLaunchKernelEx(&cfg, decode_reuse_cluster_kernel, tmK, tmV, p) != cudaSuccess)
+          return HYLRA_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
+      }
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(NTHR_BF16);
@@ -290,11 +400,11 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint
     if (policy[l]) {
       last_reset = l;
       rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
-                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0);
+                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0, true, l & 63);
     } else {
       rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
                   nullptr, workspace, workspace_bytes, (cudaStream_t)stream, l > 0,
-                  last_reset == l - 1);
+                  last_reset == l - 1, l & 63);
     }
     if (rc) return rc;
   }

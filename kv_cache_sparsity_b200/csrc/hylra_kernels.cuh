@@ -67,15 +67,27 @@ constexpr int MAX_SEGS = 8;     // segments a CTA queues before taking their tic
 #ifdef HYLRA_TRACE
 __device__ unsigned long long* g_hylra_trace = nullptr;
 constexpr int TRACE_PER_CTA = 512;
-__device__ __forceinline__ void trace_event(int& n, int base, int code) {
+constexpr int TRACE_CTAS = 256;
+__device__ __forceinline__ void trace_event(int& n, int base, int code, int slot) {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   if (g_hylra_trace && n < 255)
-    g_hylra_trace[(size_t)blockIdx.x * TRACE_PER_CTA + base + n] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
+    g_hylra_trace[((size_t)slot * TRACE_CTAS + blockIdx.x) * TRACE_PER_CTA + base + n] =
+        ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
   ++n;
 }
-#define HYLRA_TRACE_EV(n, base, code) trace_event(n, base, code)
+#define HYLRA_TRACE_EV(n, base, code) trace_event(n, base, code, p.trace_slot)
+__device__ __forceinline__ void trace_event_cta(int& n, int cta, int code, int slot) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  if (g_hylra_trace && n < 255 && cta < TRACE_CTAS)
+    g_hylra_trace[((size_t)slot * TRACE_CTAS + cta) * TRACE_PER_CTA + n] =
+        ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
+  ++n;
+}
+#define HYLRA_TRACE_CTA(n, cta, code) trace_event_cta(n, cta, code, p.trace_slot)
 #else
+#define HYLRA_TRACE_CTA(n, cta, code) ((void)0)
 #define HYLRA_TRACE_EV(n, base, code) ((void)0)
 #endif
 
@@ -96,6 +108,8 @@ struct Params {
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
   int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
+  int upc, nst;      // cluster reuse kernel: blocks per CTA, pipeline stages
+  int trace_slot;    // trace builds: which per-launch region of the trace buffer
   float scale_log2;  // log2(e) / sqrt(d)
 };
 
@@ -115,12 +129,13 @@ __device__ __forceinline__ bool meta_sane(const Params& p, const StageMeta& m) {
          m.ncontrib >= 1 && m.first_slot + m.ncontrib <= nslots && m.nvalid <= BLK;
 }
 
-struct SmemCommon {
-  float comb_o[NCOMB][GMAX][HD];  // warp states at a segment end; merge/top-k scratch
+struct alignas(16) SmemCommon {
+  alignas(16) float comb_o[NCOMB][GMAX][HD];  // warp states at a segment end; merge/top-k scratch
   float comb_m[NWMAX][GMAX];
   float comb_z[NWMAX][GMAX];
   float mg[GMAX];
   float zg[GMAX];
+  float rzg[GMAX];
   float cf[NCOMB][GMAX];  // segment-end scale factors
   int prefix[HYLRA_MAX_BATCH + 1];  // units before sequence b (all heads)
   int hist[256];
@@ -135,6 +150,7 @@ static_assert(sizeof(float) * NCOMB * GMAX * HD >= MAX_NB * 4 + HYLRA_MAX_TOPK *
               "top-k scratch must fit in the combine buffer");
 static_assert(sizeof(float) * NCOMB * GMAX * HD >= 2 * MAX_CTAS * GMAX * 4,
               "merge staging must fit in the combine buffer");
+static_assert(alignof(SmemCommon) == 16, "top-k reads the combine buffer as uint4");
 
 struct SmemBF16 {
   uint8_t stage[NSTAGE][STAGE_BYTES];  // 1024-byte aligned (128-byte swizzle atoms)
@@ -296,14 +312,76 @@ __device__ __forceinline__ int unit_index_entry(const Params& p, const UnitIter&
 // scores, so unsigned order is numeric order): rank order, score descending,
 // lower block index first among equal scores; slots k'..k-1 get -1.
 // Called by the NT merge threads (ct = 0..NT-1).
+//
+// A key "beats" another when it is larger, or equal with a lower index; the
+// answer is the kp keys beaten by fewer than kp others.  Fast path: tau0, the
+// kp-th largest of the per-thread maxima, bounds the kp-th largest key from
+// below (kp threads hold a key >= tau0), so every answer is among the keys
+// >= tau0; ranks among those candidates are their global ranks.  With few
+// candidates (the usual case) they are ranked by pairwise comparison; many
+// equal keys fall back to a radix select.
+constexpr int TOPK_LIST_CAP = (NCOMB * GMAX * HD * 4 - MAX_NB * 4) / 8 - 128;
+
 template <int NT>
 __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int ct) {
   constexpr int NW = NT / 32;
   uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
-  uint2* list = reinterpret_cast<uint2*>(reinterpret_cast<char*>(&c.comb_o[0][0][0]) + MAX_NB * 4);
+  uint32_t* tmax = keys + MAX_NB;                       // NT per-thread maxima
+  uint2* list = reinterpret_cast<uint2*>(tmax + 256);  // candidates (key, block)
   int32_t* dst = p.topk_out + (size_t)bh * p.k;
   const int kp = min(p.k, nb);
   const int lane = ct & 31, wid = ct >> 5;
+
+  bool fast = kp <= NT;
+  if (fast) {
+    uint32_t mx = 0u;
+    for (int beta = ct; beta < nb; beta += NT) mx = max(mx, keys[beta]);
+    tmax[ct] = mx;
+    if (ct == 0) c.misc[3] = 0;
+    named_bar_sync(BAR_CONS, NT);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 20 << 8);
+    // exact rank of this thread's maximum among the NT maxima
+    int rank = 0;
+    const uint4* t4 = reinterpret_cast<const uint4*>(tmax);
+#pragma unroll 4
+    for (int j4 = 0; j4 < NT / 4; ++j4) {
+      const uint4 v = t4[j4];
+      const int j = 4 * j4;
+      rank += (v.x > mx) || (v.x == mx && j < ct);
+      rank += (v.y > mx) || (v.y == mx && j + 1 < ct);
+      rank += (v.z > mx) || (v.z == mx && j + 2 < ct);
+      rank += (v.w > mx) || (v.w == mx && j + 3 < ct);
+    }
+    if (rank == kp - 1) c.misc[1] = (int)mx;
+    named_bar_sync(BAR_CONS, NT);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 21 << 8);
+    const uint32_t tau0 = (uint32_t)c.misc[1];
+    for (int beta = ct; beta < nb; beta += NT) {
+      const uint32_t key = keys[beta];
+      if (key >= tau0) {
+        const int pos = atomicAdd(&c.misc[3], 1);
+        if (pos < TOPK_LIST_CAP) list[pos] = make_uint2(key, (uint32_t)beta);
+      }
+    }
+    named_bar_sync(BAR_CONS, NT);
+    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 22 << 8);
+    const int ncand = c.misc[3];
+    fast = ncand <= TOPK_LIST_CAP;
+    if (fast) {
+      for (int e = ct; e < ncand; e += NT) {
+        const uint2 me = list[e];
+        int r = 0;
+        for (int j = 0; j < ncand; ++j) {
+          const uint2 o = list[j];
+          r += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        }
+        if (r < kp) dst[r] = (int32_t)me.y;
+      }
+      for (int slot = kp + ct; slot < p.k; slot += NT) dst[slot] = -1;
+      return;
+    }
+    named_bar_sync(BAR_CONS, NT);  // everyone has read ncand before it is reused
+  }
 
   // Radix select of the kp-th largest key, 8 bits per pass.
   uint32_t prefix = 0;
@@ -359,6 +437,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
   const uint32_t tau = prefix;  // the kp-th largest score; take `remain` of its copies
 
   // Keep every key above tau and the lowest-index `remain` keys equal to it.
+  uint2* rlist = reinterpret_cast<uint2*>(keys + MAX_NB);
   const int per = (nb + NT - 1) / NT;
   const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
   int eq = 0;
@@ -384,15 +463,15 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     }
     if (sel) {
       const int pos = atomicAdd(&c.misc[3], 1);
-      if (pos < kp) list[pos] = make_uint2(key, (uint32_t)beta);  // exactly kp are selected
+      if (pos < kp) rlist[pos] = make_uint2(key, (uint32_t)beta);  // exactly kp are selected
     }
   }
   named_bar_sync(BAR_CONS, NT);
   for (int e = ct; e < kp; e += NT) {
-    const uint2 me = list[e];
+    const uint2 me = rlist[e];
     int rank = 0;
     for (int j = 0; j < kp; ++j) {
-      const uint2 o = list[j];
+      const uint2 o = rlist[j];
       rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
     }
     dst[rank] = (int32_t)me.y;
@@ -469,6 +548,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
     if (lane == 0) {
       c.mg[g] = M;
       c.zg[g] = Z;
+      c.rzg[g] = Z > 0.f ? 1.f / Z : 0.f;
     }
   }
   named_bar_sync(BAR_CONS, NT);
@@ -530,7 +610,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
 #pragma unroll
       for (int g = 0; g < GMAX; ++g)
         if (g < r && c.zg[g] > 0.f && sv[g].y != -INFINITY)
-          score += sv[g].x * exp2f(sv[g].y - c.mg[g]) / c.zg[g];
+          score += sv[g].x * exp2f(sv[g].y - c.mg[g]) * c.rzg[g];
       uint32_t key = 0u;
       if (isfinite(score)) {
         if (score > 0.f) key = __float_as_uint(score);
@@ -646,6 +726,208 @@ __device__ __forceinline__ void combine_block_record(const float (*bs)[GMAX],
   dst[1] = mm;
 }
 
+// ------------------------------------------------------ consumer warp state
+
+// Online-softmax attention state of one consumer warp of the bf16 kernels:
+// tokens 16*cw .. 16*cw+15 of every block, the r <= 8 q-heads of one KV head.
+// The fragments follow the mma.sync m16n8k16 layouts: this lane holds heads
+// 2*c4 (A) and 2*c4+1 (B), tokens g4 and g4+8 of S^T, and O^T rows
+// (d = 16*dm + g4 [+8]) for those two heads.
+struct WarpAttn {
+  float o[8][4];
+  float m_run[2], z_run[2];
+  uint32_t qf[8][2];
+  int lane, g4, c4, tokw, krow, kchi, vrow, vchi, xr;
+
+  __device__ __forceinline__ void init(int cw, int lane_) {
+    lane = lane_;
+    g4 = lane >> 2;
+    c4 = lane & 3;
+    tokw = cw * 16;
+    const int mi = lane >> 3;
+    // this lane's ldmatrix rows: K (non-transposed) and V (transposed) tiles
+    krow = tokw + (lane & 7) + (mi & 1) * 8;
+    kchi = mi >> 1;
+    vrow = tokw + (lane & 7) + (mi >> 1) * 8;
+    vchi = mi & 1;
+    xr = lane & 7;  // == krow & 7 == vrow & 7
+    reset();
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) qf[kt][0] = qf[kt][1] = 0u;
+  }
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int dm = 0; dm < 8; ++dm)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[dm][e] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    z_run[0] = z_run[1] = 0.f;
+  }
+
+  // q rows [r][128] bf16 in shared memory -> B operand of S^T = K Q^T
+  __device__ __forceinline__ void load_q(const uint8_t* qrows, int r) {
+    const uint32_t* qs = reinterpret_cast<const uint32_t*>(qrows);
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+      qf[kt][0] = g4 < r ? qs[(g4 * HD + kt * 16 + 2 * c4) >> 1] : 0u;
+      qf[kt][1] = g4 < r ? qs[(g4 * HD + kt * 16 + 8 + 2 * c4) >> 1] : 0u;
+    }
+  }
+
+  // One 128-token block in a stage (K at stage, V at stage + 2 boxes).  Waits
+  // for V itself.  Returns the block-local max and probability sum (relative
+  // to that max) of this warp's tokens for heads A and B.
+  __device__ __forceinline__ void block(uint8_t* stage, int nvalid, float scale_log2,
+                                        uint64_t* fullV, uint32_t ph, volatile int* abort_flag,
+                                        float& mxA, float& mxB, float& sA, float& sB) {
+    const uint32_t kbase = smem_u32(stage);
+    const uint32_t vbase = kbase + 2 * BOX_BYTES;
+    const bool partial = nvalid < BLK;
+    float x[4];
+    {  // S^T = K Q^T for this warp's 16 tokens, two accumulation chains
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t kb = kbase + krow * 128;
+#pragma unroll
+      for (int kt = 0; kt < 8; ++kt) {
+        const int ch = 2 * kt + kchi;
+        const uint32_t addr = kb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(addr, r0, r1, r2, r3);
+        mma_bf16_16816((kt & 1) ? a1 : a0, r0, r1, r2, r3, qf[kt][0], qf[kt][1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = (a0[e] + a1[e]) * scale_log2;
+        if (partial) {
+          const int tok = tokw + g4 + ((e & 2) ? 8 : 0);
+          if (tok >= nvalid) v = -INFINITY;
+        }
+        x[e] = v;
+      }
+    }
+    mbar_wait_bounded(fullV, ph, abort_flag);
+    if (partial) {
+      // rows past the sequence end may hold anything (even NaN): zero V
+      for (int idx = lane; idx < 16 * 16; idx += 32) {
+        const int row = tokw + (idx >> 4);
+        if (row < nvalid) continue;
+        const int ch = idx & 15;
+        uint8_t* ptr = stage + 2 * BOX_BYTES + (ch >> 3) * BOX_BYTES + row * 128 + (ch & 7) * 16;
+        *reinterpret_cast<uint4*>(ptr) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+    // block-local max and sums for heads A and B
+    mxA = fmaxf(x[0], x[2]);
+    mxB = fmaxf(x[1], x[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, off));
+      mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, off));
+    }
+    const float msA = mxA == -INFINITY ? 0.f : mxA;
+    const float msB = mxB == -INFINITY ? 0.f : mxB;
+    const float p0 = ex2_approx(x[0] - msA), p1 = ex2_approx(x[1] - msB);
+    const float p2 = ex2_approx(x[2] - msA), p3 = ex2_approx(x[3] - msB);
+    sA = p0 + p2;
+    sB = p1 + p3;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      sA += __shfl_xor_sync(0xffffffffu, sA, off);
+      sB += __shfl_xor_sync(0xffffffffu, sB, off);
+    }
+    // online softmax update (rescale only when a running max moved)
+    const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
+    float alA = 1.f, beA = 0.f, alB = 1.f, beB = 0.f;
+    if (mnA != -INFINITY) {
+      alA = ex2_approx(m_run[0] - mnA);
+      beA = ex2_approx(mxA - mnA);
+    }
+    if (mnB != -INFINITY) {
+      alB = ex2_approx(m_run[1] - mnB);
+      beB = ex2_approx(mxB - mnB);
+    }
+    z_run[0] = z_run[0] * alA + sA * beA;
+    z_run[1] = z_run[1] * alB + sB * beB;
+    m_run[0] = mnA;
+    m_run[1] = mnB;
+    if (__any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        o[dm][0] *= alA;
+        o[dm][1] *= alB;
+        o[dm][2] *= alA;
+        o[dm][3] *= alB;
+      }
+    }
+    // P^T to the B-operand layout, then O^T += V^T P^T
+    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0 * beA, p1 * beB));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2 * beA, p3 * beB));
+    const uint32_t vb = vbase + vrow * 128;
+#pragma unroll
+    for (int dm = 0; dm < 8; ++dm) {
+      const int ch = 2 * dm + vchi;
+      const uint32_t addr = vb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_trans(addr, r0, r1, r2, r3);
+      mma_bf16_16816(o[dm], r0, r1, r2, r3, pb0, pb1);
+    }
+  }
+
+  // Merge the eight warps' states pairwise into comb_*[0..NCOMB) (warps
+  // cw >= NCOMB hand theirs to warp cw - NCOMB).  Called by the NT_BF16
+  // consumer threads together; ends with a barrier.
+  __device__ __forceinline__ void to_comb(SmemCommon& c, int cw) {
+    if (cw >= NCOMB) {
+      const int w = cw - NCOMB;
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        const int d0 = dm * 16 + g4;
+        c.comb_o[w][2 * c4][d0] = o[dm][0];
+        c.comb_o[w][2 * c4 + 1][d0] = o[dm][1];
+        c.comb_o[w][2 * c4][d0 + 8] = o[dm][2];
+        c.comb_o[w][2 * c4 + 1][d0 + 8] = o[dm][3];
+      }
+      if (g4 == 0) {
+        c.comb_m[w][2 * c4] = m_run[0];
+        c.comb_m[w][2 * c4 + 1] = m_run[1];
+        c.comb_z[w][2 * c4] = z_run[0];
+        c.comb_z[w][2 * c4 + 1] = z_run[1];
+      }
+    }
+    named_bar_sync(BAR_CONS, NT_BF16);
+    if (cw < NCOMB) {
+      const float m2A = c.comb_m[cw][2 * c4], m2B = c.comb_m[cw][2 * c4 + 1];
+      const float z2A = c.comb_z[cw][2 * c4], z2B = c.comb_z[cw][2 * c4 + 1];
+      __syncwarp();
+      const float mnA = fmaxf(m_run[0], m2A), mnB = fmaxf(m_run[1], m2B);
+      const float fA = mnA == -INFINITY ? 0.f : ex2_approx(m_run[0] - mnA);
+      const float hA = mnA == -INFINITY ? 0.f : ex2_approx(m2A - mnA);
+      const float fB = mnB == -INFINITY ? 0.f : ex2_approx(m_run[1] - mnB);
+      const float hB = mnB == -INFINITY ? 0.f : ex2_approx(m2B - mnB);
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        const int d0 = dm * 16 + g4;
+        float* a = &c.comb_o[cw][2 * c4][d0];
+        float* b = &c.comb_o[cw][2 * c4 + 1][d0];
+        a[0] = o[dm][0] * fA + a[0] * hA;
+        b[0] = o[dm][1] * fB + b[0] * hB;
+        a[8] = o[dm][2] * fA + a[8] * hA;
+        b[8] = o[dm][3] * fB + b[8] * hB;
+      }
+      if (g4 == 0) {
+        c.comb_m[cw][2 * c4] = mnA;
+        c.comb_m[cw][2 * c4 + 1] = mnB;
+        c.comb_z[cw][2 * c4] = z_run[0] * fA + z2A * hA;
+        c.comb_z[cw][2 * c4 + 1] = z_run[1] * fB + z2B * hB;
+      }
+    }
+    named_bar_sync(BAR_CONS, NT_BF16);
+  }
+};
+
 // ------------------------------------------------------------ bf16 kernel
 
 template <bool FULL>
@@ -688,10 +970,14 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   const int lo = works ? (int)((long long)blockIdx.x * T / G) : 0;
   const int hi = works ? (int)((long long)(blockIdx.x + 1) * T / G) : 0;
   const int n = hi - lo;
-  // Programmatic launch: a thread lets the next kernel in the stream launch
-  // (griddep_launch_dependents) only once it has waited for the preceding
-  // kernel (griddep_wait) or will never touch anything a kernel writes; so
-  // when a kernel runs, every kernel before its predecessor has completed.
+  // Programmatic launch between layers.  Every global write (and a reuse
+  // layer's read of indices its immediate predecessor wrote) comes after
+  // griddep_wait, which returns once the preceding kernel has completed; a
+  // kernel completes only after its own wait, so a kernel never overlaps more
+  // than its predecessor's tail.  A CTA lets the next kernel launch as soon
+  // as any of its threads executes griddep_launch_dependents, so the kernel
+  // right after a reset layer (idx_wait) triggers only after its wait: later
+  // reuse layers then read that reset layer's indices without waiting.
   write_empty_outputs<FULL>(p, c);
   volatile int* abort_flag = &c.misc[4];
 
@@ -764,29 +1050,13 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   // -------------------------------------------------------------- consumers
   const int cw = warp - 1;   // 0..7: tokens 16*cw .. 16*cw+15 of every block
   const int ct = tid - 32;
-  const int g4 = lane >> 2, c4 = lane & 3;
-  const int tokw = cw * 16;
-  const int mi = lane >> 3;
-  float o[8][4];
-  float m_run[2], z_run[2];
-  uint32_t qf[8][2];
-#pragma unroll
-  for (int dm = 0; dm < 8; ++dm)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[dm][e] = 0.f;
-  m_run[0] = m_run[1] = -INFINITY;
-  z_run[0] = z_run[1] = 0.f;
-#pragma unroll
-  for (int kt = 0; kt < 8; ++kt) qf[kt][0] = qf[kt][1] = 0u;
-  // this lane's ldmatrix rows: K (non-transposed) and V (transposed) tiles
-  const int krow = tokw + (lane & 7) + (mi & 1) * 8, kchi = mi >> 1;
-  const int vrow = tokw + (lane & 7) + (mi >> 1) * 8, vchi = mi & 1;
-  const int xr = lane & 7;  // == krow & 7 == vrow & 7
+  WarpAttn wa;
+  wa.init(cw, lane);
+  if (FULL || !p.idx_wait) griddep_launch_dependents();  // else the producer does, after its wait
   bool waited = false;  // griddep_wait done (needed before the first global write)
   auto ensure_waited = [&]() {
     if (!waited) {
       griddep_wait();
-      griddep_launch_dependents();
       waited = true;
     }
   };
@@ -799,119 +1069,18 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, (3 << 8) | (i & 0xff));
     const StageMeta m = sm.meta[s];
     if (m.flags & F_SEG_START) {
-#pragma unroll
-      for (int dm = 0; dm < 8; ++dm)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[dm][e] = 0.f;
-      m_run[0] = m_run[1] = -INFINITY;
-      z_run[0] = z_run[1] = 0.f;
-      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm.qslot[s]);
-#pragma unroll
-      for (int kt = 0; kt < 8; ++kt) {
-        // B operand of S^T = K Q^T: (k = d pair 2*c4 [+8], n = q-head g4)
-        qf[kt][0] = g4 < p.r ? qs[(g4 * HD + kt * 16 + 2 * c4) >> 1] : 0u;
-        qf[kt][1] = g4 < p.r ? qs[(g4 * HD + kt * 16 + 8 + 2 * c4) >> 1] : 0u;
-      }
+      wa.reset();
+      wa.load_q(sm.qslot[s], p.r);
     }
     if (m.blk >= 0) {
-      const uint32_t kbase = smem_u32(sm.stage[s]);
-      const uint32_t vbase = kbase + 2 * BOX_BYTES;
-      const bool partial = m.nvalid < BLK;
-      float x[4];
-      // ---- S^T = K Q^T for this warp's 16 tokens, two accumulation chains
-      {
-        float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t kb = kbase + krow * 128;
-#pragma unroll
-        for (int kt = 0; kt < 8; ++kt) {
-          const int ch = 2 * kt + kchi;
-          const uint32_t addr = kb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(addr, r0, r1, r2, r3);
-          mma_bf16_16816((kt & 1) ? a1 : a0, r0, r1, r2, r3, qf[kt][0], qf[kt][1]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = (a0[e] + a1[e]) * p.scale_log2;
-          if (partial) {
-            const int tok = tokw + g4 + ((e & 2) ? 8 : 0);
-            if (tok >= m.nvalid) v = -INFINITY;
-          }
-          x[e] = v;
-        }
-      }
-      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);
-      if (partial) {
-        // rows past the sequence end may hold anything (even NaN): zero V
-        for (int idx = lane; idx < 16 * 16; idx += 32) {
-          const int row = tokw + (idx >> 4);
-          if (row < m.nvalid) continue;
-          const int ch = idx & 15;
-          uint8_t* ptr = sm.stage[s] + 2 * BOX_BYTES + (ch >> 3) * BOX_BYTES + row * 128 + (ch & 7) * 16;
-          *reinterpret_cast<uint4*>(ptr) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      // ---- block-local max and sums for heads 2*c4 (A) and 2*c4+1 (B)
-      float mxA = fmaxf(x[0], x[2]);
-      float mxB = fmaxf(x[1], x[3]);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, off));
-        mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, off));
-      }
-      const float msA = mxA == -INFINITY ? 0.f : mxA;
-      const float msB = mxB == -INFINITY ? 0.f : mxB;
-      const float p0 = ex2_approx(x[0] - msA), p1 = ex2_approx(x[1] - msB);
-      const float p2 = ex2_approx(x[2] - msA), p3 = ex2_approx(x[3] - msB);
-      float sA = p0 + p2, sB = p1 + p3;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        sA += __shfl_xor_sync(0xffffffffu, sA, off);
-        sB += __shfl_xor_sync(0xffffffffu, sB, off);
-      }
-      if (FULL && g4 == 0) {
-        sm.bst_s[s][cw][2 * c4] = sA;
-        sm.bst_s[s][cw][2 * c4 + 1] = sB;
-        sm.bst_m[s][cw][2 * c4] = mxA;
-        sm.bst_m[s][cw][2 * c4 + 1] = mxB;
-      }
-      // ---- online softmax update (rescale only when a running max moved)
-      const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
-      float alA = 1.f, beA = 0.f, alB = 1.f, beB = 0.f;
-      if (mnA != -INFINITY) {
-        alA = ex2_approx(m_run[0] - mnA);
-        beA = ex2_approx(mxA - mnA);
-      }
-      if (mnB != -INFINITY) {
-        alB = ex2_approx(m_run[1] - mnB);
-        beB = ex2_approx(mxB - mnB);
-      }
-      z_run[0] = z_run[0] * alA + sA * beA;
-      z_run[1] = z_run[1] * alB + sB * beB;
-      m_run[0] = mnA;
-      m_run[1] = mnB;
-      if (__any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
-#pragma unroll
-        for (int dm = 0; dm < 8; ++dm) {
-          o[dm][0] *= alA;
-          o[dm][1] *= alB;
-          o[dm][2] *= alA;
-          o[dm][3] *= alB;
-        }
-      }
-      // ---- P^T to the B-operand layout, then O^T += V^T P^T
-      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0 * beA, p1 * beB));
-      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2 * beA, p3 * beB));
-      const uint32_t vb = vbase + vrow * 128;
-#pragma unroll
-      for (int dm = 0; dm < 8; ++dm) {
-        const int ch = 2 * dm + vchi;
-        const uint32_t addr = vb + (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4_trans(addr, r0, r1, r2, r3);
-        mma_bf16_16816(o[dm], r0, r1, r2, r3, pb0, pb1);
+      float mxA, mxB, sA, sB;
+      wa.block(sm.stage[s], m.nvalid, p.scale_log2, &sm.fullV_bar[s], ph, abort_flag, mxA, mxB,
+               sA, sB);
+      if (FULL && wa.g4 == 0) {
+        sm.bst_s[s][cw][2 * wa.c4] = sA;
+        sm.bst_s[s][cw][2 * wa.c4 + 1] = sB;
+        sm.bst_m[s][cw][2 * wa.c4] = mxA;
+        sm.bst_m[s][cw][2 * wa.c4 + 1] = mxB;
       }
     } else {
       mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);  // keep the phase in step
@@ -945,52 +1114,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (m.flags & F_SEG_END) {
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
       ensure_waited();
-      // eight warp states -> four (pairwise), then publish
-      if (cw >= NCOMB) {
-        const int w = cw - NCOMB;
-#pragma unroll
-        for (int dm = 0; dm < 8; ++dm) {
-          const int d0 = dm * 16 + g4;
-          c.comb_o[w][2 * c4][d0] = o[dm][0];
-          c.comb_o[w][2 * c4 + 1][d0] = o[dm][1];
-          c.comb_o[w][2 * c4][d0 + 8] = o[dm][2];
-          c.comb_o[w][2 * c4 + 1][d0 + 8] = o[dm][3];
-        }
-        if (g4 == 0) {
-          c.comb_m[w][2 * c4] = m_run[0];
-          c.comb_m[w][2 * c4 + 1] = m_run[1];
-          c.comb_z[w][2 * c4] = z_run[0];
-          c.comb_z[w][2 * c4 + 1] = z_run[1];
-        }
-      }
-      named_bar_sync(BAR_CONS, NT_BF16);
-      if (cw < NCOMB) {
-        const float m2A = c.comb_m[cw][2 * c4], m2B = c.comb_m[cw][2 * c4 + 1];
-        const float z2A = c.comb_z[cw][2 * c4], z2B = c.comb_z[cw][2 * c4 + 1];
-        __syncwarp();
-        const float mnA = fmaxf(m_run[0], m2A), mnB = fmaxf(m_run[1], m2B);
-        const float fA = mnA == -INFINITY ? 0.f : ex2_approx(m_run[0] - mnA);
-        const float hA = mnA == -INFINITY ? 0.f : ex2_approx(m2A - mnA);
-        const float fB = mnB == -INFINITY ? 0.f : ex2_approx(m_run[1] - mnB);
-        const float hB = mnB == -INFINITY ? 0.f : ex2_approx(m2B - mnB);
-#pragma unroll
-        for (int dm = 0; dm < 8; ++dm) {
-          const int d0 = dm * 16 + g4;
-          float* a = &c.comb_o[cw][2 * c4][d0];
-          float* b = &c.comb_o[cw][2 * c4 + 1][d0];
-          a[0] = o[dm][0] * fA + a[0] * hA;
-          b[0] = o[dm][1] * fB + b[0] * hB;
-          a[8] = o[dm][2] * fA + a[8] * hA;
-          b[8] = o[dm][3] * fB + b[8] * hB;
-        }
-        if (g4 == 0) {
-          c.comb_m[cw][2 * c4] = mnA;
-          c.comb_m[cw][2 * c4 + 1] = mnB;
-          c.comb_z[cw][2 * c4] = z_run[0] * fA + z2A * hA;
-          c.comb_z[cw][2 * c4 + 1] = z_run[1] * fB + z2B * hB;
-        }
-      }
-      named_bar_sync(BAR_CONS, NT_BF16);
+      wa.to_comb(c, cw);  // eight warp states -> four
       store_partial<NT_BF16>(p, c, m, ct);
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 6 << 8);
       if (c.nseg == MAX_SEGS) flush_segments<FULL, NT_BF16>(p, c, ct);
@@ -1004,6 +1128,266 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   }
   if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 9 << 8);
   if (*abort_flag && ct == 0) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------- cluster reuse kernel
+//
+// Reuse layers touch only k' blocks per (sequence, KV head), too little data
+// to hide a cross-CTA merge through global memory.  Here the CTAs sharing a
+// (b, h) form one thread-block cluster (grid = cluster size x B*Hkv): CTA
+// `rank` takes blocks rank*upc .. rank*upc+upc-1 of the index list, keeps
+// its merged state in its own shared memory, and after a cluster barrier
+// rank 0 reads every CTA's state through distributed shared memory, merges
+// and writes the output.  No workspace, fence or ticket is involved.
+
+constexpr int NST_MAX_RC = 3;
+
+struct SmemRC {
+  uint8_t qbuf[QSLOT_BYTES];
+  int meta_blk[NST_MAX_RC];
+  int meta_nvalid[NST_MAX_RC];
+  alignas(8) uint64_t fullK_bar[NST_MAX_RC];
+  alignas(8) uint64_t fullV_bar[NST_MAX_RC];
+  alignas(8) uint64_t empty_bar[NST_MAX_RC];
+  alignas(16) float part[SLOT_FLOATS];  // this CTA's merged state: O[8][128], m[8], Z[8]
+  SmemCommon c;
+};
+constexpr size_t RC_FIXED_BYTES = (sizeof(SmemRC) + 1023) / 1024 * 1024;
+
+__host__ __device__ constexpr size_t rc_smem_bytes(int nst) {
+  return RC_FIXED_BYTES + (size_t)nst * STAGE_BYTES;
+}
+
+__global__ void __launch_bounds__(NTHR_BF16, 1)
+    decode_reuse_cluster_kernel(const __grid_constant__ CUtensorMap tmK,
+                                const __grid_constant__ CUtensorMap tmV,
+                                const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  SmemRC& sm = *reinterpret_cast<SmemRC*>(base);
+  uint8_t* stages = base + RC_FIXED_BYTES;
+  SmemCommon& c = sm.c;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int CS = (int)gridDim.x;
+  const uint32_t rank = cluster_ctarank();
+  const int bh = (int)blockIdx.y;
+  const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+  const int nst = p.nst, upc = p.upc;
+
+  if (tid == 0) {
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(&sm.fullK_bar[s], 1);
+      mbar_init(&sm.fullV_bar[s], 1);
+      mbar_init(&sm.empty_bar[s], NW_BF16);
+    }
+    c.misc[4] = 0;
+    fence_mbar_init();
+  }
+  if (tid == 32) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  __syncthreads();
+  volatile int* abort_flag = &c.misc[4];
+  const int seqlen = valid_seqlen(p, b, rank == 0 && h == 0 && tid == 0);
+  const int nb = (seqlen + BLK - 1) / BLK;
+  const int kp = min(p.k, nb);
+  const int j0 = (int)rank * upc;
+  const int nu = max(0, min(upc, kp - j0));  // blocks of this CTA
+  const int tcta = bh * CS + (int)rank;
+  int tn = 0;
+  (void)tn;
+  (void)tcta;
+  if (tid == 32) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    HYLRA_TRACE_CTA(tn, tcta, (1 << 8) | (smid & 0xff));
+  }
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      if (p.idx_wait) griddep_wait();  // indices written by the preceding kernel
+      griddep_launch_dependents();     // the producer writes nothing
+      int tp = 128;
+      (void)tp;
+      HYLRA_TRACE_CTA(tp, tcta, 2 << 8);
+      const uint64_t pol = l2_evict_first_policy();
+      const long long row0 = row_base(p, b, h);
+      const uint32_t qbytes = (uint32_t)(p.r * HD * 2);
+      const int32_t* idx = p.topk_in + (size_t)bh * p.k + j0;
+      int blk_next = nu > 0 ? __ldcg(idx) : -1;
+      for (int i = 0; i < nu; ++i) {
+        const int s = i % nst;
+        const uint32_t ph = (uint32_t)((i / nst) & 1);
+        int blk = blk_next;
+        if (i + 1 < nu) blk_next = __ldcg(idx + i + 1);
+        mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
+        if (blk < 0 || blk >= nb) {
+          if (blk != -1) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
+          blk = -1;
+        }
+        sm.meta_blk[s] = blk;
+        sm.meta_nvalid[s] = blk >= 0 ? min(BLK, seqlen - blk * BLK) : 0;
+        uint32_t bytesK = (i == 0 ? qbytes : 0u) + (blk >= 0 ? 2u * BOX_BYTES : 0u);
+        uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
+        if (*abort_flag) bytesK = bytesV = 0u;
+        uint8_t* st = stages + (size_t)s * STAGE_BYTES;
+        const int row = (int)(row0 + (long long)blk * BLK);
+        if (bytesK) {
+          mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
+          if (i == 0)
+            bulk_load(sm.qbuf,
+                      static_cast<const uint8_t*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.r) * HD * 2,
+                      qbytes, &sm.fullK_bar[s]);
+          if (blk >= 0) {
+            tma_load_2d(st, &tmK, 0, row, &sm.fullK_bar[s], pol);
+            tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.fullK_bar[s], pol);
+          }
+        } else {
+          mbar_arrive(&sm.fullK_bar[s]);
+        }
+        if (bytesV) {
+          mbar_arrive_expect_tx(&sm.fullV_bar[s], bytesV);
+          tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.fullV_bar[s], pol);
+          tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.fullV_bar[s], pol);
+        } else {
+          mbar_arrive(&sm.fullV_bar[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int cw = warp - 1;
+    const int ct = tid - 32;
+    // consumers write nothing before rank 0's griddep_wait; with idx_wait the
+    // producer triggers, after its own wait
+    if (!p.idx_wait) griddep_launch_dependents();
+    WarpAttn wa;
+    wa.init(cw, lane);
+    for (int i = 0; i < nu; ++i) {
+      const int s = i % nst;
+      const uint32_t ph = (uint32_t)((i / nst) & 1);
+      mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
+      if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
+      if (i == 0) wa.load_q(sm.qbuf, p.r);
+      const int blk = sm.meta_blk[s];
+      if (blk >= 0) {
+        float mxA, mxB, sA, sB;
+        wa.block(stages + (size_t)s * STAGE_BYTES, sm.meta_nvalid[s], p.scale_log2,
+                 &sm.fullV_bar[s], ph, abort_flag, mxA, mxB, sA, sB);
+      } else {
+        mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
+    }
+    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
+    // this CTA's state: eight warps -> four -> one (into sm.part)
+    wa.to_comb(c, cw);
+    if (ct < p.r) {
+      const int g = ct;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NCOMB; ++w) M = fmaxf(M, c.comb_m[w][g]);
+      float Z = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCOMB; ++w) {
+        const float mw = c.comb_m[w][g];
+        const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        c.cf[w][g] = f;
+        Z += c.comb_z[w][g] * f;
+      }
+      sm.part[GMAX * HD + g] = M;
+      sm.part[GMAX * HD + GMAX + g] = Z;
+    }
+    named_bar_sync(BAR_CONS, NT_BF16);
+    for (int pr = ct; pr < p.r * HD; pr += NT_BF16) {
+      const int g = pr / HD, d = pr - g * HD;
+      float O = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCOMB; ++w) O = fmaf(c.comb_o[w][g][d], c.cf[w][g], O);
+      sm.part[g * HD + d] = O;
+    }
+  }
+  __syncwarp();
+  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
+  cluster_sync_all();  // every CTA's state is in its shared memory
+  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 6 << 8);
+
+  if (rank == 0 && warp > 0) {
+    // ------------------------------------------------- merge (CTA rank 0)
+    const int ct = tid - 32;
+    const int r = p.r;
+    const int cl = ct & 31, wid = ct >> 5;
+    const uint32_t part0 = smem_u32(sm.part);
+    float* fm = &c.comb_o[0][0][0];     // [CS][GMAX]: maxima, then scale factors
+    float* fz = fm + MAX_CTAS * GMAX;   // [CS][GMAX]: sums
+    for (int e = ct; e < CS * r; e += NT_BF16) {
+      const int j = e / r, g = e - j * r;
+      const uint32_t a = mapa_shared(part0, (uint32_t)j);
+      fm[j * GMAX + g] = ld_dsmem_f32(a + (GMAX * HD + g) * 4);
+      fz[j * GMAX + g] = ld_dsmem_f32(a + (GMAX * HD + GMAX + g) * 4);
+    }
+    named_bar_sync(BAR_CONS, NT_BF16);
+    for (int g = wid; g < r; g += NW_BF16) {
+      float M = -INFINITY;
+      for (int j = cl; j < CS; j += 32) M = fmaxf(M, fm[j * GMAX + g]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      float Z = 0.f;
+      for (int j = cl; j < CS; j += 32) {
+        const float mj = fm[j * GMAX + g];
+        const float f = (M == -INFINITY || mj == -INFINITY) ? 0.f : exp2f(mj - M);
+        Z += fz[j * GMAX + g] * f;
+        fm[j * GMAX + g] = f;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+      if (cl == 0) c.zg[g] = Z;
+    }
+    named_bar_sync(BAR_CONS, NT_BF16);
+    griddep_wait();  // the preceding kernel has completed before out is written
+    for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
+      const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
+      float2 acc = make_float2(0.f, 0.f);
+      float2 v[16];  // every cluster CTA's value, all loads in flight together
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < CS) v[j] = ld_dsmem_f32x2(mapa_shared(part0, (uint32_t)j) + (g * HD + col) * 4);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j < CS) {
+          const float f = fm[j * GMAX + g];
+          acc.x = fmaf(v[j].x, f, acc.x);
+          acc.y = fmaf(v[j].y, f, acc.y);
+        }
+      }
+      const float Z = c.zg[g];
+      float2 o = make_float2(0.f, 0.f);
+      if (Z > 0.f) o = make_float2(acc.x / Z, acc.y / Z);
+      *reinterpret_cast<float2*>(p.out + ((size_t)b * p.Hq + (size_t)h * r + g) * HD + col) = o;
+    }
+    // a reused list naming one block twice counts that block twice: flag it
+    named_bar_sync(BAR_CONS, NT_BF16);  // scale factors no longer needed
+    int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
+    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+    for (int e = ct; e < kp; e += NT_BF16) sidx[e] = __ldcg(idx + e);
+    named_bar_sync(BAR_CONS, NT_BF16);
+    bool dup = false;
+    for (int e = ct; e < kp; e += NT_BF16) {
+      const int32_t v = sidx[e];
+      if (v < 0) continue;
+      for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
+    }
+    if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
+  }
+  __syncwarp();
+  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 7 << 8);
+  cluster_sync_all();  // keep every CTA's shared memory alive until rank 0 is done
+  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 9 << 8);
+  if (*abort_flag && tid == 32) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
 }
 
 // ------------------------------------------------------------ fp32 kernel

@@ -222,6 +222,24 @@ def test_equal_scores_pick_lowest_indices():
     assert np.all(tk[0] == np.arange(6))
 
 
+def test_many_equal_scores_take_the_radix_path():
+    """1000 blocks of equal mass: more candidates than the fast selection
+    keeps, so the radix select runs; ranks must follow block index."""
+    w = W.custom("ties_many", batch=1, seqlens=(128 * 1000,), num_q_heads=8, num_kv_heads=2,
+                 topk=20, seed=25)
+    q, K, V = _layer(w)
+    K = torch.zeros_like(K)
+    _, _, _, tk, _ = _full_and_check(w, inputs=(q, K, V))
+    assert np.all(tk[0] == np.arange(20))
+
+
+def test_k_larger_than_the_merge_thread_count():
+    """k = 300 > 256 selection threads: the radix select path."""
+    w = W.custom("bigk", batch=1, seqlens=(128 * 400 - 17,), num_q_heads=8, num_kv_heads=2,
+                 topk=300, structure="iid", seed=26)
+    _full_and_check(w)
+
+
 def test_invalid_seqlen_is_flagged_not_faulted():
     w = W.custom("badlen", batch=2, seqlens=(300, 300), num_q_heads=8, num_kv_heads=2, topk=3,
                  seed=20)
