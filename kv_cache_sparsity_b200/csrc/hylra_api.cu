@@ -194,10 +194,11 @@ int rc_max_active(int cs, int nst) {
   return v;
 }
 
-// A small reuse layer (fewer blocks than SMs) is latency-bound: it takes at
-// most half the SMs so that, launched as a programmatic dependent, the next
-// layer's CTAs are resident and loading while this one finishes.  A large one
-// spreads over every SM.  Each CTA holds a whole SM (registers).
+// A small reuse layer (fewer blocks than SMs) is latency-bound: its clusters
+// take at most half of the CTA slots, so that, launched as a programmatic
+// dependent, the next layer's CTAs are resident, loading and computing while
+// this one finishes (a CTA with one pipeline stage leaves room for two per
+// SM).  A large layer spreads over every SM.
 bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
   const int nbmax = std::max(1, (s->max_seqlen + BLK - 1) / BLK);
   const int kmax = std::max(1, std::min(s->topk, nbmax));
@@ -208,8 +209,18 @@ bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
   const bool small = (long long)nbh * kmax <= sms;
-  const int budget = small ? sms / 2 : sms;
-  const int cs_max = std::max(1, std::min(std::min(16, kmax), budget / std::max(1, nbh)));
+  if (small) {
+    // room for two layers' clusters at once (the next layer's CTAs load and
+    // compute while this one finishes), the largest clusters first
+    for (int cs = std::min(16, kmax); cs >= 1; --cs) {
+      const RCPlan pl = rc_plan_for(cs, kmax);
+      if (rc_max_active(cs, pl.nst) >= 2 * nbh) {
+        *out = pl;
+        return true;
+      }
+    }
+  }
+  const int cs_max = std::max(1, std::min(std::min(16, kmax), sms / std::max(1, nbh)));
   for (int cs = cs_max; cs >= 1; --cs) {
     const RCPlan pl = rc_plan_for(cs, kmax);
     const int n = rc_max_active(cs, pl.nst);
@@ -323,6 +334,18 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     const cudaError_t e = full ? cudaLaunchKernelEx(&cfg, decode_bf16_kernel<true>, tmK, tmV, p)
                                : cudaLaunchKernelEx(&cfg, decode_bf16_kernel<false>, tmK, tmV, p);
     if (e != cudaSuccess) return HYLRA_ERR_CUDA;
+    // the cross-CTA merge (and top-k) as the streaming kernel's dependent
+    cudaLaunchConfig_t mcfg = {};
+    mcfg.gridDim = dim3(s->batch * s->num_kv_heads);
+    mcfg.blockDim = dim3(NT_BF16);
+    mcfg.dynamicSmemBytes = 0;
+    mcfg.stream = stream;
+    mcfg.attrs = attr;
+    mcfg.numAttrs = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
+                                : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
+    if (em != cudaSuccess) return HYLRA_ERR_CUDA;
   } else {
     if (full)
       decode_f32_kernel<true><<<G, NT_F32, 0, stream>>>(p);

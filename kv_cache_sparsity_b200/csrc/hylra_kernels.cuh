@@ -314,12 +314,14 @@ __device__ __forceinline__ int unit_index_entry(const Params& p, const UnitIter&
 // Called by the NT merge threads (ct = 0..NT-1).
 //
 // A key "beats" another when it is larger, or equal with a lower index; the
-// answer is the kp keys beaten by fewer than kp others.  Fast path: tau0, the
-// kp-th largest of the per-thread maxima, bounds the kp-th largest key from
-// below (kp threads hold a key >= tau0), so every answer is among the keys
-// >= tau0; ranks among those candidates are their global ranks.  With few
-// candidates (the usual case) they are ranked by pairwise comparison; many
-// equal keys fall back to a radix select.
+// answer is the kp keys beaten by fewer than kp others.  Fast path (kp <= 32):
+// each warp sorts its 32 per-thread maxima (bitonic network over shuffles);
+// its kp-th largest is a value that kp of its keys reach, so tau0, the
+// largest of these over the warps, bounds the kp-th largest key from below
+// and every answer is among the keys >= tau0, whose ranks among those
+// candidates are their global ranks.  With few candidates (the usual case)
+// they are ranked by pairwise comparison; otherwise (many equal keys, or
+// kp > 32) a radix select runs.
 constexpr int TOPK_LIST_CAP = (NCOMB * GMAX * HD * 4 - MAX_NB * 4) / 8 - 128;
 
 template <int NT>
@@ -332,30 +334,26 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
   const int kp = min(p.k, nb);
   const int lane = ct & 31, wid = ct >> 5;
 
-  bool fast = kp <= NT;
+  bool fast = kp <= 32;
   if (fast) {
-    uint32_t mx = 0u;
-    for (int beta = ct; beta < nb; beta += NT) mx = max(mx, keys[beta]);
-    tmax[ct] = mx;
+    uint32_t v = 0u;
+    for (int beta = ct; beta < nb; beta += NT) v = max(v, keys[beta]);
+    // descending bitonic sort of the warp's 32 per-thread maxima
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+        v = (((lane & j) == 0) == ((lane & k) == 0)) ? max(v, o) : min(v, o);
+      }
+    }
+    if (lane == kp - 1) tmax[wid] = v;
     if (ct == 0) c.misc[3] = 0;
     named_bar_sync(BAR_CONS, NT);
     if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 20 << 8);
-    // exact rank of this thread's maximum among the NT maxima
-    int rank = 0;
-    const uint4* t4 = reinterpret_cast<const uint4*>(tmax);
-#pragma unroll 4
-    for (int j4 = 0; j4 < NT / 4; ++j4) {
-      const uint4 v = t4[j4];
-      const int j = 4 * j4;
-      rank += (v.x > mx) || (v.x == mx && j < ct);
-      rank += (v.y > mx) || (v.y == mx && j + 1 < ct);
-      rank += (v.z > mx) || (v.z == mx && j + 2 < ct);
-      rank += (v.w > mx) || (v.w == mx && j + 3 < ct);
-    }
-    if (rank == kp - 1) c.misc[1] = (int)mx;
-    named_bar_sync(BAR_CONS, NT);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 21 << 8);
-    const uint32_t tau0 = (uint32_t)c.misc[1];
+    uint32_t tau0 = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) tau0 = max(tau0, tmax[w]);
     for (int beta = ct; beta < nb; beta += NT) {
       const uint32_t key = keys[beta];
       if (key >= tau0) {
@@ -482,36 +480,21 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
 // ---------------------------------------------------------------- merging
 
 // The last CTA of (b, h): LSE-merge every contributor's partial into out;
-// on reset layers also score the blocks and select the top-k.  Loads that do
-// not depend on one another are issued together: the merge sits on the
-// kernel's tail, so it is one L2 round trip plus shared-memory work.
+// on reset layers also score the blocks and select the top-k.  The merge
+// sits on the kernel's tail, so it is one L2 round trip: every thread loads
+// the (max, sum, row) of its contributors together and merges them online;
+// the NT threads split into G groups over the contributors, combined once
+// through shared memory.
 template <bool FULL, int NT>
 __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
-  constexpr int NW = NT / 32;
-  constexpr int OB = 24;  // contributors per batch of output-row loads
+  constexpr int CB = 10;  // contributors per thread and batch of loads
   const int bh = m.b * p.Hkv + m.h;
   const int nc = m.ncontrib;
   const int r = p.r;
-  const int lane = ct & 31, wid = ct >> 5;
-  float* fm = &c.comb_o[0][0][0];     // [nc][GMAX]: maxima, then scale factors
-  float* fz = fm + MAX_CTAS * GMAX;   // [nc][GMAX]: sums
   const float* pbase = p.partials + (size_t)m.first_slot * SLOT_FLOATS;
   const int kp = min(p.k, m.nb);
   const int32_t* idx = p.topk_in + (size_t)bh * p.k;
   const int32_t my_idx = (!FULL && ct < kp) ? __ldcg(idx + ct) : -1;
-
-  // Output columns of this thread: pairs (g, 2 columns); r*64 pairs in all.
-  const int npairs = r * (HD / 2);
-  const int pr0 = ct;
-  const bool has0 = pr0 < npairs;
-  const int g0 = has0 ? pr0 / (HD / 2) : 0, col0 = 2 * (pr0 % (HD / 2));
-  float2 v0[OB];
-#pragma unroll
-  for (int u = 0; u < OB; ++u) {
-    v0[u] = make_float2(0.f, 0.f);
-    if (has0 && u < nc)
-      v0[u] = __ldcg(reinterpret_cast<const float2*>(pbase + (size_t)u * SLOT_FLOATS + g0 * HD + col0));
-  }
   // block records of the first block of this thread (reset layers)
   float2 sv0[GMAX];
 #pragma unroll
@@ -521,77 +504,86 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
       sv0[g] = __ldcg(reinterpret_cast<const float2*>(
           p.bstat + ((size_t)bh * p.nbmax + ct) * (2 * r) + 2 * g));
   }
-  for (int e = ct; e < nc * r; e += NT) {
-    const int j = e / r, g = e - j * r;
-    const float* sl = pbase + (size_t)j * SLOT_FLOATS + GMAX * HD;
-    const float mv = __ldcg(sl + g), zv = __ldcg(sl + GMAX + g);
-    fm[j * GMAX + g] = mv;
-    fz[j * GMAX + g] = zv;
+
+  const int ncol = r * (HD / 4);             // float4 output columns
+  const int G = ncol >= NT ? 1 : NT / ncol;  // contributor groups
+  float4* red = reinterpret_cast<float4*>(&c.comb_o[0][0][0]);  // [G][ncol]
+  for (int t = ct; t < G * ncol; t += NT) {
+    const int q = t / ncol, col = t - q * ncol;
+    const int g = col / (HD / 4), d4 = col - g * (HD / 4);
+    float M = -INFINITY, Z = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = q; j0 < nc; j0 += G * CB) {
+      float mv[CB], zv[CB];
+      float4 ov[CB];
+#pragma unroll
+      for (int u = 0; u < CB; ++u) {
+        const int j = j0 + u * G;
+        mv[u] = -INFINITY;
+        if (j < nc) {
+          const float* sl = pbase + (size_t)j * SLOT_FLOATS;
+          mv[u] = __ldcg(sl + GMAX * HD + g);
+          zv[u] = __ldcg(sl + GMAX * HD + GMAX + g);
+          ov[u] = __ldcg(reinterpret_cast<const float4*>(sl + g * HD + 4 * d4));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < CB; ++u) {
+        if (mv[u] == -INFINITY) continue;
+        if (mv[u] > M) {
+          const float f = M == -INFINITY ? 0.f : ex2_approx(M - mv[u]);
+          acc.x *= f;
+          acc.y *= f;
+          acc.z *= f;
+          acc.w *= f;
+          Z *= f;
+          M = mv[u];
+        }
+        const float f = ex2_approx(mv[u] - M);
+        acc.x = fmaf(ov[u].x, f, acc.x);
+        acc.y = fmaf(ov[u].y, f, acc.y);
+        acc.z = fmaf(ov[u].z, f, acc.z);
+        acc.w = fmaf(ov[u].w, f, acc.w);
+        Z = fmaf(zv[u], f, Z);
+      }
+    }
+    red[t] = acc;
+    if (d4 == 0) {
+      c.comb_m[q][g] = M;
+      c.comb_z[q][g] = Z;
+    }
   }
   named_bar_sync(BAR_CONS, NT);
-  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 10 << 8);
-  // per head (one warp each): global max, global sum, per-contributor factor
-  for (int g = wid; g < r; g += NW) {
+  for (int col = ct; col < ncol; col += NT) {
+    const int g = col / (HD / 4), d4 = col - g * (HD / 4);
     float M = -INFINITY;
-    for (int j = lane; j < nc; j += 32) M = fmaxf(M, fm[j * GMAX + g]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int q = 0; q < G; ++q) M = fmaxf(M, c.comb_m[q][g]);
     float Z = 0.f;
-    for (int j = lane; j < nc; j += 32) {
-      const float mj = fm[j * GMAX + g];
-      const float f = (M == -INFINITY || mj == -INFINITY) ? 0.f : exp2f(mj - M);
-      Z += fz[j * GMAX + g] * f;
-      fm[j * GMAX + g] = f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int q = 0; q < G; ++q) {
+        const float mq = c.comb_m[q][g];
+        if (mq == -INFINITY) continue;
+        const float f = ex2_approx(mq - M);
+        const float4 v = red[q * ncol + col];
+        acc.x = fmaf(v.x, f, acc.x);
+        acc.y = fmaf(v.y, f, acc.y);
+        acc.z = fmaf(v.z, f, acc.z);
+        acc.w = fmaf(v.w, f, acc.w);
+        Z = fmaf(c.comb_z[q][g], f, Z);
+      }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
-    if (lane == 0) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (Z > 0.f) o = make_float4(acc.x / Z, acc.y / Z, acc.z / Z, acc.w / Z);
+    *reinterpret_cast<float4*>(p.out + ((size_t)m.b * p.Hq + (size_t)m.h * r + g) * HD + 4 * d4) = o;
+    if (d4 == 0) {
       c.mg[g] = M;
       c.zg[g] = Z;
       c.rzg[g] = Z > 0.f ? 1.f / Z : 0.f;
     }
   }
-  named_bar_sync(BAR_CONS, NT);
-  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 11 << 8);
-  // output rows
-  for (int pr = ct; pr < npairs; pr += NT) {
-    const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
-    float2 acc = make_float2(0.f, 0.f);
-    int j = 0;
-    if (pr == pr0) {
-#pragma unroll
-      for (int u = 0; u < OB; ++u) {
-        if (u < nc) {
-          const float f = fm[u * GMAX + g];
-          acc.x = fmaf(v0[u].x, f, acc.x);
-          acc.y = fmaf(v0[u].y, f, acc.y);
-        }
-      }
-      j = OB;
-    }
-    for (; j < nc; j += OB) {
-      float2 v[OB];
-#pragma unroll
-      for (int u = 0; u < OB; ++u)
-        v[u] = (j + u < nc) ? __ldcg(reinterpret_cast<const float2*>(
-                                  pbase + (size_t)(j + u) * SLOT_FLOATS + g * HD + col))
-                            : make_float2(0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < OB; ++u) {
-        if (j + u < nc) {
-          const float f = fm[(j + u) * GMAX + g];
-          acc.x = fmaf(v[u].x, f, acc.x);
-          acc.y = fmaf(v[u].y, f, acc.y);
-        }
-      }
-    }
-    const float Z = c.zg[g];
-    float2 o = make_float2(0.f, 0.f);
-    if (Z > 0.f) o = make_float2(acc.x / Z, acc.y / Z);
-    *reinterpret_cast<float2*>(p.out + ((size_t)m.b * p.Hq + (size_t)m.h * r + g) * HD + col) = o;
-  }
   if (FULL) {
-    named_bar_sync(BAR_CONS, NT);  // factors (comb_o) no longer needed
+    named_bar_sync(BAR_CONS, NT);  // head maxima and sums visible; comb_o free
     uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
     bool nonfinite = false;
     for (int beta = ct; beta < m.nb; beta += NT) {
@@ -626,7 +618,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
     if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 13 << 8);
   } else {
     // a reused list naming one block twice counts that block twice: flag it
-    named_bar_sync(BAR_CONS, NT);  // factors (comb_o) no longer needed
+    named_bar_sync(BAR_CONS, NT);  // comb_o free
     int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
     for (int e = ct; e < kp; e += NT) sidx[e] = e == ct ? my_idx : __ldcg(idx + e);
     named_bar_sync(BAR_CONS, NT);
@@ -646,7 +638,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
 // share of (b, h).  Merge them and store the CTA's partial (no fence: the
 // ticket that makes it visible is taken later, in flush_segments), and queue
 // the segment.  Ends with a barrier (comb_* may be rewritten afterwards).
-template <int NT>
+template <int NT, bool QUEUE>
 __device__ void store_partial(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
   const bool sane = meta_sane(p, m);
   float* slot = p.partials + (size_t)(sane ? m.seg_slot : 0) * SLOT_FLOATS;
@@ -675,7 +667,7 @@ __device__ void store_partial(const Params& p, SmemCommon& c, const StageMeta& m
       for (int w = 0; w < NCOMB; ++w) O = fmaf(c.comb_o[w][g][d], c.cf[w][g], O);
       slot[g * HD + d] = O;
     }
-    if (ct == 0) c.segs[c.nseg++] = m;
+    if (QUEUE && ct == 0) c.segs[c.nseg++] = m;
   }
   named_bar_sync(BAR_CONS, NT);
 }
@@ -978,7 +970,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   // as any of its threads executes griddep_launch_dependents, so the kernel
   // right after a reset layer (idx_wait) triggers only after its wait: later
   // reuse layers then read that reset layer's indices without waiting.
-  write_empty_outputs<FULL>(p, c);
+  // Sequences without units get their outputs from merge_kernel.
   volatile int* abort_flag = &c.misc[4];
 
   if (warp == 0) {
@@ -1115,19 +1107,65 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
       ensure_waited();
       wa.to_comb(c, cw);  // eight warp states -> four
-      store_partial<NT_BF16>(p, c, m, ct);
+      store_partial<NT_BF16, false>(p, c, m, ct);  // merged by merge_kernel
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 6 << 8);
-      if (c.nseg == MAX_SEGS) flush_segments<FULL, NT_BF16>(p, c, ct);
     }
   }
-  if (n > 0) {
-    ensure_waited();
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 7 << 8);
-    flush_segments<FULL, NT_BF16>(p, c, ct);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 8 << 8);
-  }
+  // every CTA waits once, so that this kernel completes only after its
+  // predecessor (later kernels rely on that ordering without waiting)
+  ensure_waited();
   if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 9 << 8);
   if (*abort_flag && ct == 0) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------ merge kernel
+//
+// Runs after decode_bf16_kernel (as its programmatic dependent): one CTA per
+// (sequence, KV head) merges the partials of that head's contributors, and
+// on reset layers scores the blocks and selects the top-k.  The kernel
+// boundary makes the partials visible; no fence or ticket is needed.
+template <bool FULL>
+__global__ void __launch_bounds__(NT_BF16, 1) merge_kernel(const __grid_constant__ Params p,
+                                                           int grid_stream) {
+  __shared__ SmemCommon c;
+  const int ct = threadIdx.x;
+  const int bh = (int)blockIdx.x;
+  const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+  int tn = 0;
+  (void)tn;
+  if (ct == 0) {
+    c.trace_n = 255;  // merge_bh's own trace points are off here
+    HYLRA_TRACE_CTA(tn, 160 + bh, 30 << 8);
+  }
+  build_prefix(p, c, FULL);
+  griddep_wait();  // the streaming kernel has completed: partials are visible
+  griddep_launch_dependents();
+  if (ct == 0) HYLRA_TRACE_CTA(tn, 160 + bh, 31 << 8);
+  __syncthreads();
+  const int T = c.prefix[p.B];
+  const int U = (c.prefix[b + 1] - c.prefix[b]) / p.Hkv;
+  if (U == 0) {
+    // a sequence without units: zero output (and no indices)
+    for (int i = ct; i < p.r * HD; i += NT_BF16)
+      p.out[((size_t)b * p.Hq + (size_t)h * p.r) * HD + i] = 0.f;
+    if (FULL)
+      for (int i = ct; i < p.k; i += NT_BF16) p.topk_out[(size_t)bh * p.k + i] = -1;
+    return;
+  }
+  const int G = min(grid_stream, T);
+  const int start = c.prefix[b] + h * U;
+  const int cf = owner_cta(start, T, G);
+  const int cl = owner_cta((long long)start + U - 1, T, G);
+  const int seqlen = valid_seqlen(p, b, false);
+  StageMeta m{};
+  m.b = b;
+  m.h = h;
+  m.blk = 0;
+  m.first_slot = cf + bh;
+  m.ncontrib = cl - cf + 1;
+  m.nb = (seqlen + BLK - 1) / BLK;
+  merge_bh<FULL, NT_BF16>(p, c, m, ct);
+  if (ct == 0) HYLRA_TRACE_CTA(tn, 160 + bh, 32 << 8);
 }
 
 // ------------------------------------------------- cluster reuse kernel
@@ -1150,6 +1188,7 @@ struct SmemRC {
   alignas(8) uint64_t fullV_bar[NST_MAX_RC];
   alignas(8) uint64_t empty_bar[NST_MAX_RC];
   alignas(16) float part[SLOT_FLOATS];  // this CTA's merged state: O[8][128], m[8], Z[8]
+  uint32_t seen[MAX_NB / 32];           // rank 0: blocks named so far (duplicate check)
   SmemCommon c;
 };
 constexpr size_t RC_FIXED_BYTES = (sizeof(SmemRC) + 1023) / 1024 * 1024;
@@ -1158,7 +1197,7 @@ __host__ __device__ constexpr size_t rc_smem_bytes(int nst) {
   return RC_FIXED_BYTES + (size_t)nst * STAGE_BYTES;
 }
 
-__global__ void __launch_bounds__(NTHR_BF16, 1)
+__global__ void __launch_bounds__(NTHR_BF16, 2)
     decode_reuse_cluster_kernel(const __grid_constant__ CUtensorMap tmK,
                                 const __grid_constant__ CUtensorMap tmV,
                                 const __grid_constant__ Params p) {
@@ -1207,8 +1246,23 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    if (p.idx_wait) griddep_wait();  // indices written by the preceding kernel
+    if (rank == 0) {
+      // a reused list naming one block twice counts that block twice: flag it
+      for (int i = lane; i < MAX_NB / 32; i += 32) sm.seen[i] = 0u;
+      __syncwarp();
+      const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+      bool dup = false;
+      for (int e = lane; e < kp; e += 32) {
+        const int32_t v = __ldcg(idx + e);
+        if (v >= 0 && v < nb) {
+          const uint32_t bit = 1u << (v & 31);
+          dup |= (atomicOr(&sm.seen[v >> 5], bit) & bit) != 0u;
+        }
+      }
+      if (__any_sync(0xffffffffu, dup) && lane == 0) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
+    }
     if (lane == 0) {
-      if (p.idx_wait) griddep_wait();  // indices written by the preceding kernel
       griddep_launch_dependents();     // the producer writes nothing
       int tp = 128;
       (void)tp;
@@ -1286,29 +1340,24 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
     // this CTA's state: eight warps -> four -> one (into sm.part)
     wa.to_comb(c, cw);
-    if (ct < p.r) {
-      const int g = ct;
+    for (int pr = ct; pr < p.r * HD; pr += NT_BF16) {
+      const int g = pr / HD, d = pr - g * HD;
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NCOMB; ++w) M = fmaxf(M, c.comb_m[w][g]);
-      float Z = 0.f;
+      float O = 0.f, Z = 0.f;
 #pragma unroll
       for (int w = 0; w < NCOMB; ++w) {
         const float mw = c.comb_m[w][g];
-        const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        c.cf[w][g] = f;
-        Z += c.comb_z[w][g] * f;
+        const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+        O = fmaf(c.comb_o[w][g][d], f, O);
+        Z = fmaf(c.comb_z[w][g], f, Z);
       }
-      sm.part[GMAX * HD + g] = M;
-      sm.part[GMAX * HD + GMAX + g] = Z;
-    }
-    named_bar_sync(BAR_CONS, NT_BF16);
-    for (int pr = ct; pr < p.r * HD; pr += NT_BF16) {
-      const int g = pr / HD, d = pr - g * HD;
-      float O = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCOMB; ++w) O = fmaf(c.comb_o[w][g][d], c.cf[w][g], O);
       sm.part[g * HD + d] = O;
+      if (d == 0) {
+        sm.part[GMAX * HD + g] = M;
+        sm.part[GMAX * HD + GMAX + g] = Z;
+      }
     }
   }
   __syncwarp();
@@ -1318,70 +1367,48 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 
   if (rank == 0 && warp > 0) {
     // ------------------------------------------------- merge (CTA rank 0)
+    // One pass over distributed shared memory: each thread loads, for its
+    // head and two output columns, every CTA's (max, sum, O) at once.
     const int ct = tid - 32;
     const int r = p.r;
-    const int cl = ct & 31, wid = ct >> 5;
     const uint32_t part0 = smem_u32(sm.part);
-    float* fm = &c.comb_o[0][0][0];     // [CS][GMAX]: maxima, then scale factors
-    float* fz = fm + MAX_CTAS * GMAX;   // [CS][GMAX]: sums
-    for (int e = ct; e < CS * r; e += NT_BF16) {
-      const int j = e / r, g = e - j * r;
-      const uint32_t a = mapa_shared(part0, (uint32_t)j);
-      fm[j * GMAX + g] = ld_dsmem_f32(a + (GMAX * HD + g) * 4);
-      fz[j * GMAX + g] = ld_dsmem_f32(a + (GMAX * HD + GMAX + g) * 4);
-    }
-    named_bar_sync(BAR_CONS, NT_BF16);
-    for (int g = wid; g < r; g += NW_BF16) {
-      float M = -INFINITY;
-      for (int j = cl; j < CS; j += 32) M = fmaxf(M, fm[j * GMAX + g]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      float Z = 0.f;
-      for (int j = cl; j < CS; j += 32) {
-        const float mj = fm[j * GMAX + g];
-        const float f = (M == -INFINITY || mj == -INFINITY) ? 0.f : exp2f(mj - M);
-        Z += fz[j * GMAX + g] * f;
-        fm[j * GMAX + g] = f;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
-      if (cl == 0) c.zg[g] = Z;
-    }
-    named_bar_sync(BAR_CONS, NT_BF16);
-    griddep_wait();  // the preceding kernel has completed before out is written
+    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 10 << 8);
     for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
       const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
-      float2 acc = make_float2(0.f, 0.f);
-      float2 v[16];  // every cluster CTA's value, all loads in flight together
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j < CS) v[j] = ld_dsmem_f32x2(mapa_shared(part0, (uint32_t)j) + (g * HD + col) * 4);
+      float2 v[16];
+      float mj[16], zj[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         if (j < CS) {
-          const float f = fm[j * GMAX + g];
+          const uint32_t a = mapa_shared(part0, (uint32_t)j);
+          v[j] = ld_dsmem_f32x2(a + (g * HD + col) * 4);
+          mj[j] = ld_dsmem_f32(a + (GMAX * HD + g) * 4);
+          zj[j] = ld_dsmem_f32(a + (GMAX * HD + GMAX + g) * 4);
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < CS) M = fmaxf(M, mj[j]);
+      float Z = 0.f;
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j < CS) {
+          const float f = (M == -INFINITY || mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - M);
+          Z = fmaf(zj[j], f, Z);
           acc.x = fmaf(v[j].x, f, acc.x);
           acc.y = fmaf(v[j].y, f, acc.y);
         }
       }
-      const float Z = c.zg[g];
       float2 o = make_float2(0.f, 0.f);
       if (Z > 0.f) o = make_float2(acc.x / Z, acc.y / Z);
+      if (pr == ct) {
+        if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 11 << 8);
+        griddep_wait();  // the preceding kernel has completed before out is written
+      }
       *reinterpret_cast<float2*>(p.out + ((size_t)b * p.Hq + (size_t)h * r + g) * HD + col) = o;
     }
-    // a reused list naming one block twice counts that block twice: flag it
-    named_bar_sync(BAR_CONS, NT_BF16);  // scale factors no longer needed
-    int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
-    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
-    for (int e = ct; e < kp; e += NT_BF16) sidx[e] = __ldcg(idx + e);
-    named_bar_sync(BAR_CONS, NT_BF16);
-    bool dup = false;
-    for (int e = ct; e < kp; e += NT_BF16) {
-      const int32_t v = sidx[e];
-      if (v < 0) continue;
-      for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
-    }
-    if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
   }
   __syncwarp();
   if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 7 << 8);
@@ -1528,7 +1555,7 @@ __global__ void __launch_bounds__(NT_F32, 1) decode_f32_kernel(const __grid_cons
         }
       }
       named_bar_sync(BAR_CONS, NT_F32);
-      store_partial<NT_F32>(p, c, m, ct);
+      store_partial<NT_F32, true>(p, c, m, ct);
       if (c.nseg == MAX_SEGS) flush_segments<FULL, NT_F32>(p, c, ct);
     }
   }

@@ -309,6 +309,37 @@ def test_step_in_cuda_graph_matches_eager():
     assert run.status() == 0
 
 
+@pytest.mark.parametrize("policy", [(1, 0, 0, 0, 1, 0, 0, 1), (1, 1, 0, 1, 0, 0, 0, 0)])
+def test_graph_step_ordering_under_repeated_replays(policy):
+    """Layers overlap through programmatic launch; a reuse layer must never
+    read index slots before the reset layer that owns them has written them.
+    The slots are poisoned with an invalid index before every replay, so an
+    early read shows up in the status word (and in the outputs)."""
+    w = W.custom("order", batch=1, layers=8, seqlens=(32768,), num_q_heads=32, num_kv_heads=8,
+                 topk=16, seed=27)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    args = ([l[0] for l in layers], [l[1] for l in layers], [l[2] for l in layers])
+    topk = torch.full((8, 1, 8, 16), -7, dtype=torch.int32, device="cuda")
+    outs = [run.new_out() for _ in range(8)]
+    H.decode_step(run.shape, policy, *args, run.seqlens, outs, topk, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    ref = [o.clone() for o in outs]
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        topk.fill_(-7)
+        H.decode_step(run.shape, policy, *args, run.seqlens, outs, topk, run.ws,
+                      stream=torch.cuda.current_stream())
+    for _ in range(30):
+        g.replay()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    for a, b in zip(outs, ref):
+        assert torch.equal(a, b)
+
+
 def test_step_host_buffers_match_device_step():
     w = W.custom("hoststep", batch=2, layers=3, seqlens=(2000, 900), num_q_heads=8,
                  num_kv_heads=2, topk=4, seed=23)
