@@ -22,8 +22,9 @@ namespace {
 
 constexpr size_t kSmemBF16 = sizeof(SmemBF16) + 1024;  // + alignment slack
 static_assert(kSmemBF16 <= 232448, "bf16 kernel shared memory exceeds 227 KB");
-static_assert(rc_smem_bytes(NST_MAX_RC) + 1024 <= 232448,
-              "cluster reuse kernel shared memory exceeds 227 KB");
+constexpr size_t kSmemMax = 232448;  // 227 KB of dynamic shared memory per CTA
+static_assert(rc_smem_bytes(1, HYLRA_MAX_GROUP, 1) + 1024 <= kSmemMax,
+              "cluster reuse kernel needs room for one stage");
 
 struct Layout {
   size_t status, tickets, partials, bstat, total;
@@ -141,46 +142,50 @@ int prepare_bf16_kernels() {
 }
 
 // Cluster reuse kernel: cluster size (CTAs per (b, h)), blocks per CTA and
-// pipeline stages.  The largest cluster size (<= 16, <= the blocks per head)
-// whose B*Hkv clusters the device can hold at once; 0 when none can.
+// pipeline stages.
 struct RCPlan {
   int cs, upc, nst;
   size_t smem;
 };
 
-RCPlan rc_plan_for(int cs, int kmax) {
+// Stages: one per block of the CTA up to NST_MAX_RC, as many as fit beside
+// the gather area (0: this cluster size does not fit).
+RCPlan rc_plan_for(int cs, int kmax, int r, int nst_cap = NST_MAX_RC) {
   RCPlan pl{};
   pl.cs = cs;
   pl.upc = (kmax + cs - 1) / cs;
-  pl.nst = std::min(pl.upc, NST_MAX_RC);
-  pl.smem = rc_smem_bytes(pl.nst) + 1024;
+  const size_t fixed = rc_smem_bytes(cs, r, 0) + 1024;
+  const int fit = fixed >= kSmemMax ? 0 : (int)((kSmemMax - fixed) / STAGE_BYTES);
+  pl.nst = std::min(std::min(pl.upc, nst_cap), fit);
+  pl.smem = rc_smem_bytes(cs, r, pl.nst) + 1024;
   return pl;
 }
 
-// Clusters of this size and stage count the device can hold at once
-// (queried once per device).
-int rc_max_active(int cs, int nst) {
+// Clusters of this shape the device can hold at once (queried once per
+// device and shape).
+int rc_max_active(const RCPlan& pl) {
   static std::mutex mu;
-  static std::vector<std::vector<int>> cache;  // [dev][cs * 4 + nst]: -1 unknown
+  static std::vector<std::vector<int>> cache;  // [dev][(cs * 4 + nst) * 64 + smem KB / 4]
   int dev = 0;
+  if (pl.nst < 1 || pl.cs < 1 || pl.cs > 16) return 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lock(mu);
-  if ((int)cache.size() <= dev) cache.resize(dev + 1, std::vector<int>(17 * 4, -1));
-  int& v = cache[dev][cs * 4 + nst];
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, std::vector<int>(17 * 4 * 64, -1));
+  int& v = cache[dev][(pl.cs * 4 + pl.nst) * 64 + (int)std::min<size_t>(63, pl.smem / 4096)];
   if (v < 0) {
     v = 0;
     if (cudaFuncSetAttribute(decode_reuse_cluster_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(rc_smem_bytes(NST_MAX_RC) + 1024)) == cudaSuccess &&
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax) ==
+            cudaSuccess &&
         cudaFuncSetAttribute(decode_reuse_cluster_kernel,
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(cs, 1);
+      cfg.gridDim = dim3(pl.cs, 1);
       cfg.blockDim = dim3(NTHR_BF16);
-      cfg.dynamicSmemBytes = rc_smem_bytes(nst) + 1024;
+      cfg.dynamicSmemBytes = pl.smem;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.x = pl.cs;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
@@ -194,27 +199,40 @@ int rc_max_active(int cs, int nst) {
   return v;
 }
 
-// A small reuse layer (fewer blocks than SMs) is latency-bound: its clusters
-// take at most half of the CTA slots, so that, launched as a programmatic
-// dependent, the next layer's CTAs are resident, loading and computing while
-// this one finishes (a CTA with one pipeline stage leaves room for two per
-// SM).  A large layer spreads over every SM.
+#ifdef HYLRA_TRACE
+int g_plan_cs = 0, g_plan_nst = 0;  // tuning builds: force a plan
+#endif
+
+// A small reuse layer (fewer blocks than SMs) is a latency chain: inside a
+// decode step its CTAs are launched early and stage their blocks while the
+// preceding layer runs, and after the wait each CTA computes its blocks and
+// CTA 0 merges the cluster.  Two blocks per CTA, both staged, measured
+// fastest on B200 (one block per CTA needs twice the clusters, of which
+// fewer fit at once; three or more lengthen the chain after the wait).  A
+// large layer spreads over every SM.
 bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
   const int nbmax = std::max(1, (s->max_seqlen + BLK - 1) / BLK);
   const int kmax = std::max(1, std::min(s->topk, nbmax));
   const int nbh = s->batch * s->num_kv_heads;
+  const int r = s->num_q_heads / s->num_kv_heads;
   if (nbh > 65535) return false;
   int sms = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
+#ifdef HYLRA_TRACE
+  if (g_plan_cs > 0) {
+    const RCPlan pl = rc_plan_for(std::min(g_plan_cs, kmax), kmax, r, g_plan_nst);
+    if (pl.nst < 1 || rc_max_active(pl) < 1) return false;
+    *out = pl;
+    return true;
+  }
+#endif
   const bool small = (long long)nbh * kmax <= sms;
   if (small) {
-    // room for two layers' clusters at once (the next layer's CTAs load and
-    // compute while this one finishes), the largest clusters first
-    for (int cs = std::min(16, kmax); cs >= 1; --cs) {
-      const RCPlan pl = rc_plan_for(cs, kmax);
-      if (rc_max_active(cs, pl.nst) >= 2 * nbh) {
+    for (int cs = std::min(16, (kmax + 1) / 2); cs >= 1; --cs) {
+      const RCPlan pl = rc_plan_for(cs, kmax, r);
+      if (pl.nst >= 1 && rc_max_active(pl) >= nbh) {
         *out = pl;
         return true;
       }
@@ -222,8 +240,9 @@ bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
   }
   const int cs_max = std::max(1, std::min(std::min(16, kmax), sms / std::max(1, nbh)));
   for (int cs = cs_max; cs >= 1; --cs) {
-    const RCPlan pl = rc_plan_for(cs, kmax);
-    const int n = rc_max_active(cs, pl.nst);
+    const RCPlan pl = rc_plan_for(cs, kmax, r);
+    if (pl.nst < 1) continue;
+    const int n = rc_max_active(pl);
     if (n >= nbh || (cs == 1 && n > 0)) {
       *out = pl;
       return true;
@@ -284,6 +303,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.max_seqlen = s->max_seqlen;
   p.nbmax = L.nbmax;
   p.idx_wait = idx_from_prev ? 1 : 0;
+  p.q_wait = pdl ? 1 : 0;
   p.trace_slot = trace_slot;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
 
@@ -337,7 +357,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
     mcfg.gridDim = dim3(s->batch * s->num_kv_heads);
-    mcfg.blockDim = dim3(NT_BF16);
+    mcfg.blockDim = dim3(NT_MERGE);
     mcfg.dynamicSmemBytes = 0;
     mcfg.stream = stream;
     mcfg.attrs = attr;
@@ -470,6 +490,13 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
 }
 
 #ifdef HYLRA_TRACE
+// Trace builds only: force the reuse cluster plan (cs = 0: automatic).
+int hylra_plan_override(int cs, int nst) {
+  g_plan_cs = cs;
+  g_plan_nst = nst;
+  return HYLRA_OK;
+}
+
 // Trace builds only: device buffer of TRACE_PER_CTA uint64 per CTA (or NULL).
 int hylra_trace_set(void* buf) {
   unsigned long long* p = static_cast<unsigned long long*>(buf);

@@ -50,6 +50,7 @@ constexpr int NTHR_BF16 = NT_BF16 + 32;  // + one producer warp
 constexpr int NW_F32 = 4;                // warps of the fp32 kernel (32 tokens each)
 constexpr int NT_F32 = NW_F32 * 32;
 constexpr int NWMAX = 8;
+constexpr int NT_MERGE = 512;              // threads of the merge kernel
 constexpr int NCOMB = 4;                 // per-warp states merged at a segment end
 constexpr int NSTAGE = 3;
 constexpr int BOX_BYTES = 64 * 2 * BLK;       // 64 bf16 columns x 128 rows
@@ -65,7 +66,7 @@ constexpr int MAX_SEGS = 8;     // segments a CTA queues before taking their tic
 // then free): per CTA, the producer and the first consumer thread append
 // (event code, %globaltimer) pairs to a device buffer set by the host.
 #ifdef HYLRA_TRACE
-__device__ unsigned long long* g_hylra_trace = nullptr;
+__constant__ unsigned long long* g_hylra_trace = nullptr;  // constant cache: no L2 round trip per event
 constexpr int TRACE_PER_CTA = 512;
 constexpr int TRACE_CTAS = 256;
 __device__ __forceinline__ void trace_event(int& n, int base, int code, int slot) {
@@ -86,7 +87,19 @@ __device__ __forceinline__ void trace_event_cta(int& n, int cta, int code, int s
   ++n;
 }
 #define HYLRA_TRACE_CTA(n, cta, code) trace_event_cta(n, cta, code, p.trace_slot)
+// a raw value (e.g. a cycle count) in place of the timestamp
+__device__ __forceinline__ void trace_value_cta(int& n, int cta, int code, int slot,
+                                                unsigned long long v) {
+  if (g_hylra_trace && n < 255 && cta < TRACE_CTAS)
+    g_hylra_trace[((size_t)slot * TRACE_CTAS + cta) * TRACE_PER_CTA + n] =
+        ((unsigned long long)code << 48) | (v & 0xFFFFFFFFFFFFull);
+  ++n;
+}
+#define HYLRA_TRACE_VAL(n, cta, code, v) trace_value_cta(n, cta, code, p.trace_slot, v)
+#define HYLRA_CLOCK() clock64()
 #else
+#define HYLRA_TRACE_VAL(n, cta, code, v) ((void)0)
+#define HYLRA_CLOCK() 0ll
 #define HYLRA_TRACE_CTA(n, cta, code) ((void)0)
 #define HYLRA_TRACE_EV(n, base, code) ((void)0)
 #endif
@@ -108,6 +121,7 @@ struct Params {
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
   int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
+  int q_wait;        // q and each sequence's newest K/V row come from the preceding kernel
   int upc, nst;      // cluster reuse kernel: blocks per CTA, pipeline stages
   int trace_slot;    // trace builds: which per-launch region of the trace buffer
   float scale_log2;  // log2(e) / sqrt(d)
@@ -140,11 +154,12 @@ struct alignas(16) SmemCommon {
   int prefix[HYLRA_MAX_BATCH + 1];  // units before sequence b (all heads)
   int hist[256];
   int misc[8];  // 1: radix digit, 2: remaining, 3: list size, 4: abort
-  int warp_sums[NWMAX];
+  int warp_sums[NT_MERGE / 32];
   StageMeta segs[MAX_SEGS];  // segments whose partial is stored but not yet ticketed
   int seg_last[MAX_SEGS];
   int nseg;
-  int trace_n;  // trace builds: events recorded by consumer thread 0
+  int trace_n;    // trace builds: events recorded by consumer thread 0
+  int trace_cta;  // trace builds: trace region of this CTA
 };
 static_assert(sizeof(float) * NCOMB * GMAX * HD >= MAX_NB * 4 + HYLRA_MAX_TOPK * 8,
               "top-k scratch must fit in the combine buffer");
@@ -314,17 +329,17 @@ __device__ __forceinline__ int unit_index_entry(const Params& p, const UnitIter&
 // Called by the NT merge threads (ct = 0..NT-1).
 //
 // A key "beats" another when it is larger, or equal with a lower index; the
-// answer is the kp keys beaten by fewer than kp others.  Fast path (kp <= 32):
+// answer is the kp keys beaten by fewer than kp others.  Up to NT keys and
+// kp <= 32: per-warp sorted lists (below).  Otherwise, fast path (kp <= 32):
 // each warp sorts its 32 per-thread maxima (bitonic network over shuffles);
 // its kp-th largest is a value that kp of its keys reach, so tau0, the
-// largest of these over the warps, bounds the kp-th largest key from below
-// and every answer is among the keys >= tau0, whose ranks among those
-// candidates are their global ranks.  With few candidates (the usual case)
-// they are ranked by pairwise comparison; otherwise (many equal keys, or
-// kp > 32) a radix select runs.
+// largest of these over the warps, bounds the kp-th largest key from below.
+// Keys above tau0 are candidates, ranked by pairwise comparison; keys equal
+// to tau0 fill the remaining ranks in block order.  When there are many
+// candidates (few top blocks per warp), or kp > 32, a radix select runs.
 constexpr int TOPK_LIST_CAP = (NCOMB * GMAX * HD * 4 - MAX_NB * 4) / 8 - 128;
 
-template <int NT>
+template <int NT, int BAR = BAR_CONS>
 __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int ct) {
   constexpr int NW = NT / 32;
   uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
@@ -334,10 +349,60 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
   const int kp = min(p.k, nb);
   const int lane = ct & 31, wid = ct >> 5;
 
+  if (nb <= NT && kp <= 32) {
+    // One key per thread.  (key, block) pairs compare as one 64-bit
+    // composite, descending by key then ascending by block, so all are
+    // distinct.  Each warp places its 32 composites in sorted order (an
+    // entry's place = how many of the warp's composites exceed it) and keeps
+    // the first kp.  An entry's global rank is the sum over warps of how many
+    // of their kept entries exceed it (a binary search in each sorted list);
+    // the entries of rank < kp are the answer.
+    uint64_t* comp = reinterpret_cast<uint64_t*>(tmax + 256);  // [NT] composites
+    uint64_t* lists = comp + NT;                                 // [NW][32] sorted
+    const uint64_t v = ct < nb ? ((uint64_t)keys[ct] << 32) | (uint32_t)~(uint32_t)ct : 0ull;
+    comp[ct] = v;
+    lists[ct] = 0ull;  // lists cover NW * 32 == NT entries; unused places stay 0
+    named_bar_sync(BAR, NT);
+    // place within the warp: how many of its 32 composites exceed v
+    int rw = 0;
+    const ulonglong2* wc = reinterpret_cast<const ulonglong2*>(comp + wid * 32);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const ulonglong2 o = wc[j];
+      rw += (o.x > v) + (o.y > v);
+    }
+    if (rw < kp) lists[wid * 32 + rw] = v;
+    named_bar_sync(BAR, NT);
+    if (rw < kp && v != 0ull) {
+      // the NW searches advance in lock step (independent loads in flight);
+      // in its own warp's list an entry finds exactly `rw` predecessors
+      int pos[NW];
+#pragma unroll
+      for (int w = 0; w < NW; ++w) pos[w] = 0;
+#pragma unroll
+      for (int step = 32; step > 0; step >>= 1) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const int t = pos[w] + step;
+          if (t <= kp && lists[w * 32 + t - 1] > v) pos[w] = t;
+        }
+      }
+      int rank = 0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) rank += pos[w];
+      if (rank < kp) dst[rank] = (int32_t)~(uint32_t)(v & 0xffffffffull);
+    }
+    for (int slot = kp + ct; slot < p.k; slot += NT) dst[slot] = -1;
+    return;
+  }
+
   bool fast = kp <= 32;
   if (fast) {
+    // thread ct owns blocks b0..b1-1 (index order)
+    const int per = (nb + NT - 1) / NT;
+    const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
     uint32_t v = 0u;
-    for (int beta = ct; beta < nb; beta += NT) v = max(v, keys[beta]);
+    for (int beta = b0; beta < b1; ++beta) v = max(v, keys[beta]);
     // descending bitonic sort of the warp's 32 per-thread maxima
 #pragma unroll
     for (int k = 2; k <= 32; k <<= 1) {
@@ -349,36 +414,66 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     }
     if (lane == kp - 1) tmax[wid] = v;
     if (ct == 0) c.misc[3] = 0;
-    named_bar_sync(BAR_CONS, NT);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 20 << 8);
+    named_bar_sync(BAR, NT);
+    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 20 << 8);
     uint32_t tau0 = 0u;
 #pragma unroll
     for (int w = 0; w < NW; ++w) tau0 = max(tau0, tmax[w]);
-    for (int beta = ct; beta < nb; beta += NT) {
+    // Keys above tau0 go to the candidate list; keys equal to it (often
+    // many, e.g. scores that underflow to zero) are only counted, in block
+    // order: the lowest-index ones fill whatever the list leaves of kp.
+    int eq = 0;
+    for (int beta = b0; beta < b1; ++beta) {
       const uint32_t key = keys[beta];
-      if (key >= tau0) {
+      if (key > tau0) {
         const int pos = atomicAdd(&c.misc[3], 1);
         if (pos < TOPK_LIST_CAP) list[pos] = make_uint2(key, (uint32_t)beta);
       }
+      eq += key == tau0;
     }
-    named_bar_sync(BAR_CONS, NT);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 22 << 8);
-    const int ncand = c.misc[3];
-    fast = ncand <= TOPK_LIST_CAP;
+    int incl = eq;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    if (lane == 31) c.warp_sums[wid] = incl;
+    named_bar_sync(BAR, NT);
+    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 22 << 8);
+    const int ngt = c.misc[3];
+    // ranking costs ngt^2 / 32 comparisons: with many candidates (the
+    // top blocks spread thinly over the warps) the radix select is cheaper
+    fast = ngt <= min(TOPK_LIST_CAP, 64);
     if (fast) {
-      for (int e = ct; e < ncand; e += NT) {
+      // rank of a listed key = how many listed keys beat it; one warp per
+      // candidate, its lanes comparing 32 others at a time
+      for (int e = wid; e < ngt; e += NW) {
         const uint2 me = list[e];
         int r = 0;
-        for (int j = 0; j < ncand; ++j) {
-          const uint2 o = list[j];
-          r += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        for (int j0 = 0; j0 < ngt; j0 += 32) {
+          const int j = j0 + lane;
+          bool beats = false;
+          if (j < ngt) {
+            const uint2 o = list[j];
+            beats = (o.x > me.x) || (o.x == me.x && o.y < me.y);
+          }
+          r += __popc(__ballot_sync(0xffffffffu, beats));
         }
-        if (r < kp) dst[r] = (int32_t)me.y;
+        if (lane == 0 && r < kp) dst[r] = (int32_t)me.y;
+      }
+      // keys equal to tau0 take ranks ngt, ngt+1, ... in block order
+      int before = incl - eq;
+      for (int w = 0; w < wid; ++w) before += c.warp_sums[w];
+      for (int beta = b0; beta < b1 && ngt + before < kp; ++beta) {
+        if (keys[beta] == tau0) {
+          dst[ngt + before] = beta;
+          ++before;
+        }
       }
       for (int slot = kp + ct; slot < p.k; slot += NT) dst[slot] = -1;
       return;
     }
-    named_bar_sync(BAR_CONS, NT);  // everyone has read ncand before it is reused
+    named_bar_sync(BAR, NT);  // everyone has read ngt before it is reused
   }
 
   // Radix select of the kp-th largest key, 8 bits per pass.
@@ -388,7 +483,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     const int shift = 24 - 8 * pass;
     for (int i = ct; i < 256; i += NT) c.hist[i] = 0;
     if (ct == 0) c.misc[3] = 0;
-    named_bar_sync(BAR_CONS, NT);
+    named_bar_sync(BAR, NT);
     // one shared atomic per distinct digit per warp (scores of one head
     // mostly share their top bits, so per-thread atomics would serialize)
     for (int beta0 = 0; beta0 < nb; beta0 += NT) {
@@ -399,7 +494,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
       const uint32_t peers = __match_any_sync(0xffffffffu, digit);
       if (match && (__ffs(peers) - 1) == lane) atomicAdd(&c.hist[digit], __popc(peers));
     }
-    named_bar_sync(BAR_CONS, NT);
+    named_bar_sync(BAR, NT);
     if (wid == 0) {
       int cnt[8];
       int local = 0;
@@ -428,7 +523,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
         }
       }
     }
-    named_bar_sync(BAR_CONS, NT);
+    named_bar_sync(BAR, NT);
     prefix |= (uint32_t)c.misc[1] << shift;
     remain = c.misc[2];
   }
@@ -447,7 +542,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     if (lane >= off) incl += v;
   }
   if (lane == 31) c.warp_sums[wid] = incl;
-  named_bar_sync(BAR_CONS, NT);
+  named_bar_sync(BAR, NT);
   int before = incl - eq;
 #pragma unroll
   for (int w = 0; w < NW; ++w)
@@ -464,7 +559,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
       if (pos < kp) rlist[pos] = make_uint2(key, (uint32_t)beta);  // exactly kp are selected
     }
   }
-  named_bar_sync(BAR_CONS, NT);
+  named_bar_sync(BAR, NT);
   for (int e = ct; e < kp; e += NT) {
     const uint2 me = rlist[e];
     int rank = 0;
@@ -487,7 +582,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
 // through shared memory.
 template <bool FULL, int NT>
 __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
-  constexpr int CB = 10;  // contributors per thread and batch of loads
+  constexpr int CB = NT >= 512 ? 6 : 10;  // contributors per thread and batch of loads
   const int bh = m.b * p.Hkv + m.h;
   const int nc = m.ncontrib;
   const int r = p.r;
@@ -506,7 +601,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
   }
 
   const int ncol = r * (HD / 4);             // float4 output columns
-  const int G = ncol >= NT ? 1 : NT / ncol;  // contributor groups
+  const int G = ncol >= NT ? 1 : min(NWMAX, NT / ncol);  // contributor groups
   float4* red = reinterpret_cast<float4*>(&c.comb_o[0][0][0]);  // [G][ncol]
   for (int t = ct; t < G * ncol; t += NT) {
     const int q = t / ncol, col = t - q * ncol;
@@ -553,6 +648,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
       c.comb_z[q][g] = Z;
     }
   }
+  if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 16 << 8);
   named_bar_sync(BAR_CONS, NT);
   for (int col = ct; col < ncol; col += NT) {
     const int g = col / (HD / 4), d4 = col - g * (HD / 4);
@@ -582,6 +678,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
       c.rzg[g] = Z > 0.f ? 1.f / Z : 0.f;
     }
   }
+  if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 17 << 8);
   if (FULL) {
     named_bar_sync(BAR_CONS, NT);  // head maxima and sums visible; comb_o free
     uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
@@ -613,9 +710,9 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
     }
     if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
     named_bar_sync(BAR_CONS, NT);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 12 << 8);
+    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 12 << 8);
     topk_select<NT>(p, c, bh, m.nb, ct);
-    if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 13 << 8);
+    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
   } else {
     // a reused list naming one block twice counts that block twice: flag it
     named_bar_sync(BAR_CONS, NT);  // comb_o free
@@ -678,7 +775,7 @@ template <bool FULL, int NT>
 __device__ void flush_segments(const Params& p, SmemCommon& c, int ct) {
   __threadfence();
   named_bar_sync(BAR_CONS, NT);
-  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 14 << 8);
+  if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 14 << 8);
   const int ns = c.nseg;
   if (ct < ns) {
     const StageMeta& m = c.segs[ct];
@@ -686,7 +783,7 @@ __device__ void flush_segments(const Params& p, SmemCommon& c, int ct) {
     c.seg_last[ct] = (old == (uint32_t)(m.ncontrib - 1)) ? 1 : 0;
   }
   named_bar_sync(BAR_CONS, NT);
-  if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 15 << 8);
+  if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 15 << 8);
   for (int k = 0; k < ns; ++k) {
     if (c.seg_last[k]) {
       __threadfence();
@@ -868,31 +965,51 @@ struct WarpAttn {
     }
   }
 
+  // This warp's state as is: O^T columns into so[head][dim], running max
+  // and sum into sm_[head], sz_[head].
+  __device__ __forceinline__ void store_state(float (*so)[HD], float* sm_, float* sz_) const {
+#pragma unroll
+    for (int dm = 0; dm < 8; ++dm) {
+      const int d0 = dm * 16 + g4;
+      so[2 * c4][d0] = o[dm][0];
+      so[2 * c4 + 1][d0] = o[dm][1];
+      so[2 * c4][d0 + 8] = o[dm][2];
+      so[2 * c4 + 1][d0 + 8] = o[dm][3];
+    }
+    if (g4 == 0) {
+      sm_[2 * c4] = m_run[0];
+      sm_[2 * c4 + 1] = m_run[1];
+      sz_[2 * c4] = z_run[0];
+      sz_[2 * c4 + 1] = z_run[1];
+    }
+  }
+
   // Merge the eight warps' states pairwise into comb_*[0..NCOMB) (warps
   // cw >= NCOMB hand theirs to warp cw - NCOMB).  Called by the NT_BF16
   // consumer threads together; ends with a barrier.
-  __device__ __forceinline__ void to_comb(SmemCommon& c, int cw) {
+  __device__ __forceinline__ void to_comb(float (*co)[GMAX][HD], float (*cm)[GMAX],
+                                          float (*cz)[GMAX], int cw) {
     if (cw >= NCOMB) {
       const int w = cw - NCOMB;
 #pragma unroll
       for (int dm = 0; dm < 8; ++dm) {
         const int d0 = dm * 16 + g4;
-        c.comb_o[w][2 * c4][d0] = o[dm][0];
-        c.comb_o[w][2 * c4 + 1][d0] = o[dm][1];
-        c.comb_o[w][2 * c4][d0 + 8] = o[dm][2];
-        c.comb_o[w][2 * c4 + 1][d0 + 8] = o[dm][3];
+        co[w][2 * c4][d0] = o[dm][0];
+        co[w][2 * c4 + 1][d0] = o[dm][1];
+        co[w][2 * c4][d0 + 8] = o[dm][2];
+        co[w][2 * c4 + 1][d0 + 8] = o[dm][3];
       }
       if (g4 == 0) {
-        c.comb_m[w][2 * c4] = m_run[0];
-        c.comb_m[w][2 * c4 + 1] = m_run[1];
-        c.comb_z[w][2 * c4] = z_run[0];
-        c.comb_z[w][2 * c4 + 1] = z_run[1];
+        cm[w][2 * c4] = m_run[0];
+        cm[w][2 * c4 + 1] = m_run[1];
+        cz[w][2 * c4] = z_run[0];
+        cz[w][2 * c4 + 1] = z_run[1];
       }
     }
     named_bar_sync(BAR_CONS, NT_BF16);
     if (cw < NCOMB) {
-      const float m2A = c.comb_m[cw][2 * c4], m2B = c.comb_m[cw][2 * c4 + 1];
-      const float z2A = c.comb_z[cw][2 * c4], z2B = c.comb_z[cw][2 * c4 + 1];
+      const float m2A = cm[cw][2 * c4], m2B = cm[cw][2 * c4 + 1];
+      const float z2A = cz[cw][2 * c4], z2B = cz[cw][2 * c4 + 1];
       __syncwarp();
       const float mnA = fmaxf(m_run[0], m2A), mnB = fmaxf(m_run[1], m2B);
       const float fA = mnA == -INFINITY ? 0.f : ex2_approx(m_run[0] - mnA);
@@ -902,18 +1019,18 @@ struct WarpAttn {
 #pragma unroll
       for (int dm = 0; dm < 8; ++dm) {
         const int d0 = dm * 16 + g4;
-        float* a = &c.comb_o[cw][2 * c4][d0];
-        float* b = &c.comb_o[cw][2 * c4 + 1][d0];
+        float* a = &co[cw][2 * c4][d0];
+        float* b = &co[cw][2 * c4 + 1][d0];
         a[0] = o[dm][0] * fA + a[0] * hA;
         b[0] = o[dm][1] * fB + b[0] * hB;
         a[8] = o[dm][2] * fA + a[8] * hA;
         b[8] = o[dm][3] * fB + b[8] * hB;
       }
       if (g4 == 0) {
-        c.comb_m[cw][2 * c4] = mnA;
-        c.comb_m[cw][2 * c4 + 1] = mnB;
-        c.comb_z[cw][2 * c4] = z_run[0] * fA + z2A * hA;
-        c.comb_z[cw][2 * c4 + 1] = z_run[1] * fB + z2B * hB;
+        cm[cw][2 * c4] = mnA;
+        cm[cw][2 * c4 + 1] = mnB;
+        cz[cw][2 * c4] = z_run[0] * fA + z2A * hA;
+        cz[cw][2 * c4 + 1] = z_run[1] * fB + z2B * hB;
       }
     }
     named_bar_sync(BAR_CONS, NT_BF16);
@@ -946,6 +1063,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     c.misc[4] = 0;
     c.nseg = 0;
     c.trace_n = 0;
+    c.trace_cta = (int)blockIdx.x;
     fence_mbar_init();
   }
   if (tid == 32) {
@@ -986,8 +1104,27 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     long long row0 = 0;
     const long long hstride = p.cap > 0 ? p.cap : p.total;
     // reused indices written by the preceding kernel: wait for it first
-    if (!FULL && p.idx_wait) griddep_wait();
+    bool waited = false;
+    if (!FULL && p.idx_wait) {
+      griddep_wait();
+      waited = true;
+    }
     griddep_launch_dependents();  // the producer writes nothing
+    // With q_wait, the first stages' K/V tiles are requested before the wait
+    // and their q rows after it (qpend: stages whose q load is deferred).
+    uint32_t qpend = 0u;
+    auto wait_and_flush = [&]() {
+      if (waited) return;
+      griddep_wait();
+      waited = true;
+      for (int t = 0; t < NSTAGE; ++t) {
+        if (!(qpend & (1u << t)) || *abort_flag) continue;
+        const StageMeta& mt = sm.meta[t];
+        bulk_load(sm.qslot[t], qbase + ((size_t)mt.b * p.Hq + (size_t)mt.h * p.r) * HD * 2,
+                  qbytes, &sm.fullK_bar[t]);
+      }
+      qpend = 0u;
+    };
     int idx_cur = FULL ? 0 : unit_index_entry(p, it);
     int tn = 0;
     (void)tn;
@@ -1003,10 +1140,14 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       }
       const int s = i % NSTAGE;
       const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
+      // a stage is refilled only after the consumers used it, which needs q
+      if (p.q_wait && i >= NSTAGE) wait_and_flush();
       mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
       HYLRA_TRACE_EV(tn, 256, (2 << 8) | (i & 0xff));
       const StageMeta m =
           describe_unit<FULL>(p, c, it, i, n, T, G, seqlen, FULL ? it.j : idx_cur, true);
+      // the block holding the newest token is read after the wait as well
+      if (p.q_wait && m.blk >= 0 && m.blk == m.nb - 1) wait_and_flush();
       sm.meta[s] = m;
       const bool seg_start = (m.flags & F_SEG_START) != 0;
       uint32_t bytesK = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? 2u * BOX_BYTES : 0u);
@@ -1016,9 +1157,14 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       uint8_t* st = sm.stage[s];
       if (bytesK) {
         mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
-        if (seg_start)
-          bulk_load(sm.qslot[s], qbase + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD * 2, qbytes,
-                    &sm.fullK_bar[s]);
+        if (seg_start) {
+          if (p.q_wait && !waited) {
+            qpend |= 1u << s;  // loaded after the wait; into L2 now
+            prefetch_l2_bulk(qbase + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD * 2, qbytes);
+          } else
+            bulk_load(sm.qslot[s], qbase + ((size_t)m.b * p.Hq + (size_t)m.h * p.r) * HD * 2,
+                      qbytes, &sm.fullK_bar[s]);
+        }
         if (m.blk >= 0) {
           tma_load_2d(st, &tmK, 0, row, &sm.fullK_bar[s], pol);
           tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.fullK_bar[s], pol);
@@ -1036,6 +1182,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       it = nx;
       idx_cur = idx_next;
     }
+    if (p.q_wait) wait_and_flush();
     return;
   }
 
@@ -1106,7 +1253,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (m.flags & F_SEG_END) {
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
       ensure_waited();
-      wa.to_comb(c, cw);  // eight warp states -> four
+      wa.to_comb(c.comb_o, c.comb_m, c.comb_z, cw);  // eight warp states -> four
       store_partial<NT_BF16, false>(p, c, m, ct);  // merged by merge_kernel
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 6 << 8);
     }
@@ -1121,51 +1268,246 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 // ------------------------------------------------------------ merge kernel
 //
 // Runs after decode_bf16_kernel (as its programmatic dependent): one CTA per
-// (sequence, KV head) merges the partials of that head's contributors, and
-// on reset layers scores the blocks and selects the top-k.  The kernel
-// boundary makes the partials visible; no fence or ticket is needed.
+// (sequence, KV head).  The kernel boundary makes the streaming kernel's
+// partials visible; no fence or ticket is needed.  Two independent halves
+// run side by side so that neither waits for the other:
+//   warps 0-7   merge the contributors' partial rows into the output;
+//   warps 8-15  (reset layers) derive each head's max and sum straight from
+//               the contributors' (m, Z) pairs, score the blocks and select
+//               the top-k; (reuse layers) check the index list for repeats.
+constexpr int MERGE_HALF = NT_MERGE / 2;
+constexpr int BAR_OUT = 2;   // named barrier of warps 0-7
+constexpr int BAR_TOPK = 3;  // named barrier of warps 8-15
+
+struct SmemMerge {
+  float4 red[MERGE_HALF];  // per-group partial rows, [group][float4 column]
+  float rm[NWMAX][GMAX];   // per-group running max and sum
+  float rz[NWMAX][GMAX];
+  SmemCommon c;            // prefix sums; head statistics, keys and top-k scratch
+};
+
 template <bool FULL>
-__global__ void __launch_bounds__(NT_BF16, 1) merge_kernel(const __grid_constant__ Params p,
-                                                           int grid_stream) {
-  __shared__ SmemCommon c;
-  const int ct = threadIdx.x;
+__global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constant__ Params p,
+                                                            int grid_stream) {
+  __shared__ SmemMerge sm;
+  SmemCommon& c = sm.c;
+  const int tid = threadIdx.x;
   const int bh = (int)blockIdx.x;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
-  int tn = 0;
-  (void)tn;
-  if (ct == 0) {
-    c.trace_n = 255;  // merge_bh's own trace points are off here
-    HYLRA_TRACE_CTA(tn, 160 + bh, 30 << 8);
+  const int r = p.r;
+  if (tid == 0) {
+    c.trace_n = 0;
+    c.trace_cta = 160 + bh;
+    HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 30 << 8);
   }
+  // everything that does not depend on the streaming kernel's output first
   build_prefix(p, c, FULL);
-  griddep_wait();  // the streaming kernel has completed: partials are visible
-  griddep_launch_dependents();
-  if (ct == 0) HYLRA_TRACE_CTA(tn, 160 + bh, 31 << 8);
+  const int seqlen = valid_seqlen(p, b, false);
   __syncthreads();
   const int T = c.prefix[p.B];
   const int U = (c.prefix[b + 1] - c.prefix[b]) / p.Hkv;
+  const int G = min(grid_stream, max(T, 1));
+  const int start = c.prefix[b] + h * U;
+  int first = 0, nc = 0;
+  if (U > 0) {
+    first = owner_cta(start, T, G);
+    nc = owner_cta((long long)start + U - 1, T, G) - first + 1;
+    first += bh;  // partial slot of contributor c is c + bh
+  }
+  const int nb = (seqlen + BLK - 1) / BLK;
+  const int kp = min(p.k, nb);
+  const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
+  griddep_wait();  // the streaming kernel has completed: partials are visible
+  griddep_launch_dependents();
+  if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 31 << 8);
   if (U == 0) {
     // a sequence without units: zero output (and no indices)
-    for (int i = ct; i < p.r * HD; i += NT_BF16)
-      p.out[((size_t)b * p.Hq + (size_t)h * p.r) * HD + i] = 0.f;
+    for (int i = tid; i < r * HD; i += NT_MERGE)
+      p.out[((size_t)b * p.Hq + (size_t)h * r) * HD + i] = 0.f;
     if (FULL)
-      for (int i = ct; i < p.k; i += NT_BF16) p.topk_out[(size_t)bh * p.k + i] = -1;
+      for (int i = tid; i < p.k; i += NT_MERGE) p.topk_out[(size_t)bh * p.k + i] = -1;
     return;
   }
-  const int G = min(grid_stream, T);
-  const int start = c.prefix[b] + h * U;
-  const int cf = owner_cta(start, T, G);
-  const int cl = owner_cta((long long)start + U - 1, T, G);
-  const int seqlen = valid_seqlen(p, b, false);
-  StageMeta m{};
-  m.b = b;
-  m.h = h;
-  m.blk = 0;
-  m.first_slot = cf + bh;
-  m.ncontrib = cl - cf + 1;
-  m.nb = (seqlen + BLK - 1) / BLK;
-  merge_bh<FULL, NT_BF16>(p, c, m, ct);
-  if (ct == 0) HYLRA_TRACE_CTA(tn, 160 + bh, 32 << 8);
+
+  if (tid < MERGE_HALF) {
+    // ------------------------------------------------ output rows (LSE merge)
+    constexpr int CB = 10;  // contributors per thread and batch of loads
+    const int ncol = r * (HD / 4);  // float4 columns
+    const int GA = ncol >= MERGE_HALF ? 1 : min(NWMAX, MERGE_HALF / ncol);
+    for (int t = tid; t < GA * ncol; t += MERGE_HALF) {
+      const int q = t / ncol, col = t - q * ncol;
+      const int g = col / (HD / 4), d4 = col - g * (HD / 4);
+      float M = -INFINITY, Z = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = q; j0 < nc; j0 += GA * CB) {
+        float mv[CB], zv[CB];
+        float4 ov[CB];
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+          const int j = j0 + u * GA;
+          mv[u] = -INFINITY;
+          if (j < nc) {
+            const float* sl = pbase + (size_t)j * SLOT_FLOATS;
+            mv[u] = __ldcg(sl + GMAX * HD + g);
+            zv[u] = __ldcg(sl + GMAX * HD + GMAX + g);
+            ov[u] = __ldcg(reinterpret_cast<const float4*>(sl + g * HD + 4 * d4));
+          }
+        }
+        float mb = M;
+#pragma unroll
+        for (int u = 0; u < CB; ++u) mb = fmaxf(mb, mv[u]);
+        if (mb != -INFINITY) {
+          const float fo = M == -INFINITY ? 0.f : ex2_approx(M - mb);
+          acc.x *= fo;
+          acc.y *= fo;
+          acc.z *= fo;
+          acc.w *= fo;
+          Z *= fo;
+#pragma unroll
+          for (int u = 0; u < CB; ++u) {
+            if (mv[u] == -INFINITY) continue;
+            const float f = ex2_approx(mv[u] - mb);
+            acc.x = fmaf(ov[u].x, f, acc.x);
+            acc.y = fmaf(ov[u].y, f, acc.y);
+            acc.z = fmaf(ov[u].z, f, acc.z);
+            acc.w = fmaf(ov[u].w, f, acc.w);
+            Z = fmaf(zv[u], f, Z);
+          }
+          M = mb;
+        }
+      }
+      sm.red[t] = acc;
+      if (d4 == 0) {
+        sm.rm[q][g] = M;
+        sm.rz[q][g] = Z;
+      }
+    }
+    named_bar_sync(BAR_OUT, MERGE_HALF);
+    for (int col = tid; col < ncol; col += MERGE_HALF) {
+      const int g = col / (HD / 4), d4 = col - g * (HD / 4);
+      float M = -INFINITY;
+      for (int q = 0; q < GA; ++q) M = fmaxf(M, sm.rm[q][g]);
+      float Z = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+        for (int q = 0; q < GA; ++q) {
+          const float mq = sm.rm[q][g];
+          if (mq == -INFINITY) continue;
+          const float f = ex2_approx(mq - M);
+          const float4 v = sm.red[q * ncol + col];
+          acc.x = fmaf(v.x, f, acc.x);
+          acc.y = fmaf(v.y, f, acc.y);
+          acc.z = fmaf(v.z, f, acc.z);
+          acc.w = fmaf(v.w, f, acc.w);
+          Z = fmaf(sm.rz[q][g], f, Z);
+        }
+      }
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (Z > 0.f) o = make_float4(acc.x / Z, acc.y / Z, acc.z / Z, acc.w / Z);
+      *reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + (size_t)h * r + g) * HD + 4 * d4) = o;
+    }
+    if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 17 << 8);
+    return;
+  }
+
+  const int tb = tid - MERGE_HALF;  // 0..255
+  const int wb = tb >> 5, lane = tb & 31;
+  if (FULL) {
+    // --------------------------------------------- block scores and top-k
+    // block records of this thread's first block, loaded up front
+    float2 sv0[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      sv0[g] = make_float2(0.f, -INFINITY);
+      if (tb < nb && g < r)
+        sv0[g] = __ldcg(reinterpret_cast<const float2*>(
+            p.bstat + ((size_t)bh * p.nbmax + tb) * (2 * r) + 2 * g));
+    }
+    // head g's max and sum, straight from the contributors' (m, Z): warp g
+    // (a (b, h) has at most MAX_CTAS contributors)
+    if (wb < r) {
+      const int g = wb;
+      float mj[MAX_CTAS / 32], zj[MAX_CTAS / 32];
+      float M = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < MAX_CTAS / 32; ++u) {
+        const int j = u * 32 + lane;
+        mj[u] = -INFINITY;
+        zj[u] = 0.f;
+        if (j < nc) {
+          const float* sl = pbase + (size_t)j * SLOT_FLOATS;
+          mj[u] = __ldcg(sl + GMAX * HD + g);
+          zj[u] = __ldcg(sl + GMAX * HD + GMAX + g);
+        }
+        M = fmaxf(M, mj[u]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      float Z = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int u = 0; u < MAX_CTAS / 32; ++u)
+          if (mj[u] != -INFINITY) Z = fmaf(zj[u], ex2_approx(mj[u] - M), Z);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+      if (lane == 0) {
+        c.mg[g] = M;
+        c.zg[g] = Z;
+        c.rzg[g] = Z > 0.f ? 1.f / Z : 0.f;
+      }
+    }
+    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 18 << 8);
+    // score of block beta: its attention mass summed over the r heads
+    uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
+    bool nonfinite = false;
+    for (int beta = tb; beta < nb; beta += MERGE_HALF) {
+      float2 sv[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (beta == tb) {
+          sv[g] = sv0[g];
+        } else {
+          sv[g] = g < r ? __ldcg(reinterpret_cast<const float2*>(
+                              p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * r) + 2 * g))
+                        : make_float2(0.f, -INFINITY);
+        }
+      }
+      float score = 0.f;
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g)
+        if (g < r && c.zg[g] > 0.f && sv[g].y != -INFINITY)
+          score += sv[g].x * exp2f(sv[g].y - c.mg[g]) * c.rzg[g];
+      uint32_t key = 0u;
+      if (isfinite(score)) {
+        if (score > 0.f) key = __float_as_uint(score);
+      } else {
+        nonfinite = true;
+      }
+      keys[beta] = key;
+    }
+    if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
+    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 12 << 8);
+    topk_select<MERGE_HALF, BAR_TOPK>(p, c, bh, nb, tb);
+    if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
+
+  } else {
+    // a reused list naming one block twice counts that block twice: flag it
+    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+    int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
+    for (int e = tb; e < kp; e += MERGE_HALF) sidx[e] = __ldcg(idx + e);
+    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    bool dup = false;
+    for (int e = tb; e < kp; e += MERGE_HALF) {
+      const int32_t v = sidx[e];
+      if (v < 0) continue;
+      for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
+    }
+    if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
+  }
+  (void)wb;
 }
 
 // ------------------------------------------------- cluster reuse kernel
@@ -1173,10 +1515,13 @@ __global__ void __launch_bounds__(NT_BF16, 1) merge_kernel(const __grid_constant
 // Reuse layers touch only k' blocks per (sequence, KV head), too little data
 // to hide a cross-CTA merge through global memory.  Here the CTAs sharing a
 // (b, h) form one thread-block cluster (grid = cluster size x B*Hkv): CTA
-// `rank` takes blocks rank*upc .. rank*upc+upc-1 of the index list, keeps
-// its merged state in its own shared memory, and after a cluster barrier
-// rank 0 reads every CTA's state through distributed shared memory, merges
-// and writes the output.  No workspace, fence or ticket is involved.
+// `rank` takes blocks rank*upc .. rank*upc+upc-1 of the index list, merges
+// its warps' states, and stores the result straight into slot `rank` of
+// CTA 0's shared memory (distributed shared memory stores are posted, so
+// they pipeline; loads from a peer CTA do not).  One cluster barrier later
+// CTA 0 merges the slots from its own shared memory and writes the output.
+// No workspace, fence or ticket is involved, and every CTA but rank 0
+// leaves right after its stores.
 
 constexpr int NST_MAX_RC = 3;
 
@@ -1187,14 +1532,31 @@ struct SmemRC {
   alignas(8) uint64_t fullK_bar[NST_MAX_RC];
   alignas(8) uint64_t fullV_bar[NST_MAX_RC];
   alignas(8) uint64_t empty_bar[NST_MAX_RC];
-  alignas(16) float part[SLOT_FLOATS];  // this CTA's merged state: O[8][128], m[8], Z[8]
-  uint32_t seen[MAX_NB / 32];           // rank 0: blocks named so far (duplicate check)
-  SmemCommon c;
+  uint32_t seen[MAX_NB / 32];  // rank 0: blocks named so far (duplicate check)
+  int abort_flag;
 };
-constexpr size_t RC_FIXED_BYTES = (sizeof(SmemRC) + 1023) / 1024 * 1024;
 
-__host__ __device__ constexpr size_t rc_smem_bytes(int nst) {
-  return RC_FIXED_BYTES + (size_t)nst * STAGE_BYTES;
+// The eight consumer warps' states, placed on the stage area once every
+// unit has been consumed.
+struct RCComb {
+  float o[NW_BF16][GMAX][HD];
+  float m[NW_BF16][GMAX];
+  float z[NW_BF16][GMAX];
+};
+static_assert(sizeof(RCComb) <= STAGE_BYTES, "the combine buffer lives in one stage");
+
+// Per-CTA slot in rank 0's gather area: O[r][HD] (unnormalised), m[8], Z[8].
+__host__ __device__ constexpr int rc_slot_floats(int r) { return r * HD + 2 * GMAX; }
+
+// Dynamic shared memory: header | gather (cs slots) | nst stages, each part
+// 1024-byte aligned (the stages hold 128-byte-swizzled TMA tiles).
+__host__ __device__ constexpr size_t rc_align(size_t x) { return (x + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr size_t rc_header_bytes() { return rc_align(sizeof(SmemRC)); }
+__host__ __device__ constexpr size_t rc_gather_bytes(int cs, int r) {
+  return rc_align((size_t)cs * rc_slot_floats(r) * 4);
+}
+__host__ __device__ constexpr size_t rc_smem_bytes(int cs, int r, int nst) {
+  return rc_header_bytes() + rc_gather_bytes(cs, r) + (size_t)nst * STAGE_BYTES;
 }
 
 __global__ void __launch_bounds__(NTHR_BF16, 2)
@@ -1205,14 +1567,16 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   SmemRC& sm = *reinterpret_cast<SmemRC*>(base);
-  uint8_t* stages = base + RC_FIXED_BYTES;
-  SmemCommon& c = sm.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int CS = (int)gridDim.x;
+  const int r = p.r;
+  float* gather = reinterpret_cast<float*>(base + rc_header_bytes());
+  uint8_t* stages = base + rc_header_bytes() + rc_gather_bytes(CS, r);
   const uint32_t rank = cluster_ctarank();
   const int bh = (int)blockIdx.y;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int nst = p.nst, upc = p.upc;
+  const int slot = rc_slot_floats(r);
 
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
@@ -1220,7 +1584,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       mbar_init(&sm.fullV_bar[s], 1);
       mbar_init(&sm.empty_bar[s], NW_BF16);
     }
-    c.misc[4] = 0;
+    sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (tid == 32) {
@@ -1228,7 +1592,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
     prefetch_tensormap(&tmV);
   }
   __syncthreads();
-  volatile int* abort_flag = &c.misc[4];
+  // first phase of the cluster barrier: every CTA has started (waited on
+  // before the first store into a peer's shared memory)
+  cluster_arrive_relaxed();
+  volatile int* abort_flag = &sm.abort_flag;
   const int seqlen = valid_seqlen(p, b, rank == 0 && h == 0 && tid == 0);
   const int nb = (seqlen + BLK - 1) / BLK;
   const int kp = min(p.k, nb);
@@ -1239,22 +1606,35 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
   (void)tn;
   (void)tcta;
   if (tid == 32) {
-    uint32_t smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    HYLRA_TRACE_CTA(tn, tcta, (1 << 8) | (smid & 0xff));
+    HYLRA_TRACE_CTA(tn, tcta, 1 << 8);
+    HYLRA_TRACE_VAL(tn, tcta, 41 << 8, HYLRA_CLOCK());
   }
+  const uint8_t* qsrc =
+      static_cast<const uint8_t*>(p.q) + ((size_t)b * p.Hq + (size_t)h * r) * HD * 2;
+  const uint32_t qbytes = (uint32_t)(r * HD * 2);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (p.idx_wait) griddep_wait();  // indices written by the preceding kernel
+    // With q_wait the query (and the block holding the newest token) come
+    // from the preceding kernel: they are read after griddep_wait.  Before
+    // it, the K/V tiles of the first nst blocks are requested, and q and
+    // everything else this CTA will read are brought into L2.
+    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+    bool waited = false;
+    if (p.idx_wait) {
+      griddep_wait();  // indices written by the preceding kernel
+      waited = true;
+    }
+    if (lane == 0 && p.q_wait && !waited) prefetch_l2_bulk(qsrc, qbytes);
+    // this CTA's first 32 indices, one per lane, in one round trip
+    int my_blk = lane < nu ? __ldcg(idx + j0 + lane) : -1;
     if (rank == 0) {
       // a reused list naming one block twice counts that block twice: flag it
       for (int i = lane; i < MAX_NB / 32; i += 32) sm.seen[i] = 0u;
       __syncwarp();
-      const int32_t* idx = p.topk_in + (size_t)bh * p.k;
       bool dup = false;
       for (int e = lane; e < kp; e += 32) {
-        const int32_t v = __ldcg(idx + e);
+        const int32_t v = e < nu && e < 32 ? my_blk : __ldcg(idx + e);  // rank 0: j0 = 0
         if (v >= 0 && v < nb) {
           const uint32_t bit = 1u << (v & 31);
           dup |= (atomicOr(&sm.seen[v >> 5], bit) & bit) != 0u;
@@ -1262,55 +1642,78 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       }
       if (__any_sync(0xffffffffu, dup) && lane == 0) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
     }
-    if (lane == 0) {
-      griddep_launch_dependents();     // the producer writes nothing
-      int tp = 128;
-      (void)tp;
-      HYLRA_TRACE_CTA(tp, tcta, 2 << 8);
-      const uint64_t pol = l2_evict_first_policy();
-      const long long row0 = row_base(p, b, h);
-      const uint32_t qbytes = (uint32_t)(p.r * HD * 2);
-      const int32_t* idx = p.topk_in + (size_t)bh * p.k + j0;
-      int blk_next = nu > 0 ? __ldcg(idx) : -1;
-      for (int i = 0; i < nu; ++i) {
-        const int s = i % nst;
-        const uint32_t ph = (uint32_t)((i / nst) & 1);
-        int blk = blk_next;
-        if (i + 1 < nu) blk_next = __ldcg(idx + i + 1);
-        mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
-        if (blk < 0 || blk >= nb) {
-          if (blk != -1) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
-          blk = -1;
-        }
-        sm.meta_blk[s] = blk;
-        sm.meta_nvalid[s] = blk >= 0 ? min(BLK, seqlen - blk * BLK) : 0;
-        uint32_t bytesK = (i == 0 ? qbytes : 0u) + (blk >= 0 ? 2u * BOX_BYTES : 0u);
-        uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
-        if (*abort_flag) bytesK = bytesV = 0u;
-        uint8_t* st = stages + (size_t)s * STAGE_BYTES;
-        const int row = (int)(row0 + (long long)blk * BLK);
-        if (bytesK) {
-          mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
-          if (i == 0)
-            bulk_load(sm.qbuf,
-                      static_cast<const uint8_t*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.r) * HD * 2,
-                      qbytes, &sm.fullK_bar[s]);
-          if (blk >= 0) {
-            tma_load_2d(st, &tmK, 0, row, &sm.fullK_bar[s], pol);
-            tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.fullK_bar[s], pol);
-          }
-        } else {
-          mbar_arrive(&sm.fullK_bar[s]);
-        }
-        if (bytesV) {
-          mbar_arrive_expect_tx(&sm.fullV_bar[s], bytesV);
-          tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.fullV_bar[s], pol);
-          tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.fullV_bar[s], pol);
-        } else {
-          mbar_arrive(&sm.fullV_bar[s]);
-        }
-      }
+    griddep_launch_dependents();  // the producer writes nothing
+    int tp = 128;  // trace events of the producer thread
+    (void)tp;
+    if (lane == 0) HYLRA_TRACE_CTA(tp, tcta, 2 << 8);
+    const uint64_t pol = l2_evict_first_policy();
+    const long long row0 = row_base(p, b, h);
+    // blocks beyond the pipeline depth (and, with q_wait, the newest block)
+    // into L2 now: lane i holds this CTA's i-th block
+    if (lane < nu && my_blk >= 0 && my_blk < nb &&
+        (lane >= nst || (p.q_wait && !waited && my_blk == nb - 1))) {
+      const int row = (int)(row0 + (long long)my_blk * BLK);
+      tma_prefetch_l2_2d(&tmK, 0, row);
+      tma_prefetch_l2_2d(&tmK, 64, row);
+      tma_prefetch_l2_2d(&tmV, 0, row);
+      tma_prefetch_l2_2d(&tmV, 64, row);
     }
+    int qpend = 0;
+    for (int i = 0; i < nu; ++i) {
+      const int s = i % nst;
+      const uint32_t ph = (uint32_t)((i / nst) & 1);
+      int blk = i < 32 ? __shfl_sync(0xffffffffu, my_blk, i) : 0;
+      if (lane != 0) continue;
+      if (i >= 32) blk = __ldcg(idx + j0 + i);
+      if (blk < 0 || blk >= nb) {
+        if (blk != -1) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
+        blk = -1;
+      }
+      // a stage is refilled only after the consumers used it, which needs
+      // q; the block holding the newest token is read after the wait too
+      if (p.q_wait && !waited && (i >= nst || blk == nb - 1)) {
+        griddep_wait();
+        waited = true;
+        if (qpend && !*abort_flag) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
+        qpend = 0;
+      }
+      mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
+      sm.meta_blk[s] = blk;
+      sm.meta_nvalid[s] = blk >= 0 ? min(BLK, seqlen - blk * BLK) : 0;
+      uint32_t bytesK = (i == 0 ? qbytes : 0u) + (blk >= 0 ? 2u * BOX_BYTES : 0u);
+      uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
+      if (*abort_flag) bytesK = bytesV = 0u;
+      uint8_t* st = stages + (size_t)s * STAGE_BYTES;
+      const int row = (int)(row0 + (long long)blk * BLK);
+      if (bytesK) {
+        mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
+        if (i == 0) {
+          if (p.q_wait && !waited)
+            qpend = 1;
+          else
+            bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[s]);
+        }
+        if (blk >= 0) {
+          tma_load_2d(st, &tmK, 0, row, &sm.fullK_bar[s], pol);
+          tma_load_2d(st + BOX_BYTES, &tmK, 64, row, &sm.fullK_bar[s], pol);
+        }
+      } else {
+        mbar_arrive(&sm.fullK_bar[s]);
+      }
+      if (bytesV) {
+        mbar_arrive_expect_tx(&sm.fullV_bar[s], bytesV);
+        tma_load_2d(st + 2 * BOX_BYTES, &tmV, 0, row, &sm.fullV_bar[s], pol);
+        tma_load_2d(st + 3 * BOX_BYTES, &tmV, 64, row, &sm.fullV_bar[s], pol);
+      } else {
+        mbar_arrive(&sm.fullV_bar[s]);
+      }
+      HYLRA_TRACE_CTA(tp, tcta, (12 << 8) | (i & 0x7f) | (waited ? 0x80 : 0));
+    }
+    if (lane == 0 && p.q_wait && !waited) {
+      griddep_wait();
+      if (qpend && !*abort_flag) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ consumers
     const int cw = warp - 1;
@@ -1325,7 +1728,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       const uint32_t ph = (uint32_t)((i / nst) & 1);
       mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
-      if (i == 0) wa.load_q(sm.qbuf, p.r);
+      if (i == 0) wa.load_q(sm.qbuf, r);
       const int blk = sm.meta_blk[s];
       if (blk >= 0) {
         float mxA, mxB, sA, sB;
@@ -1338,82 +1741,92 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
     }
     if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
-    // this CTA's state: eight warps -> four -> one (into sm.part)
-    wa.to_comb(c, cw);
-    for (int pr = ct; pr < p.r * HD; pr += NT_BF16) {
-      const int g = pr / HD, d = pr - g * HD;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NCOMB; ++w) M = fmaxf(M, c.comb_m[w][g]);
-      float O = 0.f, Z = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCOMB; ++w) {
-        const float mw = c.comb_m[w][g];
-        const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-        O = fmaf(c.comb_o[w][g][d], f, O);
-        Z = fmaf(c.comb_z[w][g], f, Z);
-      }
-      sm.part[g * HD + d] = O;
-      if (d == 0) {
-        sm.part[GMAX * HD + g] = M;
-        sm.part[GMAX * HD + GMAX + g] = Z;
-      }
-    }
-  }
-  __syncwarp();
-  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
-  cluster_sync_all();  // every CTA's state is in its shared memory
-  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 6 << 8);
-
-  if (rank == 0 && warp > 0) {
-    // ------------------------------------------------- merge (CTA rank 0)
-    // One pass over distributed shared memory: each thread loads, for its
-    // head and two output columns, every CTA's (max, sum, O) at once.
-    const int ct = tid - 32;
-    const int r = p.r;
-    const uint32_t part0 = smem_u32(sm.part);
-    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 10 << 8);
+    // this CTA's state: the eight warp states (on the now idle stage area)
+    // merged into one, stored into slot `rank` of CTA 0's gather area
+    RCComb& cb = *reinterpret_cast<RCComb*>(stages);
+    named_bar_sync(BAR_CONS, NT_BF16);  // every warp is done with the stages
+    wa.store_state(cb.o[cw], cb.m[cw], cb.z[cw]);
+    named_bar_sync(BAR_CONS, NT_BF16);
+    cluster_wait_acquire();  // first phase: every CTA of the cluster has started
+    const uint32_t dst = mapa_shared(smem_u32(gather), 0u) + (uint32_t)((int)rank * slot) * 4u;
     for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
       const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
-      float2 v[16];
-      float mj[16], zj[16];
+      float mw[NW_BF16];
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW_BF16; ++w) {
+        mw[w] = cb.m[w][g];
+        M = fmaxf(M, mw[w]);
+      }
+      float o0 = 0.f, o1 = 0.f, Z = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW_BF16; ++w) {
+        const float f = (M == -INFINITY || mw[w] == -INFINITY) ? 0.f : ex2_approx(mw[w] - M);
+        const float2 ov = *reinterpret_cast<const float2*>(&cb.o[w][g][col]);
+        o0 = fmaf(ov.x, f, o0);
+        o1 = fmaf(ov.y, f, o1);
+        Z = fmaf(cb.z[w][g], f, Z);
+      }
+      st_dsmem_f32x2(dst + (uint32_t)(g * HD + col) * 4u, o0, o1);
+      if (col == 0) st_dsmem_f32x2(dst + (uint32_t)(r * HD + 2 * g) * 4u, M, Z);
+    }
+    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
+  }
+  if (warp == 0) cluster_wait_acquire();  // first phase (the producer warp)
+  // second phase: every slot of CTA 0's gather area is written
+  cluster_arrive_release();
+  if (rank != 0) {
+    if (*abort_flag && tid == 32) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
+    return;  // nothing reads this CTA's shared memory
+  }
+  cluster_wait_acquire();
+  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 6 << 8);
+  if (warp > 0) {
+    // ------------------------------------------------- merge (CTA rank 0)
+    const int ct = tid - 32;
+    bool waited = false;
+    for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
+      const int g = pr / (HD / 2), col = 2 * (pr % (HD / 2));
+      // every slot's (m, Z) and O pair loaded at once (unrolled, predicated)
+      float2 mz[16], v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
+        mz[j] = make_float2(-INFINITY, 0.f);
+        v[j] = make_float2(0.f, 0.f);
         if (j < CS) {
-          const uint32_t a = mapa_shared(part0, (uint32_t)j);
-          v[j] = ld_dsmem_f32x2(a + (g * HD + col) * 4);
-          mj[j] = ld_dsmem_f32(a + (GMAX * HD + g) * 4);
-          zj[j] = ld_dsmem_f32(a + (GMAX * HD + GMAX + g) * 4);
+          const float* sl = gather + j * slot;
+          mz[j] = *reinterpret_cast<const float2*>(sl + r * HD + 2 * g);
+          v[j] = *reinterpret_cast<const float2*>(sl + g * HD + col);
         }
       }
       float M = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j < CS) M = fmaxf(M, mj[j]);
-      float Z = 0.f;
-      float2 acc = make_float2(0.f, 0.f);
+      for (int j = 0; j < 16; ++j) M = fmaxf(M, mz[j].x);
+      float Z = 0.f, a0 = 0.f, a1 = 0.f;
+      if (M != -INFINITY) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j < CS) {
-          const float f = (M == -INFINITY || mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - M);
-          Z = fmaf(zj[j], f, Z);
-          acc.x = fmaf(v[j].x, f, acc.x);
-          acc.y = fmaf(v[j].y, f, acc.y);
+        for (int j = 0; j < 16; ++j) {
+          const float f = mz[j].x == -INFINITY ? 0.f : ex2_approx(mz[j].x - M);
+          Z = fmaf(mz[j].y, f, Z);
+          a0 = fmaf(v[j].x, f, a0);
+          a1 = fmaf(v[j].y, f, a1);
         }
       }
       float2 o = make_float2(0.f, 0.f);
-      if (Z > 0.f) o = make_float2(acc.x / Z, acc.y / Z);
-      if (pr == ct) {
+      if (Z > 0.f) o = make_float2(a0 / Z, a1 / Z);
+      if (!waited) {
         if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 11 << 8);
         griddep_wait();  // the preceding kernel has completed before out is written
+        waited = true;
       }
       *reinterpret_cast<float2*>(p.out + ((size_t)b * p.Hq + (size_t)h * r + g) * HD + col) = o;
     }
   }
   __syncwarp();
-  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 7 << 8);
-  cluster_sync_all();  // keep every CTA's shared memory alive until rank 0 is done
-  if (tid == 32) HYLRA_TRACE_CTA(tn, tcta, 9 << 8);
+  if (tid == 32) {
+    HYLRA_TRACE_CTA(tn, tcta, 9 << 8);
+    HYLRA_TRACE_VAL(tn, tcta, 42 << 8, HYLRA_CLOCK());
+  }
   if (*abort_flag && tid == 32) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
 }
 
@@ -1424,7 +1837,11 @@ __global__ void __launch_bounds__(NT_F32, 1) decode_f32_kernel(const __grid_cons
   __shared__ SmemF32 sm;
   SmemCommon& c = sm.c;
   const int ct = threadIdx.x, cw = ct >> 5, lane = ct & 31;
-  if (ct == 0) c.nseg = 0;
+  if (ct == 0) {
+    c.nseg = 0;
+    c.trace_n = 0;
+    c.trace_cta = (int)blockIdx.x;
+  }
   build_prefix(p, c, FULL);
   __syncthreads();
   const int T = c.prefix[p.B];

@@ -233,6 +233,18 @@ def test_many_equal_scores_take_the_radix_path():
     assert np.all(tk[0] == np.arange(20))
 
 
+@pytest.mark.parametrize("nblocks", [200, 256, 257])
+def test_equal_scores_rank_by_block_index(nblocks):
+    """Every block of equal mass, on both sides of the one-key-per-thread
+    selection limit (256 blocks): ranks must follow block index."""
+    w = W.custom(f"ties_{nblocks}", batch=1, seqlens=(128 * nblocks,), num_q_heads=8,
+                 num_kv_heads=2, topk=24, seed=27)
+    q, K, V = _layer(w)
+    K = torch.zeros_like(K)
+    _, _, _, tk, _ = _full_and_check(w, inputs=(q, K, V))
+    assert np.all(tk[0] == np.arange(24))
+
+
 def test_k_larger_than_the_merge_thread_count():
     """k = 300 > 256 selection threads: the radix select path."""
     w = W.custom("bigk", batch=1, seqlens=(128 * 400 - 17,), num_q_heads=8, num_kv_heads=2,
