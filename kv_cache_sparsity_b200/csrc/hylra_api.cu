@@ -21,6 +21,7 @@ using namespace hylra;
 namespace {
 
 constexpr size_t kSmemBF16 = sizeof(SmemBF16) + 1024;  // + alignment slack
+constexpr int LATE_DEFICIT = 2;  // units fewer for streaming CTAs that start late
 static_assert(kSmemBF16 <= 232448, "bf16 kernel shared memory exceeds 227 KB");
 constexpr size_t kSmemMax = 232448;  // 227 KB of dynamic shared memory per CTA
 static_assert(rc_smem_bytes(1, HYLRA_MAX_GROUP, 1) + 1024 <= kSmemMax,
@@ -201,6 +202,7 @@ int rc_max_active(const RCPlan& pl) {
 
 #ifdef HYLRA_TRACE
 int g_plan_cs = 0, g_plan_nst = 0;  // tuning builds: force a plan
+int g_late_deficit = -1;            // tuning builds: force the late-start deficit
 #endif
 
 // A small reuse layer (fewer blocks than SMs) is a latency chain: inside a
@@ -267,7 +269,8 @@ int check_layer_ptrs(const hylra_shape_t* s, const void* q, const void* K, const
 int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, const void* V,
            const int32_t* seqlens, const int32_t* topk_in, float* out, int32_t* topk_out,
            void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl = false,
-           bool idx_from_prev = true, int trace_slot = 0) {
+           bool idx_from_prev = true, int trace_slot = 0, int late_ctas = 0,
+           int* last_ctas = nullptr) {
   int rc = check_shape(s);
   if (rc) return rc;
   if ((rc = check_layer_ptrs(s, q, K, V, out))) return rc;
@@ -303,6 +306,15 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.max_seqlen = s->max_seqlen;
   p.nbmax = L.nbmax;
   p.idx_wait = idx_from_prev ? 1 : 0;
+  // CTAs launched early beside the preceding kernel stage their first blocks
+  // before it ends; the last late_ctas of the grid find their SMs still held
+  // and start after it: they take LATE_DEFICIT units fewer (bf16 streaming)
+  p.late_from = G - std::min(G, std::max(0, late_ctas));
+  p.late_deficit = pdl && late_ctas > 0 ? LATE_DEFICIT : 0;
+#ifdef HYLRA_TRACE
+  if (g_late_deficit >= 0 && p.late_deficit > 0) p.late_deficit = g_late_deficit;
+#endif
+  if (last_ctas) *last_ctas = 0;
   p.q_wait = pdl ? 1 : 0;
   p.trace_slot = trace_slot;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
@@ -338,6 +350,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
         cfg.numAttrs = pdl ? 2 : 1;
         if (cudaLaunchKernelEx(&cfg, decode_reuse_cluster_kernel, tmK, tmV, p) != cudaSuccess)
           return HYLRA_ERR_CUDA;
+        if (last_ctas) *last_ctas = pl.cs * nbh;
         return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
       }
     }
@@ -366,6 +379,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
                                 : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
     if (em != cudaSuccess) return HYLRA_ERR_CUDA;
+    if (last_ctas) *last_ctas = s->batch * s->num_kv_heads;
   } else {
     if (full)
       decode_f32_kernel<true><<<G, NT_F32, 0, stream>>>(p);
@@ -439,15 +453,17 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint
   }
   const size_t per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
   int last_reset = 0;
+  int prev_ctas = 0;  // CTAs of the kernel launched last (each holds an SM)
   for (int l = 0; l < num_layers; ++l) {
     if (policy[l]) {
       last_reset = l;
       rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
-                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0, true, l & 63);
+                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0, true, l & 63,
+                  prev_ctas, &prev_ctas);
     } else {
       rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
                   nullptr, workspace, workspace_bytes, (cudaStream_t)stream, l > 0,
-                  last_reset == l - 1, l & 63);
+                  last_reset == l - 1, l & 63, prev_ctas, &prev_ctas);
     }
     if (rc) return rc;
   }
@@ -494,6 +510,11 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
 int hylra_plan_override(int cs, int nst) {
   g_plan_cs = cs;
   g_plan_nst = nst;
+  return HYLRA_OK;
+}
+
+int hylra_late_override(int d) {
+  g_late_deficit = d;
   return HYLRA_OK;
 }
 

@@ -121,6 +121,8 @@ struct Params {
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
   int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
+  int late_from;     // bf16 streaming kernel: CTAs >= late_from start late (their SM is
+  int late_deficit;  // still held by the preceding kernel) and take this many units fewer
   int q_wait;        // q and each sequence's newest K/V row come from the preceding kernel
   int upc, nst;      // cluster reuse kernel: blocks per CTA, pipeline stages
   int trace_slot;    // trace builds: which per-launch region of the trace buffer
@@ -216,6 +218,29 @@ __device__ __forceinline__ int units_of(const Params& p, int n, bool full) {
 // First row of (b, h) in the 2-D [rows][d] view of K or V.
 __device__ __forceinline__ long long row_base(const Params& p, int b, int h) {
   return p.cap > 0 ? ((long long)b * p.Hkv + h) * p.cap : (long long)h * p.total + p.seq_off[b];
+}
+
+// Static share of the bf16 streaming kernel: CTA c holds units
+// [part_lo(c), part_lo(c+1)).  The CTAs from E on start late (inside a decode
+// step their SMs are still held by the preceding kernel while the others
+// already stage their first blocks), so each takes D units fewer than the
+// rest; D applies only when every late CTA still gets a unit.
+__device__ __forceinline__ int late_deficit(const Params& p, long long T, int G) {
+  const long long E = min(max(p.late_from, 0), G), L = G - E, D = p.late_deficit;
+  return (D > 0 && L > 0 && T + L * D >= (long long)G * (D + 1)) ? (int)D : 0;
+}
+__device__ __forceinline__ long long part_lo(long long c, long long T, int G, int E, int D) {
+  const long long L = G - E;
+  return (c * (T + L * D) - (long long)D * G * max(0ll, c - E)) / G;
+}
+// CTA whose static share holds unit u (binary search over part_lo).
+__device__ __forceinline__ int part_owner(long long u, long long T, int G, int E, int D) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (part_lo(mid, T, G, E, D) <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // CTA that owns linear unit u when CTA c holds [floor(c*T/G), floor((c+1)*T/G));
@@ -1076,9 +1101,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   // least one unit (the contributor count of a (b, h) relies on it).
   const int T = c.prefix[p.B];
   const int G = T > 0 ? min((int)gridDim.x, T) : 1;
+  const int E = min(max(p.late_from, 0), G), D = late_deficit(p, T, G);
   const bool works = (int)blockIdx.x < G;
-  const int lo = works ? (int)((long long)blockIdx.x * T / G) : 0;
-  const int hi = works ? (int)((long long)(blockIdx.x + 1) * T / G) : 0;
+  const int lo = works ? (int)part_lo(blockIdx.x, T, G, E, D) : 0;
+  const int hi = works ? (int)part_lo(blockIdx.x + 1, T, G, E, D) : 0;
   const int n = hi - lo;
   // Programmatic launch between layers.  Every global write (and a reuse
   // layer's read of indices its immediate predecessor wrote) comes after
@@ -1315,11 +1341,14 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int T = c.prefix[p.B];
   const int U = (c.prefix[b + 1] - c.prefix[b]) / p.Hkv;
   const int G = min(grid_stream, max(T, 1));
+  const int E = min(max(p.late_from, 0), G), D = late_deficit(p, T, G);
   const int start = c.prefix[b] + h * U;
   int first = 0, nc = 0;
   if (U > 0) {
-    first = owner_cta(start, T, G);
-    nc = owner_cta((long long)start + U - 1, T, G) - first + 1;
+    // the streaming kernel's static split (part_lo): every CTA of it owns
+    // at least one unit, so the owners of (b, h) are contiguous
+    first = part_owner(start, T, G, E, D);
+    nc = part_owner((long long)start + U - 1, T, G, E, D) - first + 1;
     first += bh;  // partial slot of contributor c is c + bh
   }
   const int nb = (seqlen + BLK - 1) / BLK;
