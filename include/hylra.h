@@ -68,8 +68,7 @@ typedef enum {
   HYLRA_ERR_INVALID = -1,      /* null pointer, bad size, misaligned pointer   */
   HYLRA_ERR_UNSUPPORTED = -2,  /* d != 128, block != 128, r > 8, limits above  */
   HYLRA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed            */
-  HYLRA_ERR_WORKSPACE = -4,    /* workspace smaller than hylra_workspace_bytes */
-  HYLRA_ERR_INFEASIBLE = -5    /* no policy satisfies the constraints          */
+  HYLRA_ERR_WORKSPACE = -4     /* workspace smaller than hylra_workspace_bytes */
 } hylra_error_t;
 
 typedef enum { HYLRA_BF16 = 0, HYLRA_FP32 = 1 } hylra_dtype_t;
@@ -128,7 +127,13 @@ int hylra_decode_reuse(const hylra_shape_t* shape, const void* q, const void* K,
  * hylra_decode_reuse when policy[l] == 0 (reading the slot of the most recent
  * reset layer).  policy[0] must be 1.  q, K, V, out: HOST arrays of
  * num_layers DEVICE pointers.  topk: device int32 [num_layers][B][Hkv][k];
- * slots of reuse layers are left untouched.  Capturable in a CUDA graph. */
+ * slots of reuse layers are left untouched.  Capturable in a CUDA graph.
+ * Layers are ordered as in a model, where a layer's query and its newest
+ * K/V row are computed from the previous layer's output: layer l > 0 reads
+ * q[l] and the block holding each sequence's newest token only after layer
+ * l-1's kernels have completed (its kernels are launched early, as
+ * programmatic dependents, and may only stage older K/V blocks before
+ * that).  The step time is thus a sum of per-layer latencies. */
 int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers,
                       const uint8_t* policy, const void* const* q,
                       const void* const* K, const void* const* V,
