@@ -218,18 +218,55 @@ def graph_kernel_nodes(g) -> int:
     return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
 
 
-def derive_policy(m: Model, H):
-    """Profiling run (every layer full) -> overlap matrix -> DP policy."""
+def policy_rule(args, w) -> str:
+    if args.policy == "jump3":
+        return "jump3 (reset every 3rd layer)"
+    if w.policy is not None:
+        return "fixed by the workload"
+    theta = w.theta if args.theta is None else args.theta
+    return f"dp theta={theta:g} profile_steps={max(1, args.profile_steps)}"
+
+
+def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int = 1):
+    """The step's reset/reuse policy.
+
+    dp: profiling run(s) with every layer full -> overlap matrix -> DP policy
+    (HyLRA summary §2.2).  With profile_steps P > 1 the index sets of P decode
+    steps (fresh queries, same cache) are pooled into one matrix.  A workload
+    with a fixed policy keeps it.  jump3: a reset every third layer (the
+    static baseline of §4)."""
     w = m.w
+    if rule == "jump3":
+        pol, _ = H.static_policy(w.layers, 3)
+        return pol, None
     if w.policy is not None:
         return tuple(w.policy), None
     allfull = (1,) * w.layers
-    m.step(allfull)
-    torch.cuda.synchronize()
-    tk = m.topk.cpu().numpy().reshape(w.layers, w.batch * w.num_kv_heads, w.topk)
-    M = H.similarity(tk)
-    pol, R, S = H.dp_policy(M, w.theta)
+    sets = []
+    q0 = list(m.q)
+    for p in range(max(1, profile_steps)):
+        if p > 0:
+            m.q = [W.step_query(w, l, p, device="cuda") for l in range(w.layers)]
+        m.step(allfull)
+        torch.cuda.synchronize()
+        sets.append(m.topk.cpu().numpy().reshape(w.layers, w.batch * w.num_kv_heads, w.topk))
+    m.q = q0
+    M = H.similarity(np.concatenate(sets, axis=1))
+    pol, R, S = H.dp_policy(M, w.theta if theta is None else theta)
     return pol, M
+
+
+def output_error_vs_full(m: Model, g_h, g_f):
+    """Relative Frobenius error of each layer's hybrid output against full
+    attention on the same inputs (a synthetic stand-in for the pages'
+    accuracy comparison): (mean over reuse layers, max over layers)."""
+    g_h.replay()
+    torch.cuda.synchronize()
+    oh = [o.clone() for o in m.outs]
+    g_f.replay()
+    torch.cuda.synchronize()
+    errs = [float((a - b).norm() / b.norm().clamp_min(1e-30)) for a, b in zip(oh, m.outs)]
+    return errs
 
 
 def timed_replays(g, steps, dist_on):
@@ -335,7 +372,7 @@ def run_ours(args, rank, world, dist_on):
     if per_layer * w.layers > free * 0.85:
         resident = max(1, int(free * 0.85 // per_layer))
     m = Model(w, H, resident)
-    policy, M = derive_policy(m, H)
+    policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps)
     allfull = (1,) * w.layers
     R = sum(policy)
     g_h = m.graph(policy)
@@ -368,6 +405,8 @@ def run_ours(args, rank, world, dist_on):
                                      dist_on)
     e2e_ms = max_over_ranks(e2e_ms, dist_on)
     g_launches = g_h.kernel_nodes
+    errs = output_error_vs_full(m, g_h, g_f)
+    reuse_errs = [e for e, x in zip(errs, policy) if not x] or [0.0]
     del g_h, g_f
 
     full_b = w.kv_bytes_per_layer()
@@ -394,6 +433,7 @@ def run_ours(args, rank, world, dist_on):
         "config": {
             "workload": workload_desc(w),
             "policy": "".join("R" if x else "U" for x in policy),
+            "policy_rule": policy_rule(args, w),
             "resets": R,
             "resident_layer_caches": m.resident,
             "l2": "inputs larger than L2: a step streams %.2f GB" % (step_bytes / 1e9),
@@ -420,6 +460,8 @@ def run_ours(args, rank, world, dist_on):
         "e2e": {"value": round(e2e_ms * 1000.0, 3), "unit": "us/step",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": g_launches * args.steps,
+        "quality_vs_full": {"rel_err_mean_reuse_layers": round(statistics.mean(reuse_errs), 5),
+                            "rel_err_max": round(max(errs), 5)},
         "clocks": clocks,
         "device_status": status,
     }
@@ -449,21 +491,25 @@ def run_reference(args):
         m.Ks.append(K)
         m.Vs.append(V)
     # policy: the oracle's own profiling + DP on this sample (every layer full)
-    if w.policy is not None:
+    if args.policy == "jump3":
+        policy, _ = O.static_policy(w.layers, 3)
+    elif w.policy is not None:
         policy = tuple(w.policy)
     else:
         sets = []
         for l in range(w.layers):
             per = []
-            for b in range(w.batch):
-                kb = W.per_sequence(w, m.Ks[l], b).double().numpy()
-                vb = W.per_sequence(w, m.Vs[l], b).double().numpy()
-                _, _, tk = O.full_layer(m.q[l][b].double().numpy(), kb, vb, w.seqlens[b],
-                                        w.topk)
-                per.extend(list(tk))
+            for p in range(max(1, args.profile_steps)):
+                ql = m.q[l] if p == 0 else W.step_query(w, l, p, device="cpu")
+                for b in range(w.batch):
+                    kb = W.per_sequence(w, m.Ks[l], b).double().numpy()
+                    vb = W.per_sequence(w, m.Vs[l], b).double().numpy()
+                    _, _, tk = O.full_layer(ql[b].double().numpy(), kb, vb, w.seqlens[b],
+                                            w.topk)
+                    per.extend(list(tk))
             sets.append(per)
         M = O.similarity_matrix(np.array(sets))
-        policy, _, _ = O.dp_policy(M, w.theta)
+        policy, _, _ = O.dp_policy(M, w.theta if args.theta is None else args.theta)
     times = []
     for _ in range(args.warmup):
         oracle_sample(w, m, policy, heads=heads, reps=1)
@@ -488,7 +534,8 @@ def run_reference(args):
         "dtype": "f64",
         "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
         "config": {"workload": workload_desc(w),
-                   "policy": "".join("R" if x else "U" for x in policy)},
+                   "policy": "".join("R" if x else "U" for x in policy),
+                   "policy_rule": policy_rule(args, w)},
         "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
@@ -506,6 +553,12 @@ def main():
     ap.add_argument("--config", default="llama8b_32k", choices=W.CONFIG_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--policy", default="dp", choices=["dp", "jump3"],
+                    help="dp: profiled overlap matrix + DP (HyLRA); jump3: reset every 3rd layer")
+    ap.add_argument("--theta", type=float, default=None,
+                    help="DP threshold (default: the workload's, 0.8)")
+    ap.add_argument("--profile-steps", type=int, default=1,
+                    help="decode steps pooled into the profiled overlap matrix")
     ap.add_argument("--no-clock-fill", action="store_true",
                     help="skip the extra busy window for the clock sampler (profiler runs)")
     args = ap.parse_args()

@@ -175,6 +175,14 @@ int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k,
 int hylra_dp_policy(int32_t num_layers, const double* M, double theta,
                     uint8_t* policy, int32_t* num_resets, double* cum_similarity);
 
+/* Static policy (HyLRA summary §4 "Results": the Jump3 baseline, "a static
+ * variant with fixed jump steps"; read as a reset every `period` layers,
+ * Jump3 = period 3): policy[l] = 1 when l % period == 0, else 0, for
+ * l < num_layers.  policy: HOST uint8 [num_layers]; num_resets may be NULL.
+ * period >= 1.  Synchronous; no similarity threshold is applied. */
+int hylra_static_policy(int32_t num_layers, int32_t period, uint8_t* policy,
+                        int32_t* num_resets);
+
 /* hylra_decode_full without a caller-supplied workspace.  The paper has no
  * counterpart: this exists for callers that cannot allocate device memory
  * when they call (a process that reserved all free device memory up front,

@@ -146,4 +146,16 @@ int hylra_dp_policy(int32_t num_layers, const double* M, double theta, uint8_t* 
   return HYLRA_OK;
 }
 
+int hylra_static_policy(int32_t num_layers, int32_t period, uint8_t* policy,
+                        int32_t* num_resets) {
+  if (num_layers < 1 || period < 1 || !policy) return HYLRA_ERR_INVALID;
+  int32_t resets = 0;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    policy[l] = (l % period == 0) ? 1 : 0;
+    resets += policy[l];
+  }
+  if (num_resets) *num_resets = resets;
+  return HYLRA_OK;
+}
+
 }  // extern "C"

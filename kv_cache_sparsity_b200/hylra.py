@@ -40,7 +40,7 @@ ERRORS = {0: "HYLRA_OK", -1: "HYLRA_ERR_INVALID", -2: "HYLRA_ERR_UNSUPPORTED",
 EXPORTS = ("hylra_workspace_bytes", "hylra_workspace_init", "hylra_decode_full",
            "hylra_decode_reuse", "hylra_decode_step", "hylra_decode_step_host",
            "hylra_similarity", "hylra_dp_policy", "hylra_read_status", "hylra_strerror",
-           "hylra_version", "hylra_decode_full_noalloc")
+           "hylra_version", "hylra_decode_full_noalloc", "hylra_static_policy")
 
 
 class HylraError(RuntimeError):
@@ -95,6 +95,7 @@ def load() -> ctypes.CDLL:
                             ctypes.POINTER(ctypes.c_double)],
         "hylra_read_status": [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P],
         "hylra_decode_full_noalloc": [SP, P, P, P, P, P, P, P, P],
+        "hylra_static_policy": [I32, I32, P, ctypes.POINTER(I32)],
         "hylra_strerror": [ctypes.c_int],
         "hylra_version": [],
     }
@@ -223,3 +224,12 @@ def dp_policy(M: np.ndarray, theta: float):
     _check(load().hylra_dp_policy(L, m.ctypes.data, float(theta), pol.ctypes.data,
                                   ctypes.byref(R), ctypes.byref(S)), "hylra_dp_policy")
     return tuple(int(x) for x in pol), R.value, S.value
+
+
+def static_policy(num_layers: int, period: int):
+    """-> (policy tuple, resets): a reset every `period` layers (Jump3: 3)."""
+    pol = np.zeros(num_layers, dtype=np.uint8)
+    R = ctypes.c_int32(0)
+    _check(load().hylra_static_policy(int(num_layers), int(period), pol.ctypes.data,
+                                      ctypes.byref(R)), "hylra_static_policy")
+    return tuple(int(x) for x in pol), R.value

@@ -178,6 +178,26 @@ def _gen(device, seed: int) -> torch.Generator:
     return g
 
 
+def step_query(w: Workload, layer: int, step: int, device="cpu"):
+    """The query of one layer at decode step `step` ([B][Hq][d]); step 0 is the
+    query of layer_inputs.  Later steps draw fresh noise around the same
+    salient directions (the cache is left as it is: over a few profiled steps
+    its growth by one token each is negligible)."""
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    B, Hq, d = w.batch, w.num_q_heads, w.head_dim
+    base = (w.seed * 1000003 + layer * 101) * 4
+    # step 0: the layer's own stream; later steps: a distinct 32-bit seed
+    gq = _gen(device, (base + 1) ^ ((int(step) * 0x9E3779B1) & 0xFFFFFFFF))
+    if w.structure == "iid":
+        q = torch.randn(B, Hq, d, generator=gq, device=device)
+    else:
+        st = structure(w)
+        u = st.u.to(device)
+        q = math.sqrt(d) * u.repeat_interleave(w.group, dim=1) + torch.randn(
+            B, Hq, d, generator=gq, device=device)
+    return q.to(dt)
+
+
 def layer_inputs(w: Workload, layer: int, device="cpu"):
     """(q, K, V) of one layer, in the workload's dtype and layout, on ``device``.
 
@@ -185,17 +205,9 @@ def layer_inputs(w: Workload, layer: int, device="cpu"):
     """
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     B, Hq, H, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
-    r = w.group
     base = (w.seed * 1000003 + layer * 101) * 4
-    gq, gk, gv = _gen(device, base + 1), _gen(device, base + 2), _gen(device, base + 3)
-    if w.structure == "iid":
-        q = torch.randn(B, Hq, d, generator=gq, device=device)
-    else:
-        st = structure(w)
-        u = st.u.to(device)
-        q = math.sqrt(d) * u.repeat_interleave(r, dim=1) + torch.randn(
-            B, Hq, d, generator=gq, device=device)
-    q = q.to(dt)
+    gk, gv = _gen(device, base + 2), _gen(device, base + 3)
+    q = step_query(w, layer, 0, device)
 
     def key_rows(b, n, noise):
         # noise: [H, n, d] fp32 ; add the salient part for sequence b

@@ -365,3 +365,13 @@ def dp_policy_bruteforce(M: np.ndarray, theta: float):
             best = cand
     R, S, pol = best
     return pol, R, S
+
+
+def static_policy(num_layers: int, period: int):
+    """HyLRA summary §4 "Results", the Jump3 baseline ("a static variant with
+    fixed jump steps"), READING: a reset every `period` layers starting at
+    layer 0 (Jump3: period 3), with no similarity threshold."""
+    pol = []
+    for layer in range(num_layers):
+        pol.append(RESET if layer % period == 0 else REUSE)
+    return tuple(pol), sum(pol)

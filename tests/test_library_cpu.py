@@ -145,3 +145,46 @@ def test_dp_golden(lib):
 def test_dp_rejects_nan_theta(lib):
     with pytest.raises(H.HylraError):
         H.dp_policy(np.eye(3), float("nan"))
+
+
+@pytest.mark.parametrize("L,period", [(1, 3), (4, 3), (32, 3), (32, 1), (7, 7), (5, 9)])
+def test_static_policy_matches_oracle(lib, L, period):
+    assert H.static_policy(L, period) == O.static_policy(L, period)
+
+
+def test_static_policy_rejects_bad_period(lib):
+    with pytest.raises(H.HylraError):
+        H.static_policy(4, 0)
+
+
+def test_jump3_against_dp_on_the_same_matrix(lib):
+    """Where Jump3 is feasible under theta, the DP optimum never resets more."""
+    rng = np.random.default_rng(11)
+    for trial in range(40):
+        L = int(rng.integers(2, 13))
+        M = _dyadic(L, rng, denom=8)
+        theta = float(rng.choice([0.0, 0.25, 0.5]))
+        jump, Rj = H.static_policy(L, 3)
+        ok, Rc, _ = O.policy_cost(M, theta, jump)
+        assert Rc == Rj or not ok
+        _, Rdp, _ = H.dp_policy(M, theta)
+        if ok:
+            assert Rdp <= Rj
+
+
+def test_pooled_profiling_steps(lib):
+    """Index sets of several profiled decode steps pool into one matrix: P
+    copies of one step give that step's matrix; mixed steps match the oracle."""
+    rng = np.random.default_rng(21)
+    L, S, k, nb = 6, 8, 4, 24
+    steps = []
+    for p in range(3):
+        t = np.empty((L, S, k), dtype=np.int32)
+        for l in range(L):
+            for u in range(S):
+                t[l, u] = rng.permutation(nb)[:k]
+        steps.append(t)
+    one = H.similarity(steps[0])
+    assert H.similarity(np.concatenate([steps[0]] * 3, axis=1)).tobytes() == one.tobytes()
+    mixed = np.concatenate(steps, axis=1)
+    assert H.similarity(mixed).tobytes() == O.similarity_matrix(mixed).tobytes()

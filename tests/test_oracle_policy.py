@@ -92,3 +92,13 @@ def test_dp_strict_threshold():
     M = np.array([[1.0, 0.0], [0.5, 1.0]])
     assert O.dp_policy(M, 0.5)[0] == (1, 1)     # 0.5 does not exceed 0.5
     assert O.dp_policy(M, 0.4999)[0] == (1, 0)
+
+
+@pytest.mark.parametrize("L,period", [(1, 3), (2, 3), (3, 3), (4, 3), (10, 3), (32, 3), (9, 1),
+                                      (6, 6), (6, 100)])
+def test_static_policy_closed_form(L, period):
+    """A reset at layers 0, period, 2 period, ...: ceil(L / period) resets."""
+    pol, R = O.static_policy(L, period)
+    assert len(pol) == L and pol[0] == O.RESET
+    assert R == -(-L // period) == sum(pol)
+    assert [i for i, x in enumerate(pol) if x == O.RESET] == list(range(0, L, period))
