@@ -320,6 +320,64 @@ def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
     return ms, h2d, d2h
 
 
+def offload_measure(m: Model, H, policy, steps, warmup, dist_on):
+    """Index-guided offloading (HyLRA summary §2.4): the reuse layers' caches
+    move to pinned host memory and each reuse layer gathers only its reused
+    blocks across the host link.  Times the graph-replayed step and, for
+    reference, a plain host-to-device copy of the same bytes per step."""
+    w = m.w
+    offloaded = tuple(0 if x else 1 for x in policy)
+    Ko, Vo = [], []
+    host_bytes = 0
+    for l in range(w.layers):
+        if offloaded[l]:
+            Ko.append(m.Ks[l].cpu().pin_memory())
+            Vo.append(m.Vs[l].cpu().pin_memory())
+        else:
+            Ko.append(m.Ks[l])
+            Vo.append(m.Vs[l])
+    n = H.stage_bytes(m.shape) // 2
+    Ks = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    Vs = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        H.decode_step_offload(m.shape, policy, m.q, Ko, Vo, offloaded, m.seqlens, m.outs, m.topk,
+                              Ks, Vs, m.ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        H.decode_step_offload(m.shape, policy, m.q, Ko, Vo, offloaded, m.seqlens, m.outs, m.topk,
+                              Ks, Vs, m.ws, stream=torch.cuda.current_stream())
+    for _ in range(warmup):
+        g.replay()
+    ms = timed_replays(g, steps, dist_on)
+    # bytes that cross the link per step: k' blocks of K and V per (b, h) per
+    # offloaded layer
+    per_layer = w.kv_bytes_reuse_layer()
+    host_bytes = per_layer * sum(offloaded)
+    # a plain pinned-host-to-device copy of those bytes, for the link's rate
+    src = torch.empty(host_bytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(host_bytes, dtype=torch.uint8, device="cuda")
+    dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        dst.copy_(src, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    copy_ms = e0.elapsed_time(e1) / 3
+    del g
+    return {"us_per_step": round(ms * 1000.0, 3),
+            "offloaded_layers": int(sum(offloaded)),
+            "host_link_bytes_per_step": int(host_bytes),
+            "host_link_gbs": round(host_bytes / (ms * 1e-3) / 1e9, 1),
+            "plain_copy_gbs": round(host_bytes / (copy_ms * 1e-3) / 1e9, 1),
+            "device_cache_bytes_moved_to_host": int(w.kv_bytes_per_layer() * sum(offloaded))}
+
+
 def oracle_sample(w: W.Workload, m: Model, policy, heads=(0,), reps=1):
     """Time the fp64 oracle on a bounded sample of one decode step: all
     layers under ``policy`` for the KV heads ``heads`` of every sequence.
@@ -408,6 +466,8 @@ def run_ours(args, rank, world, dist_on):
     errs = output_error_vs_full(m, g_h, g_f)
     reuse_errs = [e for e, x in zip(errs, policy) if not x] or [0.0]
     del g_h, g_f
+    offload = (offload_measure(m, H, policy, max(3, args.steps // 4), args.warmup, dist_on)
+               if args.offload else None)
 
     full_b = w.kv_bytes_per_layer()
     reuse_b = w.kv_bytes_reuse_layer()
@@ -462,6 +522,7 @@ def run_ours(args, rank, world, dist_on):
         "gpu_launches": g_launches * args.steps,
         "quality_vs_full": {"rel_err_mean_reuse_layers": round(statistics.mean(reuse_errs), 5),
                             "rel_err_max": round(max(errs), 5)},
+        "offload": offload,
         "clocks": clocks,
         "device_status": status,
     }
@@ -557,6 +618,8 @@ def main():
                     help="dp: profiled overlap matrix + DP (HyLRA); jump3: reset every 3rd layer")
     ap.add_argument("--theta", type=float, default=None,
                     help="DP threshold (default: the workload's, 0.8)")
+    ap.add_argument("--offload", action="store_true",
+                    help="also time the step with the reuse layers' caches in host memory")
     ap.add_argument("--profile-steps", type=int, default=1,
                     help="decode steps pooled into the profiled overlap matrix")
     ap.add_argument("--no-clock-fill", action="store_true",

@@ -140,6 +140,47 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers,
                       const int32_t* seqlens, float* const* out, int32_t* topk,
                       void* workspace, size_t workspace_bytes, hylra_stream_t stream);
 
+/* Index-guided offloading (HyLRA summary §2.4 "Index-Guided Offloading":
+ * when the KV cache exceeds device memory, the reused indices name the only
+ * blocks a tolerant layer needs, so only those cross the host link).
+ *
+ * A host-resident cache has the same layout as a device cache (dense or
+ * packed, bf16) but lives in pinned host memory the device can address
+ * (cudaHostAlloc / cudaHostRegister with mapping; on systems with unified
+ * addressing the host pointer itself is passed).  The staging cache is a
+ * device buffer [B][Hkv][k][128][d] bf16 (hylra_stage_bytes each for K and
+ * V); its slot e of (b, h) holds block topk_in[b][h][e]. */
+
+/* Bytes of one staging cache (K or V) for this shape.  bf16 only. */
+int hylra_stage_bytes(const hylra_shape_t* shape, size_t* bytes);
+
+/* Copy the blocks listed in topk_in (device int32 [B][Hkv][k]; slots
+ * 0..k'-1, -1 and out-of-range entries skipped) from the host-resident
+ * K_host / V_host into the staging caches K_stage / V_stage (device); only
+ * a block's valid rows are copied.  Asynchronous on stream. */
+int hylra_gather_blocks(const hylra_shape_t* shape, const void* K_host, const void* V_host,
+                        const int32_t* seqlens, const int32_t* topk_in, void* K_stage,
+                        void* V_stage, hylra_stream_t stream);
+
+/* hylra_decode_reuse over staging caches written by hylra_gather_blocks with
+ * the same topk_in: same result as hylra_decode_reuse on the original cache. */
+int hylra_decode_reuse_staged(const hylra_shape_t* shape, const void* q, const void* K_stage,
+                              const void* V_stage, const int32_t* seqlens,
+                              const int32_t* topk_in, float* out, void* workspace,
+                              size_t workspace_bytes, hylra_stream_t stream);
+
+/* hylra_decode_step where offloaded[l] == 1 marks a reuse layer whose K[l],
+ * V[l] are host-resident: the layer gathers its reused blocks into K_stage /
+ * V_stage (one pair, reused layer after layer) and runs on them.  Reset
+ * layers must be device-resident (HYLRA_ERR_INVALID otherwise).  offloaded:
+ * HOST uint8 [num_layers]. */
+int hylra_decode_step_offload(const hylra_shape_t* shape, int32_t num_layers,
+                              const uint8_t* policy, const void* const* q,
+                              const void* const* K, const void* const* V,
+                              const uint8_t* offloaded, const int32_t* seqlens,
+                              float* const* out, int32_t* topk, void* K_stage, void* V_stage,
+                              void* workspace, size_t workspace_bytes, hylra_stream_t stream);
+
 /* The same step with the per-step inputs and outputs in HOST memory:
  * q_host [num_layers][B][Hq][d] is copied to q_dev (same shape, device) and,
  * after the step, out_dev [num_layers][B][Hq][d] fp32 to out_host and

@@ -270,9 +270,10 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
            const int32_t* seqlens, const int32_t* topk_in, float* out, int32_t* topk_out,
            void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl = false,
            bool idx_from_prev = true, int trace_slot = 0, int late_ctas = 0,
-           int* last_ctas = nullptr) {
+           int* last_ctas = nullptr, bool staged = false) {
   int rc = check_shape(s);
   if (rc) return rc;
+  if (staged && (full || s->dtype != HYLRA_BF16)) return HYLRA_ERR_UNSUPPORTED;
   if ((rc = check_layer_ptrs(s, q, K, V, out))) return rc;
   if (!seqlens || !ws || !aligned(seqlens, 4) || !aligned(ws, 256)) return HYLRA_ERR_INVALID;
   if (full && (!topk_out || !aligned(topk_out, 4))) return HYLRA_ERR_INVALID;
@@ -305,7 +306,10 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.k = s->topk;
   p.max_seqlen = s->max_seqlen;
   p.nbmax = L.nbmax;
-  p.idx_wait = idx_from_prev ? 1 : 0;
+  // a staged cache is written by the preceding kernel (the gather): wait
+  // before any read, as for indices written just before
+  p.idx_wait = (idx_from_prev || staged) ? 1 : 0;
+  p.staged = staged ? 1 : 0;
   // CTAs launched early beside the preceding kernel stage their first blocks
   // before it ends; the last late_ctas of the grid find their SMs still held
   // and start after it: they take LATE_DEFICIT units fewer (bf16 streaming)
@@ -321,9 +325,10 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
 
   if (s->dtype == HYLRA_BF16) {
     if ((rc = prepare_bf16_kernels())) return rc;
-    const long long rows = s->kv_capacity > 0
-                               ? (long long)s->batch * s->num_kv_heads * s->kv_capacity
-                               : (long long)s->num_kv_heads * s->total_tokens;
+    const long long rows =
+        staged ? (long long)s->batch * s->num_kv_heads * s->topk * BLK
+               : (s->kv_capacity > 0 ? (long long)s->batch * s->num_kv_heads * s->kv_capacity
+                                     : (long long)s->num_kv_heads * s->total_tokens);
     CUtensorMap tmK, tmV;
     if ((rc = make_tmap(&tmK, K, rows))) return rc;
     if ((rc = make_tmap(&tmV, V, rows))) return rc;
@@ -391,6 +396,104 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
 
 size_t elem_size(const hylra_shape_t* s) { return s->dtype == HYLRA_BF16 ? 2 : 4; }
 
+size_t stage_bytes(const hylra_shape_t* s) {
+  return (size_t)s->batch * s->num_kv_heads * s->topk * BLK * HD * 2;
+}
+
+int check_stage_rows(const hylra_shape_t* s) {
+  const long long rows = (long long)s->batch * s->num_kv_heads * s->topk * BLK;
+  return rows > INT_MAX - 2 * HYLRA_BLOCK_TOKENS ? HYLRA_ERR_UNSUPPORTED : HYLRA_OK;
+}
+
+// Copy the listed blocks of a host-resident cache into a staging cache.
+int gather(const hylra_shape_t* s, const void* Kh, const void* Vh, const int32_t* seqlens,
+           const int32_t* topk_in, void* Ks, void* Vs, cudaStream_t stream, bool pdl) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (s->dtype != HYLRA_BF16) return HYLRA_ERR_UNSUPPORTED;
+  if ((rc = check_stage_rows(s))) return rc;
+  if (!Kh || !Vh || !seqlens || !topk_in || !Ks || !Vs) return HYLRA_ERR_INVALID;
+  if (!aligned(Kh, 16) || !aligned(Vh, 16) || !aligned(Ks, 16) || !aligned(Vs, 16) ||
+      !aligned(seqlens, 4) || !aligned(topk_in, 4))
+    return HYLRA_ERR_INVALID;
+  Params p{};
+  p.K = Kh;
+  p.V = Vh;
+  p.seqlens = seqlens;
+  p.seq_off = s->kv_capacity > 0 ? nullptr : s->seq_offsets;
+  p.topk_in = topk_in;
+  p.cap = s->kv_capacity;
+  p.total = s->kv_capacity > 0 ? 0 : s->total_tokens;
+  p.B = s->batch;
+  p.Hq = s->num_q_heads;
+  p.Hkv = s->num_kv_heads;
+  p.r = s->num_q_heads / s->num_kv_heads;
+  p.k = s->topk;
+  p.max_seqlen = s->max_seqlen;
+  // status bits of a bad length are left to the reuse kernel that follows
+  p.status = nullptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s->topk, s->batch * s->num_kv_heads);
+  cfg.blockDim = dim3(NT_GATHER);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, gather_blocks_kernel, p, static_cast<uint8_t*>(Ks),
+                         static_cast<uint8_t*>(Vs)) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
+}
+
+// One decode step; offloaded (may be NULL): per layer, 1 = K[l], V[l] are a
+// host-resident cache (reuse layers only), gathered into K_stage / V_stage.
+int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,
+             const void* const* q, const void* const* K, const void* const* V,
+             const uint8_t* offloaded, const int32_t* seqlens, float* const* out, int32_t* topk,
+             void* K_stage, void* V_stage, void* workspace, size_t workspace_bytes,
+             cudaStream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (num_layers < 1 || !policy || !q || !K || !V || !out || !topk) return HYLRA_ERR_INVALID;
+  if (policy[0] != 1) return HYLRA_ERR_INVALID;
+  for (int l = 0; l < num_layers; ++l) {
+    if (policy[l] > 1) return HYLRA_ERR_INVALID;
+    if (offloaded && offloaded[l] > 1) return HYLRA_ERR_INVALID;
+    // a reset layer reads every block: its cache must be on the device
+    if (offloaded && offloaded[l] && policy[l]) return HYLRA_ERR_INVALID;
+    if ((rc = check_layer_ptrs(shape, q[l], K[l], V[l], out[l]))) return rc;
+  }
+  const size_t per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
+  int last_reset = 0;
+  int prev_ctas = 0;  // CTAs of the kernel launched last (each holds an SM)
+  for (int l = 0; l < num_layers; ++l) {
+    if (policy[l]) {
+      last_reset = l;
+      rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
+                  workspace, workspace_bytes, stream, l > 0, true, l & 63, prev_ctas,
+                  &prev_ctas);
+    } else if (offloaded && offloaded[l]) {
+      // index-guided offloading: only the reused blocks cross the host link
+      const int32_t* idx = topk + last_reset * per_layer;
+      rc = gather(shape, K[l], V[l], seqlens, idx, K_stage, V_stage, stream, true);
+      if (!rc)
+        rc = launch(shape, false, q[l], K_stage, V_stage, seqlens, idx, out[l], nullptr,
+                    workspace, workspace_bytes, stream, true, true, l & 63, 0, &prev_ctas,
+                    true);
+    } else {
+      rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
+                  nullptr, workspace, workspace_bytes, stream, l > 0, last_reset == l - 1,
+                  l & 63, prev_ctas, &prev_ctas);
+    }
+    if (rc) return rc;
+  }
+  return HYLRA_OK;
+}
+
+
+
 }  // namespace
 
 extern "C" {
@@ -443,31 +546,47 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint
                       const void* const* q, const void* const* K, const void* const* V,
                       const int32_t* seqlens, float* const* out, int32_t* topk, void* workspace,
                       size_t workspace_bytes, hylra_stream_t stream) {
+  return run_step(shape, num_layers, policy, q, K, V, nullptr, seqlens, out, topk, nullptr,
+                  nullptr, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+int hylra_stage_bytes(const hylra_shape_t* shape, size_t* bytes) {
   int rc = check_shape(shape);
   if (rc) return rc;
-  if (num_layers < 1 || !policy || !q || !K || !V || !out || !topk) return HYLRA_ERR_INVALID;
-  if (policy[0] != 1) return HYLRA_ERR_INVALID;
-  for (int l = 0; l < num_layers; ++l) {
-    if (policy[l] > 1) return HYLRA_ERR_INVALID;
-    if ((rc = check_layer_ptrs(shape, q[l], K[l], V[l], out[l]))) return rc;
-  }
-  const size_t per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
-  int last_reset = 0;
-  int prev_ctas = 0;  // CTAs of the kernel launched last (each holds an SM)
-  for (int l = 0; l < num_layers; ++l) {
-    if (policy[l]) {
-      last_reset = l;
-      rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
-                  workspace, workspace_bytes, (cudaStream_t)stream, l > 0, true, l & 63,
-                  prev_ctas, &prev_ctas);
-    } else {
-      rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
-                  nullptr, workspace, workspace_bytes, (cudaStream_t)stream, l > 0,
-                  last_reset == l - 1, l & 63, prev_ctas, &prev_ctas);
-    }
-    if (rc) return rc;
-  }
+  if (!bytes) return HYLRA_ERR_INVALID;
+  if (shape->dtype != HYLRA_BF16) return HYLRA_ERR_UNSUPPORTED;
+  if ((rc = check_stage_rows(shape))) return rc;
+  *bytes = stage_bytes(shape);
   return HYLRA_OK;
+}
+
+int hylra_gather_blocks(const hylra_shape_t* shape, const void* K_host, const void* V_host,
+                        const int32_t* seqlens, const int32_t* topk_in, void* K_stage,
+                        void* V_stage, hylra_stream_t stream) {
+  return gather(shape, K_host, V_host, seqlens, topk_in, K_stage, V_stage, (cudaStream_t)stream,
+                false);
+}
+
+int hylra_decode_reuse_staged(const hylra_shape_t* shape, const void* q, const void* K_stage,
+                              const void* V_stage, const int32_t* seqlens,
+                              const int32_t* topk_in, float* out, void* workspace,
+                              size_t workspace_bytes, hylra_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if ((rc = check_stage_rows(shape))) return rc;
+  return launch(shape, false, q, K_stage, V_stage, seqlens, topk_in, out, nullptr, workspace,
+                workspace_bytes, (cudaStream_t)stream, false, true, 0, 0, nullptr, true);
+}
+
+int hylra_decode_step_offload(const hylra_shape_t* shape, int32_t num_layers,
+                              const uint8_t* policy, const void* const* q,
+                              const void* const* K, const void* const* V,
+                              const uint8_t* offloaded, const int32_t* seqlens,
+                              float* const* out, int32_t* topk, void* K_stage, void* V_stage,
+                              void* workspace, size_t workspace_bytes, hylra_stream_t stream) {
+  if (!offloaded || !K_stage || !V_stage) return HYLRA_ERR_INVALID;
+  return run_step(shape, num_layers, policy, q, K, V, offloaded, seqlens, out, topk, K_stage,
+                  V_stage, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,

@@ -121,6 +121,8 @@ struct Params {
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
   int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
+  int staged;        // reuse: K/V are a staging cache [B][Hkv][k][128][d] whose slot e holds
+                     // block topk_in[b][h][e] (written by gather_blocks_kernel)
   int late_from;     // bf16 streaming kernel: CTAs >= late_from start late (their SM is
   int late_deficit;  // still held by the preceding kernel) and take this many units fewer
   int q_wait;        // q and each sequence's newest K/V row come from the preceding kernel
@@ -130,7 +132,7 @@ struct Params {
 };
 
 struct StageMeta {
-  int b, h, blk, nvalid, flags, seg_slot, first_slot, ncontrib, nb, pad0, pad1, pad2;
+  int b, h, blk, nvalid, flags, seg_slot, first_slot, ncontrib, nb, pos, pad1, pad2;
 };
 constexpr int F_SEG_START = 1;
 constexpr int F_SEG_END = 2;
@@ -338,7 +340,8 @@ __device__ __forceinline__ StageMeta describe_unit(const Params& p, const SmemCo
   m.first_slot = cf + bh;
   m.ncontrib = cl - cf + 1;
   m.nb = nb;
-  m.pad0 = m.pad1 = m.pad2 = 0;
+  m.pos = it.j;  // place in the (b, h) index list (reuse) or block (reset)
+  m.pad1 = m.pad2 = 0;
   return m;
 }
 
@@ -1179,7 +1182,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       uint32_t bytesK = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? 2u * BOX_BYTES : 0u);
       uint32_t bytesV = m.blk >= 0 ? 2u * BOX_BYTES : 0u;
       if (*abort_flag) bytesK = bytesV = 0u;
-      const int row = (int)(row0 + (long long)m.h * hstride + (long long)m.blk * BLK);
+      const int row = p.staged ? (int)(((long long)(m.b * p.Hkv + m.h) * p.k + m.pos) * BLK)
+                               : (int)(row0 + (long long)m.h * hstride + (long long)m.blk * BLK);
       uint8_t* st = sm.stage[s];
       if (bytesK) {
         mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
@@ -1729,9 +1733,12 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
     const long long row0 = row_base(p, b, h);
     // blocks beyond the pipeline depth (and, with q_wait, the newest block)
     // into L2 now: lane i holds this CTA's i-th block
+    auto unit_row = [&](int i, int blk) -> int {
+      return p.staged ? (int)(((long long)bh * p.k + j0 + i) * BLK) : (int)(row0 + (long long)blk * BLK);
+    };
     if (lane < nu && my_blk >= 0 && my_blk < nb &&
         (lane >= nst || (p.q_wait && !waited && my_blk == nb - 1))) {
-      const int row = (int)(row0 + (long long)my_blk * BLK);
+      const int row = unit_row(lane, my_blk);
       tma_prefetch_l2_2d(&tmK, 0, row);
       tma_prefetch_l2_2d(&tmK, 64, row);
       tma_prefetch_l2_2d(&tmV, 0, row);
@@ -1763,7 +1770,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
       if (*abort_flag) bytesK = bytesV = 0u;
       uint8_t* st = stages + (size_t)s * STAGE_BYTES;
-      const int row = (int)(row0 + (long long)blk * BLK);
+      const int row = unit_row(i, blk);
       if (bytesK) {
         mbar_arrive_expect_tx(&sm.fullK_bar[s], bytesK);
         if (i == 0) {
@@ -1881,6 +1888,57 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
     HYLRA_TRACE_VAL(tn, tcta, 42 << 8, HYLRA_CLOCK());
   }
   if (*abort_flag && tid == 32) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------ block gather
+//
+// Index-guided offloading (HyLRA summary §2.4): a reuse layer whose cache is
+// in host memory needs only the blocks its index list names.  CTA (e, bh)
+// copies block topk_in[b][h][e] of K and of V (the valid rows of it) from
+// the host-resident cache (p.K, p.V: pinned host memory, read by the device
+// across the host link) into slot e of the device staging cache
+// [B][Hkv][k][128][d] (Ks, Vs).  Every thread keeps its loads in flight
+// before storing, so the link sees many outstanding requests.
+constexpr int NT_GATHER = 256;
+
+__global__ void __launch_bounds__(NT_GATHER) gather_blocks_kernel(const __grid_constant__ Params p,
+                                                                 uint8_t* Ks, uint8_t* Vs) {
+  const int e = (int)blockIdx.x, bh = (int)blockIdx.y;
+  const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+  const int seqlen = valid_seqlen(p, b, false);
+  const int nb = (seqlen + BLK - 1) / BLK;
+  griddep_wait();  // the index list and the cache rows come from earlier work
+  griddep_launch_dependents();
+  if (e >= min(p.k, nb)) return;
+  const int blk = __ldcg(p.topk_in + (size_t)bh * p.k + e);
+  if (blk < 0 || blk >= nb) return;  // flagged by the reuse kernel
+  const int rows = min(BLK, seqlen - blk * BLK);
+  const long long src_row = row_base(p, b, h) + (long long)blk * BLK;
+  const long long dst_row = ((long long)bh * p.k + e) * BLK;
+  constexpr int CH = HD * 2 / 16;        // 16-byte chunks per row
+  constexpr int PER = BLK * CH / NT_GATHER;  // chunks per thread and tensor
+  const uint4* sk = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.K) + src_row * HD * 2);
+  const uint4* sv = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.V) + src_row * HD * 2);
+  uint4* dk = reinterpret_cast<uint4*>(Ks + dst_row * HD * 2);
+  uint4* dv = reinterpret_cast<uint4*>(Vs + dst_row * HD * 2);
+  uint4 vk[PER], vv[PER];
+  const int nch = rows * CH;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int c = u * NT_GATHER + (int)threadIdx.x;
+    if (c < nch) {
+      vk[u] = sk[c];
+      vv[u] = sv[c];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int c = u * NT_GATHER + (int)threadIdx.x;
+    if (c < nch) {
+      dk[c] = vk[u];
+      dv[c] = vv[u];
+    }
+  }
 }
 
 // ------------------------------------------------------------ fp32 kernel

@@ -40,7 +40,9 @@ ERRORS = {0: "HYLRA_OK", -1: "HYLRA_ERR_INVALID", -2: "HYLRA_ERR_UNSUPPORTED",
 EXPORTS = ("hylra_workspace_bytes", "hylra_workspace_init", "hylra_decode_full",
            "hylra_decode_reuse", "hylra_decode_step", "hylra_decode_step_host",
            "hylra_similarity", "hylra_dp_policy", "hylra_read_status", "hylra_strerror",
-           "hylra_version", "hylra_decode_full_noalloc", "hylra_static_policy")
+           "hylra_version", "hylra_decode_full_noalloc", "hylra_static_policy",
+           "hylra_stage_bytes", "hylra_gather_blocks", "hylra_decode_reuse_staged",
+           "hylra_decode_step_offload")
 
 
 class HylraError(RuntimeError):
@@ -96,6 +98,10 @@ def load() -> ctypes.CDLL:
         "hylra_read_status": [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P],
         "hylra_decode_full_noalloc": [SP, P, P, P, P, P, P, P, P],
         "hylra_static_policy": [I32, I32, P, ctypes.POINTER(I32)],
+        "hylra_stage_bytes": [SP, ctypes.POINTER(ctypes.c_size_t)],
+        "hylra_gather_blocks": [SP, P, P, P, P, P, P, P],
+        "hylra_decode_reuse_staged": [SP, P, P, P, P, P, P, P, S, P],
+        "hylra_decode_step_offload": [SP, I32, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "hylra_strerror": [ctypes.c_int],
         "hylra_version": [],
     }
@@ -233,3 +239,38 @@ def static_policy(num_layers: int, period: int):
     _check(load().hylra_static_policy(int(num_layers), int(period), pol.ctypes.data,
                                       ctypes.byref(R)), "hylra_static_policy")
     return tuple(int(x) for x in pol), R.value
+
+
+def stage_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().hylra_stage_bytes(ctypes.byref(shape), ctypes.byref(n)), "hylra_stage_bytes")
+    return n.value
+
+
+def gather_blocks(shape: Shape, K_host, V_host, seqlens, topk_in, K_stage, V_stage, stream=None):
+    """K_host / V_host: pinned torch CPU tensors (the device reads them in place)."""
+    _check(load().hylra_gather_blocks(ctypes.byref(shape), _ptr(K_host), _ptr(V_host),
+                                      _ptr(seqlens), _ptr(topk_in), _ptr(K_stage), _ptr(V_stage),
+                                      _stream(stream)), "hylra_gather_blocks")
+
+
+def decode_reuse_staged(shape: Shape, q, K_stage, V_stage, seqlens, topk_in, out, ws,
+                        stream=None):
+    _check(load().hylra_decode_reuse_staged(ctypes.byref(shape), _ptr(q), _ptr(K_stage),
+                                            _ptr(V_stage), _ptr(seqlens), _ptr(topk_in),
+                                            _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)), "hylra_decode_reuse_staged")
+
+
+def decode_step_offload(shape: Shape, policy: Sequence[int], qs, Ks, Vs, offloaded, seqlens,
+                        outs, topk, K_stage, V_stage, ws, stream=None):
+    """Ks[l] / Vs[l] of layers with offloaded[l] = 1 are pinned torch CPU tensors."""
+    L = len(policy)
+    pol = (ctypes.c_uint8 * L)(*[int(x) for x in policy])
+    off = (ctypes.c_uint8 * L)(*[int(x) for x in offloaded])
+    _check(load().hylra_decode_step_offload(ctypes.byref(shape), L, pol, _ptr_array(qs),
+                                            _ptr_array(Ks), _ptr_array(Vs), off, _ptr(seqlens),
+                                            _ptr_array(outs), _ptr(topk), _ptr(K_stage),
+                                            _ptr(V_stage), _ptr(ws),
+                                            ws.numel() * ws.element_size(), _stream(stream)),
+           "hylra_decode_step_offload")
