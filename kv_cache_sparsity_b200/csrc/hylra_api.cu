@@ -433,7 +433,7 @@ int gather(const hylra_shape_t* s, const void* Kh, const void* Vh, const int32_t
   // status bits of a bad length are left to the reuse kernel that follows
   p.status = nullptr;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s->topk, s->batch * s->num_kv_heads);
+  cfg.gridDim = dim3(s->batch * s->num_kv_heads, s->topk);
   cfg.blockDim = dim3(NT_GATHER);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

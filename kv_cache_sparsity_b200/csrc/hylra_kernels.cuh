@@ -1893,7 +1893,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
 // ------------------------------------------------------------ block gather
 //
 // Index-guided offloading (HyLRA summary §2.4): a reuse layer whose cache is
-// in host memory needs only the blocks its index list names.  CTA (e, bh)
+// in host memory needs only the blocks its index list names.  CTA (bh, e)
 // copies block topk_in[b][h][e] of K and of V (the valid rows of it) from
 // the host-resident cache (p.K, p.V: pinned host memory, read by the device
 // across the host link) into slot e of the device staging cache
@@ -1903,7 +1903,7 @@ constexpr int NT_GATHER = 256;
 
 __global__ void __launch_bounds__(NT_GATHER) gather_blocks_kernel(const __grid_constant__ Params p,
                                                                  uint8_t* Ks, uint8_t* Vs) {
-  const int e = (int)blockIdx.x, bh = (int)blockIdx.y;
+  const int bh = (int)blockIdx.x, e = (int)blockIdx.y;  // B*Hkv may exceed a y extent
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int seqlen = valid_seqlen(p, b, false);
   const int nb = (seqlen + BLK - 1) / BLK;

@@ -129,3 +129,31 @@ def test_offloaded_reset_layer_is_rejected():
                               [l[2] for l in layers], (1, 0), run.seqlens, outs, topk, Ks, Vs,
                               run.ws)
     assert e.value.code == -1
+
+
+def test_reuse_beyond_the_cluster_grid_limit():
+    """B * Hkv = 65,536 (one more than a grid's y extent): reuse layers take
+    the streaming kernel + merge kernel path, plain and staged."""
+    w = W.custom("wide", batch=1024, layers=2, seqlens=(256,) * 1024, num_q_heads=64,
+                 num_kv_heads=64, topk=2, seed=47)
+    run = T.Runner(w)
+    q0, K0, V0 = W.layer_inputs(w, 0, "cuda")
+    _, tk = run.full(q0, K0, V0)
+    assert run.status() == 0
+    del K0, V0
+    q1, K1, V1 = W.layer_inputs(w, 1, "cuda")
+    out = run.reuse(q1, K1, V1, tk)
+    assert run.status() == 0
+    tkn = tk.cpu().numpy()
+    for b in (0, 517, 1023):
+        o_ref = T.oracle_reuse(w, q1, K1, V1, b, tkn[b])
+        T.check_out(out[b].cpu().numpy(), o_ref, "bf16", f"wide reuse b={b}")
+    Kh, Vh = _pinned(K1), _pinned(V1)
+    del K1, V1
+    torch.cuda.empty_cache()
+    Ks, Vs = _stage(run)
+    H.gather_blocks(run.shape, Kh, Vh, run.seqlens, tk, Ks, Vs)
+    out_s = run.new_out()
+    H.decode_reuse_staged(run.shape, q1, Ks, Vs, run.seqlens, tk, out_s, run.ws)
+    assert run.status() == 0
+    assert torch.equal(out_s, out)
