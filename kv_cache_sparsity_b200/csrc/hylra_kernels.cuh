@@ -993,6 +993,114 @@ struct WarpAttn {
     }
   }
 
+  // Zero the V rows of a partial block past the sequence end (they may hold
+  // anything, even NaN) before the PV step reads them.
+  __device__ __forceinline__ void zero_tail_v(uint8_t* stage, int nvalid) {
+    for (int idx = lane; idx < 16 * 16; idx += 32) {
+      const int row = tokw + (idx >> 4);
+      if (row < nvalid) continue;
+      const int ch = idx & 15;
+      uint8_t* ptr = stage + 2 * BOX_BYTES + (ch >> 3) * BOX_BYTES + row * 128 + (ch & 7) * 16;
+      *reinterpret_cast<uint4*>(ptr) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+  }
+
+  // Two staged blocks as one 256-token step (reuse layers): the two QK
+  // chains, one softmax update and the two PV chains interleave, so the
+  // pair costs little more than one block.
+  __device__ __forceinline__ void block2(uint8_t* st0, int nv0, uint64_t* fullV0, uint32_t ph0,
+                                         uint8_t* st1, int nv1, uint64_t* fullV1, uint32_t ph1,
+                                         float scale_log2, volatile int* abort_flag) {
+    float x0[4], x1[4];
+    {
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      float b0[4] = {0.f, 0.f, 0.f, 0.f}, b1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t kb0 = smem_u32(st0) + krow * 128, kb1 = smem_u32(st1) + krow * 128;
+#pragma unroll
+      for (int kt = 0; kt < 8; ++kt) {
+        const int ch = 2 * kt + kchi;
+        const uint32_t off = (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+        uint32_t r0, r1, r2, r3, t0, t1, t2, t3;
+        ldsm_x4(kb0 + off, r0, r1, r2, r3);
+        ldsm_x4(kb1 + off, t0, t1, t2, t3);
+        mma_bf16_16816((kt & 1) ? a1 : a0, r0, r1, r2, r3, qf[kt][0], qf[kt][1]);
+        mma_bf16_16816((kt & 1) ? b1 : b0, t0, t1, t2, t3, qf[kt][0], qf[kt][1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = tokw + g4 + ((e & 2) ? 8 : 0);
+        x0[e] = tok < nv0 ? (a0[e] + a1[e]) * scale_log2 : -INFINITY;
+        x1[e] = tok < nv1 ? (b0[e] + b1[e]) * scale_log2 : -INFINITY;
+      }
+    }
+    mbar_wait_bounded(fullV0, ph0, abort_flag);
+    mbar_wait_bounded(fullV1, ph1, abort_flag);
+    if (nv0 < BLK) zero_tail_v(st0, nv0);
+    if (nv1 < BLK) zero_tail_v(st1, nv1);
+    // max and sums over the pair's tokens for heads A and B
+    float mxA = fmaxf(fmaxf(x0[0], x0[2]), fmaxf(x1[0], x1[2]));
+    float mxB = fmaxf(fmaxf(x0[1], x0[3]), fmaxf(x1[1], x1[3]));
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, off));
+      mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, off));
+    }
+    const float msA = mxA == -INFINITY ? 0.f : mxA;
+    const float msB = mxB == -INFINITY ? 0.f : mxB;
+    const float p00 = ex2_approx(x0[0] - msA), p01 = ex2_approx(x0[1] - msB);
+    const float p02 = ex2_approx(x0[2] - msA), p03 = ex2_approx(x0[3] - msB);
+    const float p10 = ex2_approx(x1[0] - msA), p11 = ex2_approx(x1[1] - msB);
+    const float p12 = ex2_approx(x1[2] - msA), p13 = ex2_approx(x1[3] - msB);
+    float sA = (p00 + p02) + (p10 + p12);
+    float sB = (p01 + p03) + (p11 + p13);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      sA += __shfl_xor_sync(0xffffffffu, sA, off);
+      sB += __shfl_xor_sync(0xffffffffu, sB, off);
+    }
+    const float mnA = fmaxf(m_run[0], mxA), mnB = fmaxf(m_run[1], mxB);
+    float alA = 1.f, beA = 0.f, alB = 1.f, beB = 0.f;
+    if (mnA != -INFINITY) {
+      alA = ex2_approx(m_run[0] - mnA);
+      beA = ex2_approx(mxA - mnA);
+    }
+    if (mnB != -INFINITY) {
+      alB = ex2_approx(m_run[1] - mnB);
+      beB = ex2_approx(mxB - mnB);
+    }
+    z_run[0] = z_run[0] * alA + sA * beA;
+    z_run[1] = z_run[1] * alB + sB * beB;
+    m_run[0] = mnA;
+    m_run[1] = mnB;
+    if (__any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
+#pragma unroll
+      for (int dm = 0; dm < 8; ++dm) {
+        o[dm][0] *= alA;
+        o[dm][1] *= alB;
+        o[dm][2] *= alA;
+        o[dm][3] *= alB;
+      }
+    }
+    const uint32_t q00 = movmatrix_trans(pack_bf16x2(p00 * beA, p01 * beB));
+    const uint32_t q01 = movmatrix_trans(pack_bf16x2(p02 * beA, p03 * beB));
+    const uint32_t q10 = movmatrix_trans(pack_bf16x2(p10 * beA, p11 * beB));
+    const uint32_t q11 = movmatrix_trans(pack_bf16x2(p12 * beA, p13 * beB));
+    const uint32_t vb0 = smem_u32(st0) + 2 * BOX_BYTES + vrow * 128;
+    const uint32_t vb1 = smem_u32(st1) + 2 * BOX_BYTES + vrow * 128;
+#pragma unroll
+    for (int dm = 0; dm < 8; ++dm) {
+      const int ch = 2 * dm + vchi;
+      const uint32_t off = (ch >> 3) * BOX_BYTES + (((ch & 7) ^ xr) << 4);
+      uint32_t r0, r1, r2, r3, t0, t1, t2, t3;
+      ldsm_x4_trans(vb0 + off, r0, r1, r2, r3);
+      ldsm_x4_trans(vb1 + off, t0, t1, t2, t3);
+      mma_bf16_16816(o[dm], r0, r1, r2, r3, q00, q01);
+      mma_bf16_16816(o[dm], t0, t1, t2, t3, q10, q11);
+    }
+  }
+
   // This warp's state as is: O^T columns into so[head][dim], running max
   // and sum into sm_[head], sz_[head].
   __device__ __forceinline__ void store_state(float (*so)[HD], float* sm_, float* sz_) const {
@@ -1636,7 +1744,7 @@ __device__ __forceinline__ float2 rc_merge_pair(const float* gather, int slot, i
   return Z > 0.f ? make_float2(a0 / Z, a1 / Z) : make_float2(0.f, 0.f);
 }
 
-__global__ void __launch_bounds__(NTHR_BF16, 2)
+__global__ void __launch_bounds__(NTHR_BF16, 1)
     decode_reuse_cluster_kernel(const __grid_constant__ CUtensorMap tmK,
                                 const __grid_constant__ CUtensorMap tmV,
                                 const __grid_constant__ Params p) {
@@ -1817,7 +1925,25 @@ __global__ void __launch_bounds__(NTHR_BF16, 2)
       wa.block(stages, BLK, p.scale_log2, &sm.fullV_bar[0], 0u, abort_flag, d0, d1, d2, d3);
       wa.reset();
     }
-    for (int i = 0; i < nu; ++i) {
+    // blocks in pairs while two stages hold them (one 256-token step each)
+    int i = 0;
+    for (; nst >= 2 && i + 1 < nu; i += 2) {
+      const int s0 = i % nst, s1 = (i + 1) % nst;
+      const uint32_t ph0 = (uint32_t)((i / nst) & 1), ph1 = (uint32_t)(((i + 1) / nst) & 1);
+      mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag);
+      mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag);
+      if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
+      if (i == 0) wa.load_q(sm.qbuf, r);
+      wa.block2(stages + (size_t)s0 * STAGE_BYTES, sm.meta_nvalid[s0], &sm.fullV_bar[s0], ph0,
+                stages + (size_t)s1 * STAGE_BYTES, sm.meta_nvalid[s1], &sm.fullV_bar[s1], ph1,
+                p.scale_log2, abort_flag);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sm.empty_bar[s0]);
+        mbar_arrive(&sm.empty_bar[s1]);
+      }
+    }
+    for (; i < nu; ++i) {
       const int s = i % nst;
       const uint32_t ph = (uint32_t)((i / nst) & 1);
       mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
