@@ -536,7 +536,8 @@ def run_ours(args, rank, world, dist_on):
 # ----------------------------------------------------------- reference arm
 
 def run_reference(args):
-    """The fp64 oracle, as it stands, on the host cores (no GPU needed)."""
+    """The fp64 oracle, as it stands, on the host cores (no GPU needed; with
+    one, only to draw the same inputs as our arm)."""
     from oracle import hylra_oracle as O
     w = W.config(args.config)
     heads = (0,)  # bounded sample: one KV head of every sequence, scaled to all heads
@@ -546,11 +547,17 @@ def run_reference(args):
 
     m = _M()
     m.q, m.Ks, m.Vs = [], [], []
+    # the same values as our arm: torch's generator differs between CPU and
+    # GPU, so the inputs are drawn on the GPU when there is one (and only
+    # then copied to the host, where all the timed work runs)
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
     for l in range(w.layers):
-        q, K, V = W.layer_inputs(w, l, device="cpu")
+        q, K, V = (t.cpu() for t in W.layer_inputs(w, l, device=gen))
         m.q.append(q)
         m.Ks.append(K)
         m.Vs.append(V)
+    if gen == "cuda":
+        torch.cuda.empty_cache()
     # policy: the oracle's own profiling + DP on this sample (every layer full)
     if args.policy == "jump3":
         policy, _ = O.static_policy(w.layers, 3)
@@ -561,7 +568,7 @@ def run_reference(args):
         for l in range(w.layers):
             per = []
             for p in range(max(1, args.profile_steps)):
-                ql = m.q[l] if p == 0 else W.step_query(w, l, p, device="cpu")
+                ql = m.q[l] if p == 0 else W.step_query(w, l, p, device=gen).cpu()
                 for b in range(w.batch):
                     kb = W.per_sequence(w, m.Ks[l], b).double().numpy()
                     vb = W.per_sequence(w, m.Vs[l], b).double().numpy()
