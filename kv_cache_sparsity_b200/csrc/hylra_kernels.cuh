@@ -1925,9 +1925,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       wa.block(stages, BLK, p.scale_log2, &sm.fullV_bar[0], 0u, abort_flag, d0, d1, d2, d3);
       wa.reset();
     }
-    // blocks in pairs while two stages hold them (one 256-token step each)
+    // blocks in pairs (one 256-token step each) when every block has its own
+    // stage; with refills, one at a time so each freed stage reloads early
     int i = 0;
-    for (; nst >= 2 && i + 1 < nu; i += 2) {
+    for (; nu <= nst && i + 1 < nu; i += 2) {
       const int s0 = i % nst, s1 = (i + 1) % nst;
       const uint32_t ph0 = (uint32_t)((i / nst) & 1), ph1 = (uint32_t)(((i + 1) / nst) & 1);
       mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag);
