@@ -1844,8 +1844,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     auto unit_row = [&](int i, int blk) -> int {
       return p.staged ? (int)(((long long)bh * p.k + j0 + i) * BLK) : (int)(row0 + (long long)blk * BLK);
     };
-    if (lane < nu && my_blk >= 0 && my_blk < nb &&
-        (lane >= nst || (p.q_wait && !waited && my_blk == nb - 1))) {
+    if (lane < nu && my_blk >= 0 && my_blk < nb && lane >= nst) {
       const int row = unit_row(lane, my_blk);
       tma_prefetch_l2_2d(&tmK, 0, row);
       tma_prefetch_l2_2d(&tmK, 64, row);
@@ -1863,9 +1862,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         if (blk != -1) atomicOr(p.status, HYLRA_STATUS_BAD_INDEX);
         blk = -1;
       }
-      // a stage is refilled only after the consumers used it, which needs
-      // q; the block holding the newest token is read after the wait too
-      if (p.q_wait && !waited && (i >= nst || blk == nb - 1)) {
+      // a stage is refilled only after the consumers used it, which needs q
+      // (the block holding the newest token is staged early like the rest:
+      // its consumer warp rewrites the newest row after the wait)
+      if (p.q_wait && !waited && i >= nst) {
         griddep_wait();
         waited = true;
         if (qpend && !*abort_flag) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
@@ -1917,6 +1917,27 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (!p.idx_wait) griddep_launch_dependents();
     WarpAttn wa;
     wa.init(cw, lane);
+    // With q_wait the newest row of the sequence (written by the preceding
+    // kernel in a model) is re-read after the wait by the one warp whose 16
+    // rows hold it (each warp reads only its own rows of a stage): one
+    // 16-byte chunk of K or V per lane, into its swizzled place.
+    const long long row0c = (p.q_wait && !p.staged) ? row_base(p, b, h) : 0;
+    auto patch_newest = [&](int s, uint32_t ph) {
+      const int blk = sm.meta_blk[s];
+      if (!p.q_wait || p.staged || blk < 0 || blk != nb - 1) return;
+      const int rr = sm.meta_nvalid[s] - 1;  // the newest row within the block
+      if ((rr >> 4) != cw) return;
+      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);  // V landed (K: fullK)
+      griddep_wait();
+      const int c = lane & 15;
+      const long long grow = row0c + (long long)blk * BLK + rr;
+      const uint8_t* src =
+          static_cast<const uint8_t*>(lane < 16 ? p.K : p.V) + grow * (HD * 2) + c * 16;
+      uint8_t* dst = stages + (size_t)s * STAGE_BYTES + (lane < 16 ? 0 : 2 * BOX_BYTES) +
+                     (c >> 3) * BOX_BYTES + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
+      if (!*abort_flag) *reinterpret_cast<uint4*>(dst) = __ldcg(reinterpret_cast<const uint4*>(src));
+      __syncwarp();
+    };
     if (p.q_wait && !p.idx_wait && nu > 0) {
       // while q is on its way: one pass over the first staged block with a
       // zero query, result discarded (brings the code into the instruction
@@ -1935,6 +1956,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
+      patch_newest(s0, ph0);
+      patch_newest(s1, ph1);
       wa.block2(stages + (size_t)s0 * STAGE_BYTES, sm.meta_nvalid[s0], &sm.fullV_bar[s0], ph0,
                 stages + (size_t)s1 * STAGE_BYTES, sm.meta_nvalid[s1], &sm.fullV_bar[s1], ph1,
                 p.scale_log2, abort_flag);
@@ -1950,6 +1973,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
+      patch_newest(s, ph);
       const int blk = sm.meta_blk[s];
       if (blk >= 0) {
         float mxA, mxB, sA, sB;
