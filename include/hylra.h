@@ -12,10 +12,17 @@
  *        the KV cache.                     -> hylra_decode_full, hylra_decode_reuse,
  *                                             hylra_decode_step
  *   §2.4 Block-level Sparsity: selection works on fixed 128-token blocks.
+ *   §2.4 Index-Guided Offloading: a cache in host memory sends only the
+ *        reused blocks across the host link.
+ *                                          -> hylra_gather_blocks,
+ *                                             hylra_decode_reuse_staged,
+ *                                             hylra_decode_step_offload
  *   §2.2 Offline policy: a lower-triangular overlap matrix M of top-k indices
  *        between source and target layers, and a dynamic program over states
  *        (i, j) with reset jumps and vertical moves gated by theta.
  *                                          -> hylra_similarity, hylra_dp_policy
+ *   §4   The Jump3 baseline (a reset every third layer).
+ *                                          -> hylra_static_policy
  *
  * Conventions shared by every entry point
  * ---------------------------------------
