@@ -200,7 +200,7 @@ int rc_max_active(const RCPlan& pl) {
   return v;
 }
 
-#ifdef HYLRA_TRACE
+#if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
 int g_plan_cs = 0, g_plan_nst = 0;  // tuning builds: force a plan
 int g_late_deficit = -1;            // tuning builds: force the late-start deficit
 #endif
@@ -222,7 +222,7 @@ bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
-#ifdef HYLRA_TRACE
+#if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
   if (g_plan_cs > 0) {
     const RCPlan pl = rc_plan_for(std::min(g_plan_cs, kmax), kmax, r, g_plan_nst);
     if (pl.nst < 1 || rc_max_active(pl) < 1) return false;
@@ -315,7 +315,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   // and start after it: they take LATE_DEFICIT units fewer (bf16 streaming)
   p.late_from = G - std::min(G, std::max(0, late_ctas));
   p.late_deficit = pdl && late_ctas > 0 ? LATE_DEFICIT : 0;
-#ifdef HYLRA_TRACE
+#if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
   if (g_late_deficit >= 0 && p.late_deficit > 0) p.late_deficit = g_late_deficit;
 #endif
   if (last_ctas) *last_ctas = 0;
@@ -624,8 +624,8 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
   return HYLRA_OK;
 }
 
-#ifdef HYLRA_TRACE
-// Trace builds only: force the reuse cluster plan (cs = 0: automatic).
+#if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
+// Tuning and trace builds only: force the reuse cluster plan (cs = 0: automatic).
 int hylra_plan_override(int cs, int nst) {
   g_plan_cs = cs;
   g_plan_nst = nst;
@@ -636,7 +636,9 @@ int hylra_late_override(int d) {
   g_late_deficit = d;
   return HYLRA_OK;
 }
+#endif
 
+#ifdef HYLRA_TRACE
 // Trace builds only: device buffer of TRACE_PER_CTA uint64 per CTA (or NULL).
 int hylra_trace_set(void* buf) {
   unsigned long long* p = static_cast<unsigned long long*>(buf);

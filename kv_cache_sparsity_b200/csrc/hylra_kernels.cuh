@@ -116,7 +116,7 @@ struct Params {
   uint32_t* status;
   uint32_t* tickets;
   float* partials;
-  float* bstat;
+  float* bstat;     // block records, float2 [B*Hkv][r][nbmax] (bstat_at)
   long long cap;    // dense rows per (b, h) plane; 0 = packed layout
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
@@ -251,6 +251,13 @@ __device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
   return (int)(((u + 1) * G - 1) / T);
 }
 
+// Block records (max, probability sum) of reset layers: float2 at
+// [b * Hkv + h][g][block], head-major so that consecutive blocks of one head
+// are adjacent (the merge reads them one block per lane).
+__device__ __forceinline__ size_t bstat_at(const Params& p, int bh, int g, int beta) {
+  return (((size_t)bh * p.r + g) * p.nbmax + beta) * 2;
+}
+
 // prefix[b] = number of units of sequences 0..b-1 (all KV heads); warp 0.
 __device__ void build_prefix(const Params& p, SmemCommon& c, bool full) {
   if (threadIdx.x >= 32) return;
@@ -358,21 +365,130 @@ __device__ __forceinline__ int unit_index_entry(const Params& p, const UnitIter&
 //
 // A key "beats" another when it is larger, or equal with a lower index; the
 // answer is the kp keys beaten by fewer than kp others.  Up to NT keys and
-// kp <= 32: per-warp sorted lists (below).  Otherwise, fast path (kp <= 32):
-// each warp sorts its 32 per-thread maxima (bitonic network over shuffles);
-// its kp-th largest is a value that kp of its keys reach, so tau0, the
-// largest of these over the warps, bounds the kp-th largest key from below.
-// Keys above tau0 are candidates, ranked by pairwise comparison; keys equal
-// to tau0 fill the remaining ranks in block order.  When there are many
-// candidates (few top blocks per warp), or kp > 32, a radix select runs.
-constexpr int TOPK_LIST_CAP = (NCOMB * GMAX * HD * 4 - MAX_NB * 4) / 8 - 128;
+// kp <= 32: per-warp sorted lists ranked by counting (below).  Other cases
+// with kp <= 32: a merge tree of per-warp sorted lists (topk_tree).  Larger
+// kp: a radix select on the keys' bit patterns.
+
+// Warp-level compare-exchange networks on 64-bit values, descending.  A
+// warp holds 32 * N values, element e = lane * N + i in register i: pairs at
+// distance j < N are in one lane's registers, the others one shuffle apart.
+template <int N>
+__device__ __forceinline__ void cx_desc(uint64_t (&v)[N], int lane, int j, int k) {
+  if (j < N) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if (i & j) continue;
+      // (lane, i) is the lower element of its pair; its run of k elements
+      // is sorted descending when bit k of its index is clear
+      const bool desc = ((lane * N + i) & k) == 0;
+      const uint64_t a = v[i], b = v[i | j];
+      const bool swap = desc ? (a < b) : (a > b);
+      v[i] = swap ? b : a;
+      v[i | j] = swap ? a : b;
+    }
+  } else {
+    const int lj = j / N;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, v[i], lj);
+      const bool desc = ((lane * N + i) & k) == 0;
+      const bool lower = (lane & lj) == 0;
+      v[i] = (lower == desc) ? (v[i] > o ? v[i] : o) : (v[i] < o ? v[i] : o);
+    }
+  }
+}
+
+// Sorts a bitonic sequence of 32 * N values descending (one merge pass).
+template <int N>
+__device__ __forceinline__ void warp_bitonic_merge_desc(uint64_t (&v)[N], int lane) {
+#pragma unroll
+  for (int j = 16 * N; j > 0; j >>= 1) cx_desc<N>(v, lane, j, 64 * N);  // bit 64N: never set
+}
+
+// Top-k' for k' <= LIST = 32 * LPL, without data-dependent work.  (key,
+// block) pairs compare as distinct 64-bit composites (score descending, block
+// ascending).  Two facts do all the work: for A and B sorted descending,
+// max(A[e], B[LIST-1-e]) is bitonic and holds the LIST largest of A and B
+// (so one merge pass sorts them), and the largest of a union are the
+// largest of the parts' largest.  Each warp keeps a sorted list of its
+// LIST largest so far; per round of 32 keys (one per lane) it sorts them
+// and merges them in.  Then the warps' lists merge pairwise in a tree.
+// The networks run inside loops, not unrolled, so the code that runs once
+// per launch stays small (it is fetched cold).
+template <int NT, int LPL, int BAR>
+__device__ void topk_tree(const uint32_t* keys, uint32_t* scratch, int32_t* dst, int nb, int kp,
+                          int k, int ct) {
+  constexpr int NW = NT / 32, LIST = 32 * LPL;
+  static_assert((NW & (NW - 1)) == 0, "power-of-two warps");
+  static_assert((MAX_NB + 256) * 4 + NW * LIST * 8 <= NCOMB * GMAX * HD * 4,
+                "keys, maxima and lists share the combine area");
+  uint64_t* lists = reinterpret_cast<uint64_t*>(scratch + 256);  // [NW][LIST]
+  const int lane = ct & 31, wid = ct >> 5;
+  for (int slot = kp + ct; slot < k; slot += NT) dst[slot] = -1;
+  uint64_t L[LPL];
+#pragma unroll
+  for (int i = 0; i < LPL; ++i) L[i] = 0ull;
+#pragma unroll 1
+  for (int base = wid * 32; base < nb; base += NT) {
+    const int beta = base + lane;
+    uint64_t x[1] = {beta < nb ? ((uint64_t)keys[beta] << 32) | (uint32_t)~(uint32_t)beta : 0ull};
+    // nothing to do when no key beats the list's last entry
+    const uint64_t last = __shfl_sync(0xffffffffu, L[LPL - 1], 31);
+    if (!__any_sync(0xffffffffu, x[0] > last)) continue;
+#pragma unroll
+    for (int kk = 2; kk <= 32; kk <<= 1)
+#pragma unroll
+      for (int j = kk >> 1; j > 0; j >>= 1) cx_desc<1>(x, lane, j, kk);
+    // the 32 sorted keys, padded with zeros to LIST, reversed against L
+#pragma unroll
+    for (int i = 0; i < LPL; ++i) {
+      const int f = LIST - 1 - (lane * LPL + i);
+      const uint64_t xf = __shfl_sync(0xffffffffu, x[0], f & 31);
+      const uint64_t b = f < 32 ? xf : 0ull;
+      L[i] = L[i] > b ? L[i] : b;
+    }
+    warp_bitonic_merge_desc<LPL>(L, lane);
+  }
+#pragma unroll
+  for (int i = 0; i < LPL; ++i) lists[wid * LIST + lane * LPL + i] = L[i];
+  named_bar_sync(BAR, NT);
+  // Every warp takes every level's barrier (the same barrier at the same
+  // count as the caller's, which the early warps may reach next).
+#pragma unroll 1
+  for (int span = 1; span < NW; span <<= 1) {
+    const int nm = NW / (2 * span);  // merging warps at this level
+    if (wid < nm) {
+      const uint64_t* A = lists + (2 * span * wid) * LIST;
+      const uint64_t* B = A + span * LIST;
+#pragma unroll
+      for (int i = 0; i < LPL; ++i) {
+        const int e = lane * LPL + i;
+        const uint64_t a = A[e], b = B[LIST - 1 - e];
+        L[i] = a > b ? a : b;
+      }
+      warp_bitonic_merge_desc<LPL>(L, lane);
+      if (nm > 1) {
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < LPL; ++i) lists[(2 * span * wid) * LIST + lane * LPL + i] = L[i];
+      }
+    }
+    if (nm > 1) named_bar_sync(BAR, NT);
+  }
+  if (wid != 0) return;
+  // warp 0 holds the answer (with one warp, its own list)
+#pragma unroll
+  for (int i = 0; i < LPL; ++i) {
+    const int e = lane * LPL + i;
+    if (e < kp) dst[e] = (int32_t)~(uint32_t)(L[i] & 0xffffffffull);
+  }
+}
 
 template <int NT, int BAR = BAR_CONS>
 __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int ct) {
   constexpr int NW = NT / 32;
   uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
-  uint32_t* tmax = keys + MAX_NB;                       // NT per-thread maxima
-  uint2* list = reinterpret_cast<uint2*>(tmax + 256);  // candidates (key, block)
+  uint32_t* tmax = keys + MAX_NB;  // scratch past the keys (lists)
   int32_t* dst = p.topk_out + (size_t)bh * p.k;
   const int kp = min(p.k, nb);
   const int lane = ct & 31, wid = ct >> 5;
@@ -424,84 +540,9 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     return;
   }
 
-  bool fast = kp <= 32;
-  if (fast) {
-    // thread ct owns blocks b0..b1-1 (index order)
-    const int per = (nb + NT - 1) / NT;
-    const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
-    uint32_t v = 0u;
-    for (int beta = b0; beta < b1; ++beta) v = max(v, keys[beta]);
-    // descending bitonic sort of the warp's 32 per-thread maxima
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
-        v = (((lane & j) == 0) == ((lane & k) == 0)) ? max(v, o) : min(v, o);
-      }
-    }
-    if (lane == kp - 1) tmax[wid] = v;
-    if (ct == 0) c.misc[3] = 0;
-    named_bar_sync(BAR, NT);
-    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 20 << 8);
-    uint32_t tau0 = 0u;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) tau0 = max(tau0, tmax[w]);
-    // Keys above tau0 go to the candidate list; keys equal to it (often
-    // many, e.g. scores that underflow to zero) are only counted, in block
-    // order: the lowest-index ones fill whatever the list leaves of kp.
-    int eq = 0;
-    for (int beta = b0; beta < b1; ++beta) {
-      const uint32_t key = keys[beta];
-      if (key > tau0) {
-        const int pos = atomicAdd(&c.misc[3], 1);
-        if (pos < TOPK_LIST_CAP) list[pos] = make_uint2(key, (uint32_t)beta);
-      }
-      eq += key == tau0;
-    }
-    int incl = eq;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += t;
-    }
-    if (lane == 31) c.warp_sums[wid] = incl;
-    named_bar_sync(BAR, NT);
-    if (ct == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 22 << 8);
-    const int ngt = c.misc[3];
-    // ranking costs ngt^2 / 32 comparisons: with many candidates (the
-    // top blocks spread thinly over the warps) the radix select is cheaper
-    fast = ngt <= min(TOPK_LIST_CAP, 64);
-    if (fast) {
-      // rank of a listed key = how many listed keys beat it; one warp per
-      // candidate, its lanes comparing 32 others at a time
-      for (int e = wid; e < ngt; e += NW) {
-        const uint2 me = list[e];
-        int r = 0;
-        for (int j0 = 0; j0 < ngt; j0 += 32) {
-          const int j = j0 + lane;
-          bool beats = false;
-          if (j < ngt) {
-            const uint2 o = list[j];
-            beats = (o.x > me.x) || (o.x == me.x && o.y < me.y);
-          }
-          r += __popc(__ballot_sync(0xffffffffu, beats));
-        }
-        if (lane == 0 && r < kp) dst[r] = (int32_t)me.y;
-      }
-      // keys equal to tau0 take ranks ngt, ngt+1, ... in block order
-      int before = incl - eq;
-      for (int w = 0; w < wid; ++w) before += c.warp_sums[w];
-      for (int beta = b0; beta < b1 && ngt + before < kp; ++beta) {
-        if (keys[beta] == tau0) {
-          dst[ngt + before] = beta;
-          ++before;
-        }
-      }
-      for (int slot = kp + ct; slot < p.k; slot += NT) dst[slot] = -1;
-      return;
-    }
-    named_bar_sync(BAR, NT);  // everyone has read ngt before it is reused
+  if (kp <= 32) {
+    topk_tree<NT, 1, BAR>(keys, tmax, dst, nb, kp, p.k, ct);
+    return;
   }
 
   // Radix select of the kp-th largest key, 8 bits per pass.
@@ -625,7 +666,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
     sv0[g] = make_float2(0.f, -INFINITY);
     if (FULL && ct < m.nb && g < r)
       sv0[g] = __ldcg(reinterpret_cast<const float2*>(
-          p.bstat + ((size_t)bh * p.nbmax + ct) * (2 * r) + 2 * g));
+          p.bstat + bstat_at(p, bh, g, ct)));
   }
 
   const int ncol = r * (HD / 4);             // float4 output columns
@@ -719,7 +760,7 @@ __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int
           sv[g] = sv0[g];
         } else {
           sv[g] = g < r ? __ldcg(reinterpret_cast<const float2*>(
-                              p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * r) + 2 * g))
+                              p.bstat + bstat_at(p, bh, g, beta)))
                         : make_float2(0.f, -INFINITY);
         }
       }
@@ -1101,22 +1142,32 @@ struct WarpAttn {
     }
   }
 
-  // This warp's state as is: O^T columns into so[head][dim], running max
-  // and sum into sm_[head], sz_[head].
-  __device__ __forceinline__ void store_state(float (*so)[HD], float* sm_, float* sz_) const {
+  // This warp's state as is, heads below r only: O^T rows into
+  // so[head * ld + dim], running max and sum into sm_[head], sz_[head].
+  __device__ __forceinline__ void store_state(float* so, int ld, float* sm_, float* sz_,
+                                              int r) const {
+    const int h0 = 2 * c4, h1 = 2 * c4 + 1;
 #pragma unroll
     for (int dm = 0; dm < 8; ++dm) {
       const int d0 = dm * 16 + g4;
-      so[2 * c4][d0] = o[dm][0];
-      so[2 * c4 + 1][d0] = o[dm][1];
-      so[2 * c4][d0 + 8] = o[dm][2];
-      so[2 * c4 + 1][d0 + 8] = o[dm][3];
+      if (h0 < r) {
+        so[h0 * ld + d0] = o[dm][0];
+        so[h0 * ld + d0 + 8] = o[dm][2];
+      }
+      if (h1 < r) {
+        so[h1 * ld + d0] = o[dm][1];
+        so[h1 * ld + d0 + 8] = o[dm][3];
+      }
     }
     if (g4 == 0) {
-      sm_[2 * c4] = m_run[0];
-      sm_[2 * c4 + 1] = m_run[1];
-      sz_[2 * c4] = z_run[0];
-      sz_[2 * c4 + 1] = z_run[1];
+      if (h0 < r) {
+        sm_[h0] = m_run[0];
+        sz_[h0] = z_run[0];
+      }
+      if (h1 < r) {
+        sm_[h1] = m_run[1];
+        sz_[h1] = z_run[1];
+      }
     }
   }
 
@@ -1220,11 +1271,13 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   // Programmatic launch between layers.  Every global write (and a reuse
   // layer's read of indices its immediate predecessor wrote) comes after
   // griddep_wait, which returns once the preceding kernel has completed; a
-  // kernel completes only after its own wait, so a kernel never overlaps more
-  // than its predecessor's tail.  A CTA lets the next kernel launch as soon
-  // as any of its threads executes griddep_launch_dependents, so the kernel
-  // right after a reset layer (idx_wait) triggers only after its wait: later
-  // reuse layers then read that reset layer's indices without waiting.
+  // kernel completes only after its own wait, so after a kernel's wait every
+  // earlier kernel has completed.  A CTA lets the next kernel launch as soon
+  // as any of its threads executes griddep_launch_dependents (the merge
+  // kernel does so at once, so the next layer can start on the SMs that this
+  // kernel's tail frees), and the kernel right after a reset layer (idx_wait)
+  // triggers only after its wait: later reuse layers then read that reset
+  // layer's indices without waiting.
   // Sequences without units get their outputs from merge_kernel.
   volatile int* abort_flag = &c.misc[4];
 
@@ -1383,7 +1436,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         __threadfence_block();
         ensure_waited();
         if (lane < p.r && meta_sane(p, m)) {
-          float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
+          float* dst = p.bstat + bstat_at(p, m.b * p.Hkv + m.h, lane, m.blk);
           float rec[2];
           combine_block_record<NW_BF16>(sm.bst_s[s], sm.bst_m[s], lane, rec);
           dst[0] = rec[0];
@@ -1441,6 +1494,11 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int bh = (int)blockIdx.x;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int r = p.r;
+  // The next layer's kernel may launch now: it reads nothing of this layer
+  // and writes nothing before its own wait, which returns only after this
+  // kernel, and so the streaming kernel, has completed.  Its CTAs take the
+  // SMs the streaming kernel's tail frees and start staging their tiles.
+  griddep_launch_dependents();
   if (tid == 0) {
     c.trace_n = 0;
     c.trace_cta = 160 + bh;
@@ -1467,7 +1525,6 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int kp = min(p.k, nb);
   const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
   griddep_wait();  // the streaming kernel has completed: partials are visible
-  griddep_launch_dependents();
   if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 31 << 8);
   if (U == 0) {
     // a sequence without units: zero output (and no indices)
@@ -1531,7 +1588,9 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
         sm.rz[q][g] = Z;
       }
     }
+    if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 23 << 8);
     named_bar_sync(BAR_OUT, MERGE_HALF);
+    if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 24 << 8);
     for (int col = tid; col < ncol; col += MERGE_HALF) {
       const int g = col / (HD / 4), d4 = col - g * (HD / 4);
       float M = -INFINITY;
@@ -1563,14 +1622,20 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int wb = tb >> 5, lane = tb & 31;
   if (FULL) {
     // --------------------------------------------- block scores and top-k
-    // block records of this thread's first block, loaded up front
-    float2 sv0[GMAX];
+    // block records of this thread's first SPT blocks (tb, tb + 256, ...),
+    // all loaded up front, together with the head statistics below
+    constexpr int SPT = 4;
+    float2 sv0[SPT][GMAX];
 #pragma unroll
-    for (int g = 0; g < GMAX; ++g) {
-      sv0[g] = make_float2(0.f, -INFINITY);
-      if (tb < nb && g < r)
-        sv0[g] = __ldcg(reinterpret_cast<const float2*>(
-            p.bstat + ((size_t)bh * p.nbmax + tb) * (2 * r) + 2 * g));
+    for (int u = 0; u < SPT; ++u) {
+      const int beta = tb + u * MERGE_HALF;
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        sv0[u][g] = make_float2(0.f, -INFINITY);
+        if (beta < nb && g < r)
+          sv0[u][g] = __ldcg(reinterpret_cast<const float2*>(
+              p.bstat + bstat_at(p, bh, g, beta)));
+      }
     }
     // head g's max and sum, straight from the contributors' (m, Z): warp g
     // (a (b, h) has at most MAX_CTAS contributors)
@@ -1592,6 +1657,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 19 << 8);
       float Z = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
@@ -1611,18 +1677,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     // score of block beta: its attention mass summed over the r heads
     uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
     bool nonfinite = false;
-    for (int beta = tb; beta < nb; beta += MERGE_HALF) {
-      float2 sv[GMAX];
-#pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        if (beta == tb) {
-          sv[g] = sv0[g];
-        } else {
-          sv[g] = g < r ? __ldcg(reinterpret_cast<const float2*>(
-                              p.bstat + ((size_t)bh * p.nbmax + beta) * (2 * r) + 2 * g))
-                        : make_float2(0.f, -INFINITY);
-        }
-      }
+    auto score_key = [&](const float2 (&sv)[GMAX]) {
       float score = 0.f;
 #pragma unroll
       for (int g = 0; g < GMAX; ++g)
@@ -1634,13 +1689,33 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       } else {
         nonfinite = true;
       }
-      keys[beta] = key;
+      return key;
+    };
+#pragma unroll
+    for (int u = 0; u < SPT; ++u) {
+      const int beta = tb + u * MERGE_HALF;
+      if (beta < nb) keys[beta] = score_key(sv0[u]);
+    }
+    for (int beta = tb + SPT * MERGE_HALF; beta < nb; beta += MERGE_HALF) {
+      float2 sv[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g)
+        sv[g] = g < r ? __ldcg(reinterpret_cast<const float2*>(
+                            p.bstat + bstat_at(p, bh, g, beta)))
+                      : make_float2(0.f, -INFINITY);
+      keys[beta] = score_key(sv);
     }
     if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
     named_bar_sync(BAR_TOPK, MERGE_HALF);
-    if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 12 << 8);
+    if (tb == 0) {
+      HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 12 << 8);
+      HYLRA_TRACE_VAL(c.trace_n, c.trace_cta, 43 << 8, HYLRA_CLOCK());
+    }
     topk_select<MERGE_HALF, BAR_TOPK>(p, c, bh, nb, tb);
-    if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
+    if (tb == 0) {
+      HYLRA_TRACE_VAL(c.trace_n, c.trace_cta, 44 << 8, HYLRA_CLOCK());
+      HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
+    }
 
   } else {
     // a reused list naming one block twice counts that block twice: flag it
@@ -1686,12 +1761,10 @@ struct SmemRC {
   int abort_flag;
 };
 
-// The eight consumer warps' states.
-struct RCComb {
-  float o[NW_BF16][GMAX][HD];
-  float m[NW_BF16][GMAX];
-  float z[NW_BF16][GMAX];
-};
+// The eight consumer warps' states: O^T rows [warp][head < r][RC_LD] (the
+// row pitch of HD + 4 floats spreads a warp's stores over all banks), then
+// running max and sum [warp][GMAX] each.
+constexpr int RC_LD = HD + 4;
 
 // Per-CTA slot in rank 0's gather area: O[r][HD] (unnormalised), then
 // (m, Z) per head; only the first 4 r (HD + 2) bytes are sent.
@@ -1706,9 +1779,11 @@ __host__ __device__ constexpr size_t rc_header_bytes() { return rc_align(sizeof(
 __host__ __device__ constexpr size_t rc_gather_bytes(int cs, int r) {
   return rc_align((size_t)cs * rc_slot_floats(r) * 4);
 }
-__host__ __device__ constexpr size_t rc_comb_bytes() { return rc_align(sizeof(RCComb)); }
+__host__ __device__ constexpr size_t rc_comb_bytes(int r) {
+  return rc_align((size_t)NW_BF16 * (r * RC_LD + 2 * GMAX) * 4);
+}
 __host__ __device__ constexpr size_t rc_smem_bytes(int cs, int r, int nst) {
-  return rc_header_bytes() + rc_gather_bytes(cs, r) + rc_comb_bytes() +
+  return rc_header_bytes() + rc_gather_bytes(cs, r) + rc_comb_bytes(r) +
          (size_t)nst * STAGE_BYTES;
 }
 
@@ -1756,8 +1831,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   const int CS = (int)gridDim.x;
   const int r = p.r;
   float* gather = reinterpret_cast<float*>(base + rc_header_bytes());
-  RCComb& cb = *reinterpret_cast<RCComb*>(base + rc_header_bytes() + rc_gather_bytes(CS, r));
-  uint8_t* stages = base + rc_header_bytes() + rc_gather_bytes(CS, r) + rc_comb_bytes();
+  float* comb_o = reinterpret_cast<float*>(base + rc_header_bytes() + rc_gather_bytes(CS, r));
+  float* comb_m = comb_o + NW_BF16 * r * RC_LD;  // [warp][GMAX]
+  float* comb_z = comb_m + NW_BF16 * GMAX;
+  uint8_t* stages = base + rc_header_bytes() + rc_gather_bytes(CS, r) + rc_comb_bytes(r);
   const uint32_t rank = cluster_ctarank();
   const int bh = (int)blockIdx.y;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
@@ -1938,34 +2015,33 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (!*abort_flag) *reinterpret_cast<uint4*>(dst) = __ldcg(reinterpret_cast<const uint4*>(src));
       __syncwarp();
     };
-    if (p.q_wait && !p.idx_wait && nu > 0) {
-      // while q is on its way: one pass over the first staged block with a
-      // zero query, result discarded (brings the code into the instruction
-      // cache before the timed chain starts)
-      float d0, d1, d2, d3;
-      wa.block(stages, BLK, p.scale_log2, &sm.fullV_bar[0], 0u, abort_flag, d0, d1, d2, d3);
-      wa.reset();
-    }
-    // blocks in pairs (one 256-token step each) when every block has its own
-    // stage; with refills, one at a time so each freed stage reloads early
+    // first phase of the cluster barrier (every CTA has started), needed
+    // before the stores into CTA 0; taken now, while the data is on its way
+    cluster_wait_acquire();
+    // Blocks go in pairs (one 256-token step each) when every block has its
+    // own stage; with refills, one at a time so each freed stage reloads
+    // early.  A stage is released only when a refill follows.
     int i = 0;
     for (; nu <= nst && i + 1 < nu; i += 2) {
       const int s0 = i % nst, s1 = (i + 1) % nst;
       const uint32_t ph0 = (uint32_t)((i / nst) & 1), ph1 = (uint32_t)(((i + 1) / nst) & 1);
       mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag);
       mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag);
-      if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
-      if (i == 0) wa.load_q(sm.qbuf, r);
-      patch_newest(s0, ph0);
-      patch_newest(s1, ph1);
-      wa.block2(stages + (size_t)s0 * STAGE_BYTES, sm.meta_nvalid[s0], &sm.fullV_bar[s0], ph0,
-                stages + (size_t)s1 * STAGE_BYTES, sm.meta_nvalid[s1], &sm.fullV_bar[s1], ph1,
-                p.scale_log2, abort_flag);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.empty_bar[s0]);
-        mbar_arrive(&sm.empty_bar[s1]);
+      if (ct == 0) {
+        HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
+        HYLRA_TRACE_VAL(tn, tcta, 47 << 8, HYLRA_CLOCK());
       }
+      if (i == 0) wa.load_q(sm.qbuf, r);
+      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 48 << 8, HYLRA_CLOCK());
+      const int blk0 = sm.meta_blk[s0], blk1 = sm.meta_blk[s1];
+      const int nv0 = sm.meta_nvalid[s0], nv1 = sm.meta_nvalid[s1];
+      if (blk0 == nb - 1) patch_newest(s0, ph0);
+      if (blk1 == nb - 1) patch_newest(s1, ph1);
+      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 45 << 8, HYLRA_CLOCK());
+      wa.block2(stages + (size_t)s0 * STAGE_BYTES, nv0, &sm.fullV_bar[s0], ph0,
+                stages + (size_t)s1 * STAGE_BYTES, nv1, &sm.fullV_bar[s1], ph1, p.scale_log2,
+                abort_flag);
+      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 46 << 8, HYLRA_CLOCK());
     }
     for (; i < nu; ++i) {
       const int s = i % nst;
@@ -1973,8 +2049,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
-      patch_newest(s, ph);
       const int blk = sm.meta_blk[s];
+      if (blk == nb - 1) patch_newest(s, ph);
       if (blk >= 0) {
         float mxA, mxB, sA, sB;
         wa.block(stages + (size_t)s * STAGE_BYTES, sm.meta_nvalid[s], p.scale_log2,
@@ -1982,16 +2058,21 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       } else {
         mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
+      if (i + nst < nu) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
+      }
     }
-    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
+    if (ct == 0) {
+      HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
+      HYLRA_TRACE_VAL(tn, tcta, 49 << 8, HYLRA_CLOCK());
+    }
     // this CTA's state: the eight warp states merged into one and sent to
     // slot `rank` of CTA 0's gather area (st.async: the bytes complete CTA
     // 0's gather barrier, so no cluster barrier is needed afterwards)
-    wa.store_state(cb.o[cw], cb.m[cw], cb.z[cw]);
+    wa.store_state(comb_o + cw * r * RC_LD, RC_LD, comb_m + cw * GMAX, comb_z + cw * GMAX, r);
     named_bar_sync(BAR_CONS, NT_BF16);
-    cluster_wait_acquire();  // first phase: every CTA of the cluster has started
+    if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 50 << 8, HYLRA_CLOCK());
     const uint32_t dst = mapa_shared(smem_u32(gather), 0u) + (uint32_t)((int)rank * slot) * 4u;
     const uint32_t gbar = mapa_shared(smem_u32(&sm.gather_bar), 0u);
     for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
@@ -2000,22 +2081,26 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NW_BF16; ++w) {
-        mw[w] = cb.m[w][g];
+        mw[w] = comb_m[w * GMAX + g];
         M = fmaxf(M, mw[w]);
       }
       float o0 = 0.f, o1 = 0.f, Z = 0.f;
 #pragma unroll
       for (int w = 0; w < NW_BF16; ++w) {
         const float f = (M == -INFINITY || mw[w] == -INFINITY) ? 0.f : ex2_approx(mw[w] - M);
-        const float2 ov = *reinterpret_cast<const float2*>(&cb.o[w][g][col]);
+        const float2 ov =
+            *reinterpret_cast<const float2*>(&comb_o[(w * r + g) * RC_LD + col]);
         o0 = fmaf(ov.x, f, o0);
         o1 = fmaf(ov.y, f, o1);
-        Z = fmaf(cb.z[w][g], f, Z);
+        Z = fmaf(comb_z[w * GMAX + g], f, Z);
       }
       st_async_f32x2(dst + (uint32_t)(g * HD + col) * 4u, o0, o1, gbar);
       if (col == 0) st_async_f32x2(dst + (uint32_t)(r * HD + 2 * g) * 4u, M, Z, gbar);
     }
-    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
+    if (ct == 0) {
+      HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
+      HYLRA_TRACE_VAL(tn, tcta, 52 << 8, HYLRA_CLOCK());
+    }
     if (rank == 0) {
       // ----------------------------------------------- merge (CTA rank 0)
       mbar_wait_cluster_bounded(&sm.gather_bar, 0u, abort_flag);
@@ -2212,7 +2297,7 @@ __global__ void __launch_bounds__(NT_F32, 1) decode_f32_kernel(const __grid_cons
     if (FULL && m.blk >= 0) {
       named_bar_sync(BAR_CONS, NT_F32);
       if (cw == 0 && lane < p.r && meta_sane(p, m)) {
-        float* dst = p.bstat + ((size_t)(m.b * p.Hkv + m.h) * p.nbmax + m.blk) * (2 * p.r) + 2 * lane;
+        float* dst = p.bstat + bstat_at(p, m.b * p.Hkv + m.h, lane, m.blk);
         float rec[2];
         combine_block_record<NW_F32>(sm.bst_s[i & 1], sm.bst_m[i & 1], lane, rec);
         dst[0] = rec[0];

@@ -222,9 +222,9 @@ def test_equal_scores_pick_lowest_indices():
     assert np.all(tk[0] == np.arange(6))
 
 
-def test_many_equal_scores_take_the_radix_path():
-    """1000 blocks of equal mass: more candidates than the fast selection
-    keeps, so the radix select runs; ranks must follow block index."""
+def test_many_equal_scores_rank_by_block_index():
+    """1000 blocks of equal mass (the merge tree); ranks must follow block
+    index."""
     w = W.custom("ties_many", batch=1, seqlens=(128 * 1000,), num_q_heads=8, num_kv_heads=2,
                  topk=20, seed=25)
     q, K, V = _layer(w)
@@ -243,6 +243,38 @@ def test_equal_scores_rank_by_block_index(nblocks):
     K = torch.zeros_like(K)
     _, _, _, tk, _ = _full_and_check(w, inputs=(q, K, V))
     assert np.all(tk[0] == np.arange(24))
+
+
+@pytest.mark.parametrize("nblocks,topk,dtype,structure", [
+    (300, 20, "bf16", "salient"),
+    (512, 32, "bf16", "iid"),
+    (1000, 24, "bf16", "salient"),
+    (2000, 32, "bf16", "iid"),
+    (200, 30, "fp32", "iid"),
+    (400, 32, "fp32", "salient"),
+    (513, 33, "bf16", "salient"),
+    (1024, 64, "bf16", "iid"),
+])
+def test_selection_paths_match_oracle(nblocks, topk, dtype, structure):
+    """More blocks than selection threads: the merge tree of per-warp sorted
+    lists for k' <= 32 (bf16: 256 threads, fp32: 128), the radix select
+    above; each with a ragged last block."""
+    w = W.custom(f"sel_{nblocks}_{topk}_{dtype}", batch=1, seqlens=(128 * nblocks - 37,),
+                 num_q_heads=8, num_kv_heads=2, topk=topk, dtype=dtype, structure=structure,
+                 seed=60 + nblocks % 17)
+    _full_and_check(w)
+
+
+@pytest.mark.parametrize("nblocks,topk", [(300, 20), (700, 32), (2048, 32), (600, 48)])
+def test_equal_mass_ranks_by_block_index_on_larger_paths(nblocks, topk):
+    """Every full block of equal mass on the merge-tree (k' <= 32) and radix
+    paths: ranks follow block index."""
+    w = W.custom(f"ties_tree_{nblocks}", batch=1, seqlens=(128 * nblocks,), num_q_heads=8,
+                 num_kv_heads=2, topk=topk, seed=28)
+    q, K, V = _layer(w)
+    K = torch.zeros_like(K)
+    _, _, _, tk, _ = _full_and_check(w, inputs=(q, K, V))
+    assert np.all(tk[0] == np.arange(topk))
 
 
 def test_k_larger_than_the_merge_thread_count():
