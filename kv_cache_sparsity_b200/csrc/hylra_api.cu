@@ -449,11 +449,19 @@ int gather(const hylra_shape_t* s, const void* Kh, const void* Vh, const int32_t
 
 // One decode step; offloaded (may be NULL): per layer, 1 = K[l], V[l] are a
 // host-resident cache (reuse layers only), gathered into K_stage / V_stage.
+// Host-side hooks around each layer's launches (stream order), used to
+// interleave copies with the step; nullptr: none.
+struct LayerHooks {
+  int (*before)(void* ctx, int layer);
+  int (*after)(void* ctx, int layer);
+  void* ctx;
+};
+
 int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,
              const void* const* q, const void* const* K, const void* const* V,
              const uint8_t* offloaded, const int32_t* seqlens, float* const* out, int32_t* topk,
              void* K_stage, void* V_stage, void* workspace, size_t workspace_bytes,
-             cudaStream_t stream) {
+             cudaStream_t stream, const LayerHooks* hooks = nullptr) {
   int rc = check_shape(shape);
   if (rc) return rc;
   if (num_layers < 1 || !policy || !q || !K || !V || !out || !topk) return HYLRA_ERR_INVALID;
@@ -469,6 +477,7 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
   int last_reset = 0;
   int prev_ctas = 0;  // CTAs of the kernel launched last (each holds an SM)
   for (int l = 0; l < num_layers; ++l) {
+    if (hooks && hooks->before && (rc = hooks->before(hooks->ctx, l))) return rc;
     if (policy[l]) {
       last_reset = l;
       rc = launch(shape, true, q[l], K[l], V[l], seqlens, nullptr, out[l], topk + l * per_layer,
@@ -488,7 +497,94 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
                   l & 63, prev_ctas, &prev_ctas);
     }
     if (rc) return rc;
+    if (hooks && hooks->after && (rc = hooks->after(hooks->ctx, l))) return rc;
   }
+  return HYLRA_OK;
+}
+
+// hylra_decode_step_host: a second stream carries the copies so that they
+// overlap the step.  Layer 0's query goes first on the caller's stream, the
+// other layers' queries on the copy stream (layer 1 waits for them), and the
+// outputs and indices of every OUT_CHUNK layers go back as soon as those
+// layers are done; the caller's stream joins the copy stream at the end.
+// The stream and events are per host thread and device.
+constexpr int OUT_CHUNK = 4;
+
+struct HostPipe {
+  cudaStream_t main = nullptr, copy = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_q = nullptr, ev_out = nullptr, ev_join = nullptr;
+  const uint8_t* q_host = nullptr;
+  uint8_t* q_dev = nullptr;
+  size_t q_layer_bytes = 0;
+  const float* out_dev = nullptr;
+  float* out_host = nullptr;
+  size_t out_layer_floats = 0;
+  const int32_t* topk_dev = nullptr;
+  int32_t* topk_host = nullptr;
+  size_t topk_layer = 0;
+  int num_layers = 0, copied = 0;
+};
+
+int host_pipe_resources(HostPipe* hp) {
+  struct Res {
+    cudaStream_t copy = nullptr;
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  };
+  thread_local std::vector<Res> per_dev;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
+  if ((int)per_dev.size() <= dev) per_dev.resize(dev + 1);
+  Res& r = per_dev[dev];
+  if (!r.copy) {
+    if (cudaStreamCreateWithFlags(&r.copy, cudaStreamNonBlocking) != cudaSuccess) {
+      r.copy = nullptr;
+      return HYLRA_ERR_CUDA;
+    }
+    for (auto& e : r.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return HYLRA_ERR_CUDA;
+  }
+  hp->copy = r.copy;
+  hp->ev_fork = r.ev[0];
+  hp->ev_q = r.ev[1];
+  hp->ev_out = r.ev[2];
+  hp->ev_join = r.ev[3];
+  return HYLRA_OK;
+}
+
+// the outputs (and indices) of layers [copied, upto) back to the host
+int host_pipe_copy_out(HostPipe* hp, int upto) {
+  if (upto <= hp->copied) return HYLRA_OK;
+  const int l0 = hp->copied, n = upto - l0;
+  if (cudaEventRecord(hp->ev_out, hp->main) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->copy, hp->ev_out, 0) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  if (hp->out_host &&
+      cudaMemcpyAsync(hp->out_host + l0 * hp->out_layer_floats,
+                      hp->out_dev + l0 * hp->out_layer_floats,
+                      n * hp->out_layer_floats * sizeof(float), cudaMemcpyDeviceToHost,
+                      hp->copy) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  if (hp->topk_host &&
+      cudaMemcpyAsync(hp->topk_host + l0 * hp->topk_layer, hp->topk_dev + l0 * hp->topk_layer,
+                      n * hp->topk_layer * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                      hp->copy) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  hp->copied = upto;
+  return HYLRA_OK;
+}
+
+int host_pipe_before(void* ctx, int layer) {
+  HostPipe* hp = static_cast<HostPipe*>(ctx);
+  // layer 1 on reads the queries that the copy stream brings in
+  if (layer == 1 && cudaStreamWaitEvent(hp->main, hp->ev_q, 0) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return HYLRA_OK;
+}
+
+int host_pipe_after(void* ctx, int layer) {
+  HostPipe* hp = static_cast<HostPipe*>(ctx);
+  const int done = layer + 1;
+  if (done % OUT_CHUNK == 0 && done < hp->num_layers) return host_pipe_copy_out(hp, done);
   return HYLRA_OK;
 }
 
@@ -598,30 +694,47 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
   if (rc) return rc;
   if (num_layers < 1 || !q_host || !q_dev || !out_dev || !topk_dev || !K || !V)
     return HYLRA_ERR_INVALID;
-  cudaStream_t st = (cudaStream_t)stream;
+  HostPipe hp;
+  if ((rc = host_pipe_resources(&hp))) return rc;
+  hp.main = (cudaStream_t)stream;
   const size_t q_layer = (size_t)shape->batch * shape->num_q_heads * HD;
-  const size_t q_bytes = q_layer * elem_size(shape) * num_layers;
-  const size_t out_bytes = q_layer * sizeof(float) * num_layers;
-  const size_t topk_bytes =
-      (size_t)shape->batch * shape->num_kv_heads * shape->topk * sizeof(int32_t) * num_layers;
+  hp.q_host = static_cast<const uint8_t*>(q_host);
+  hp.q_dev = static_cast<uint8_t*>(q_dev);
+  hp.q_layer_bytes = q_layer * elem_size(shape);
+  hp.out_dev = out_dev;
+  hp.out_host = out_host;
+  hp.out_layer_floats = q_layer;
+  hp.topk_dev = topk_dev;
+  hp.topk_host = topk_host;
+  hp.topk_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
+  hp.num_layers = num_layers;
   std::vector<const void*> qp(num_layers);
   std::vector<float*> op(num_layers);
   for (int l = 0; l < num_layers; ++l) {
-    qp[l] = static_cast<const uint8_t*>(q_dev) + l * q_layer * elem_size(shape);
+    qp[l] = hp.q_dev + l * hp.q_layer_bytes;
     op[l] = out_dev + l * q_layer;
   }
-  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  // layer 0's query on the caller's stream, the others on the copy stream
+  if (cudaMemcpyAsync(hp.q_dev, hp.q_host, hp.q_layer_bytes, cudaMemcpyHostToDevice, hp.main) !=
+          cudaSuccess ||
+      cudaEventRecord(hp.ev_fork, hp.main) != cudaSuccess ||
+      cudaStreamWaitEvent(hp.copy, hp.ev_fork, 0) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  rc = hylra_decode_step(shape, num_layers, policy, qp.data(), K, V, seqlens, op.data(), topk_dev,
-                         workspace, workspace_bytes, stream);
-  if (rc) return rc;
-  if (out_host &&
-      cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  if (num_layers > 1 &&
+      cudaMemcpyAsync(hp.q_dev + hp.q_layer_bytes, hp.q_host + hp.q_layer_bytes,
+                      (num_layers - 1) * hp.q_layer_bytes, cudaMemcpyHostToDevice,
+                      hp.copy) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  if (topk_host &&
-      cudaMemcpyAsync(topk_host, topk_dev, topk_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  if (cudaEventRecord(hp.ev_q, hp.copy) != cudaSuccess) return HYLRA_ERR_CUDA;
+  const LayerHooks hooks{host_pipe_before, host_pipe_after, &hp};
+  rc = run_step(shape, num_layers, policy, qp.data(), K, V, nullptr, seqlens, op.data(), topk_dev,
+                nullptr, nullptr, workspace, workspace_bytes, hp.main, &hooks);
+  // the copy stream always rejoins the caller's stream (also after an error)
+  const int rc_out = rc ? rc : host_pipe_copy_out(&hp, num_layers);
+  if (cudaEventRecord(hp.ev_join, hp.copy) != cudaSuccess ||
+      cudaStreamWaitEvent(hp.main, hp.ev_join, 0) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  return HYLRA_OK;
+  return rc_out;
 }
 
 #if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)

@@ -1524,6 +1524,24 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int nb = (seqlen + BLK - 1) / BLK;
   const int kp = min(p.k, nb);
   const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
+  if (U > 0 && tid < 8) {
+    // Before the wait: a line at each end of every range read or written
+    // after it, so that their address translations are cached when it
+    // returns (hints only; no data is used before the wait).
+    const int32_t* idx_row = (FULL ? p.topk_out : p.topk_in) + (size_t)bh * p.k;
+    const float* out_row = p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD;
+    const float* bs0 = FULL ? p.bstat + bstat_at(p, bh, 0, 0) : pbase;
+    const float* bs1 = FULL ? p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1 : pbase;
+    const void* ptr = tid == 0   ? (const void*)pbase
+                      : tid == 1 ? (const void*)(pbase + (size_t)nc * SLOT_FLOATS - 1)
+                      : tid == 2 ? (const void*)bs0
+                      : tid == 3 ? (const void*)bs1
+                      : tid == 4 ? (const void*)out_row
+                      : tid == 5 ? (const void*)(out_row + r * HD - 1)
+                      : tid == 6 ? (const void*)idx_row
+                                 : (const void*)(idx_row + max(p.k - 1, 0));
+    prefetch_line_l2(ptr);
+  }
   griddep_wait();  // the streaming kernel has completed: partials are visible
   if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 31 << 8);
   if (U == 0) {
@@ -1890,6 +1908,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     const int32_t* idx = p.topk_in + (size_t)bh * p.k;
     bool waited = false;
     if (p.idx_wait) {
+      // warm the index row's address translation (a hint) before the wait
+      if (lane == 0) prefetch_line_l2(idx + j0);
       griddep_wait();  // indices written by the preceding kernel
       waited = true;
     }
@@ -2018,6 +2038,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     // first phase of the cluster barrier (every CTA has started), needed
     // before the stores into CTA 0; taken now, while the data is on its way
     cluster_wait_acquire();
+    if (rank == 0 && ct == 0)  // the output row's address translation (a hint)
+      prefetch_line_l2(p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD);
     // Blocks go in pairs (one 256-token step each) when every block has its
     // own stage; with refills, one at a time so each freed stage reloads
     // early.  A stage is released only when a refill follows.

@@ -410,6 +410,54 @@ def test_step_host_buffers_match_device_step():
     assert run.status() == 0
 
 
+def test_step_host_buffers_in_a_cuda_graph():
+    """The host-buffer step (its copies run on a second stream, overlapped
+    with the layers) captured in a CUDA graph and replayed with new queries:
+    every replay's host outputs equal the device step on the same inputs."""
+    w = W.custom("hostgraph", batch=2, layers=9, seqlens=(3000, 1200), num_q_heads=8,
+                 num_kv_heads=2, topk=6, seed=29)
+    policy = (1, 0, 0, 1, 0, 1, 1, 0, 0)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    K, V = [l[1] for l in layers], [l[2] for l in layers]
+    L = w.layers
+    q_host = torch.stack([l[0].cpu() for l in layers]).pin_memory()
+    q_dev = torch.empty_like(q_host, device="cuda")
+    out_dev = torch.empty(L, 2, 8, 128, dtype=torch.float32, device="cuda")
+    out_host = torch.empty(L, 2, 8, 128, dtype=torch.float32).pin_memory()
+    tk_dev = torch.full((L, 2, 2, 6), -1, dtype=torch.int32, device="cuda")
+    tk_host = torch.empty(L, 2, 2, 6, dtype=torch.int32).pin_memory()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        H.decode_step_host(run.shape, policy, q_host, q_dev, K, V, run.seqlens, out_dev,
+                           out_host, tk_dev, tk_host, run.ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        H.decode_step_host(run.shape, policy, q_host, q_dev, K, V, run.seqlens, out_dev,
+                           out_host, tk_dev, tk_host, run.ws, stream=torch.cuda.current_stream())
+    gen = torch.Generator().manual_seed(5)
+    for rep in range(3):
+        q_host.copy_(torch.randn(q_host.shape, generator=gen).to(q_host.dtype))
+        out_host.fill_(float("nan"))
+        tk_host.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        outs = [run.new_out() for _ in range(L)]
+        tk2 = torch.full((L, 2, 2, 6), -1, dtype=torch.int32, device="cuda")
+        H.decode_step(run.shape, policy, [q_host[l].cuda() for l in range(L)], K, V, run.seqlens,
+                      outs, tk2, run.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out_host, torch.stack([o.cpu() for o in outs])), f"replay {rep}"
+        for l in range(L):
+            if policy[l]:
+                assert torch.equal(tk_host[l], tk2[l].cpu()), f"replay {rep} layer {l}"
+    assert run.status() == 0
+    del g
+
+
 def test_repeated_calls_are_deterministic():
     w = CASES[2]
     run = T.Runner(w)
