@@ -6,31 +6,35 @@
 //        extraction; reuse layers: attention restricted to the reused subset.
 //   §2.4 Block-level Sparsity - 128-token blocks, regular coalesced access.
 //
-// Design (one persistent CTA per SM, static "stream-K" split of the work):
-//   * A unit of work is one 128-token block of one (sequence b, KV head h):
+// Kernels:
+//   * decode_bf16_kernel: one persistent CTA per SM, static "stream-K" split.
+//     A unit of work is one 128-token block of one (sequence b, KV head h):
 //     every block of the cache on a reset layer, the k' reused blocks on a
-//     reuse layer.  Units are laid out (b, h, j)-major and CTA c takes the
-//     contiguous range [c*T/G, (c+1)*T/G), so the load is balanced to one
-//     block whatever the batch raggedness.  A CTA's range crosses (b, h)
-//     boundaries; each maximal run of one (b, h) is a "segment".
-//   * bf16 kernel: warp 0 issues TMA tile loads (128-byte swizzle, L2
-//     evict-first) of K and V blocks (64 KB per stage, 3 stages) plus the
-//     GQA group's q rows into shared memory; eight consumer warps take 16
-//     tokens each.  Q.K^T runs as S^T = K Q^T on bf16 mma.sync (M = tokens,
-//     N = the r <= 8 q-heads), the softmax is online in the log2 domain with
-//     an fp32 running max and sum per warp, P^T moves from the accumulator
-//     layout to the B-operand layout with movmatrix, and O^T = V^T P^T
-//     accumulates in fp32 registers.
-//   * Reset layers also record, per block and q-head, the block's local max
-//     and probability sum (relative to that max): the exact ingredients of
-//     the block's attention mass once the global max and sum are known.
-//   * At a segment end the four warps' states are merged (LSE) into a partial
-//     in the workspace; the last CTA to finish a (b, h) (an atomic ticket, no
-//     spinning) merges all partials into the output and, on reset layers,
-//     turns the block records into fp32 block masses and selects the top-k
-//     (radix select on the fp32 bit patterns, index order among equals).
-//   * fp32 inputs (small cases) take a CUDA-core kernel with the same work
-//     split, block records, merge and selection.
+//     reuse layer.  Units are laid out (b, h, j)-major and CTA c takes a
+//     contiguous range (part_lo: CTAs that start late, behind the preceding
+//     kernel, take a few units fewer).  Each maximal run of one (b, h) in a
+//     CTA is a "segment" and leaves one partial state in the workspace.  Warp
+//     0 issues TMA tile loads (128-byte swizzle, L2 evict-first) of K and V
+//     (64 KB per stage, 3 stages) plus the GQA group's q rows; eight consumer
+//     warps take 16 tokens each.  Q.K^T runs as S^T = K Q^T on bf16
+//     mma.sync (M = tokens, N = the r <= 8 q-heads), the softmax is online in
+//     the log2 domain with an fp32 running max and sum per warp, P^T moves
+//     to the B-operand layout with movmatrix, and O^T = V^T P^T accumulates
+//     in fp32 registers.  Reset layers also record, per block and q-head, the
+//     block's local max and probability sum relative to it: the exact
+//     ingredients of the block's attention mass once the global max and sum
+//     are known.
+//   * merge_kernel: the streaming kernel's programmatic dependent, one CTA
+//     per (b, h): LSE merge of the segments' partials into the output and,
+//     on reset layers, the block masses and the top-k (topk_select).
+//   * decode_reuse_cluster_kernel: a reuse layer as one thread-block
+//     cluster per (b, h); the CTAs' states meet in CTA 0's shared memory
+//     (st.async), which writes the output.
+//   * gather_blocks_kernel: index-guided offloading, the reused blocks from
+//     host memory into a device staging cache.
+//   * decode_f32_kernel: fp32 inputs (small cases), CUDA cores, the same
+//     split and records; the last CTA of a (b, h) (an atomic ticket, no
+//     spinning) merges and selects in-kernel (merge_bh).
 #pragma once
 
 #include <cuda_bf16.h>
