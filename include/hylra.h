@@ -189,12 +189,16 @@ int hylra_decode_step_offload(const hylra_shape_t* shape, int32_t num_layers,
                               void* workspace, size_t workspace_bytes, hylra_stream_t stream);
 
 /* The same step with the per-step inputs and outputs in HOST memory:
- * q_host [num_layers][B][Hq][d] is copied to q_dev (same shape, device) and,
- * after the step, out_dev [num_layers][B][Hq][d] fp32 to out_host and
- * topk_dev [num_layers][B][Hkv][k] to topk_host (either host pointer may be
- * NULL to skip that copy).  Host buffers should be pinned for asynchronous
- * copies.  Returns after enqueueing; synchronise the stream before reading
- * the host outputs. */
+ * q_host [num_layers][B][Hq][d] is copied to q_dev (same shape, device) and
+ * out_dev [num_layers][B][Hq][d] fp32 to out_host and topk_dev
+ * [num_layers][B][Hkv][k] to topk_host (either host pointer may be NULL to
+ * skip that copy).  The copies overlap the layers: they run on a second
+ * stream owned by the library (one per host thread and device, created by
+ * the thread's first call, which should therefore not be inside a stream
+ * capture), with event dependencies on `stream`, which has waited for all of
+ * them when the call's work on it completes.  Host buffers should be pinned
+ * for asynchronous copies.  Returns after enqueueing; synchronise the stream
+ * before reading the host outputs. */
 int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers,
                            const uint8_t* policy, const void* q_host, void* q_dev,
                            const void* const* K, const void* const* V,
