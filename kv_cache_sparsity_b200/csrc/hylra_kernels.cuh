@@ -1320,8 +1320,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       qpend = 0u;
     };
     int idx_cur = FULL ? 0 : unit_index_entry(p, it);
-    int tn = 0;
-    (void)tn;
+#ifdef HYLRA_TRACE
+    int tn = 0;  // trace events of the producer thread
+#endif
     for (int i = 0; i < n; ++i) {
       UnitIter nx = it;
       nx.advance(c, p);
@@ -1892,8 +1893,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   const int j0 = (int)rank * upc;
   const int nu = max(0, min(upc, kp - j0));  // blocks of this CTA
   const int tcta = bh * CS + (int)rank;
-  int tn = 0;
-  (void)tn;
+#ifdef HYLRA_TRACE
+  int tn = 0;  // trace events of the first consumer thread
+#endif
   (void)tcta;
   if (tid == 32) {
     HYLRA_TRACE_CTA(tn, tcta, 1 << 8);
@@ -1935,8 +1937,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (__any_sync(0xffffffffu, dup) && lane == 0) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
     }
     griddep_launch_dependents();  // the producer writes nothing
+#ifdef HYLRA_TRACE
     int tp = 128;  // trace events of the producer thread
-    (void)tp;
+#endif
     if (lane == 0) HYLRA_TRACE_CTA(tp, tcta, 2 << 8);
     const uint64_t pol = l2_evict_first_policy();
     const long long row0 = row_base(p, b, h);
