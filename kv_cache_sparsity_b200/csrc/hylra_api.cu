@@ -280,6 +280,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   if (!full && (!topk_in || !aligned(topk_in, 4))) return HYLRA_ERR_INVALID;
   int G = 0;
   if ((rc = sm_count(&G))) return rc;
+  const int G_sms = G;  // before G becomes this launch's streaming grid
   const Layout L = make_layout(s, G);
   if (ws_bytes < L.total) return HYLRA_ERR_WORKSPACE;
 
@@ -374,7 +375,9 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     if (e != cudaSuccess) return HYLRA_ERR_CUDA;
     // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
-    mcfg.gridDim = dim3(s->batch * s->num_kv_heads);
+    const int nout = merge_out_ctas(s->num_q_heads / s->num_kv_heads,
+                                    (long long)s->batch * s->num_kv_heads, G_sms);
+    mcfg.gridDim = dim3(s->batch * s->num_kv_heads, 1 + nout);
     mcfg.blockDim = dim3(NT_MERGE);
     mcfg.dynamicSmemBytes = 0;
     mcfg.stream = stream;
@@ -384,7 +387,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
                                 : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
     if (em != cudaSuccess) return HYLRA_ERR_CUDA;
-    if (last_ctas) *last_ctas = s->batch * s->num_kv_heads;
+    if (last_ctas) *last_ctas = s->batch * s->num_kv_heads * (1 + nout);
   } else {
     if (full)
       decode_f32_kernel<true><<<G, NT_F32, 0, stream>>>(p);

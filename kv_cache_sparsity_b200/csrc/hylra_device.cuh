@@ -106,10 +106,14 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-// Touch one line (a hint: warms the address translation and L2, returns
-// no data).
-__device__ __forceinline__ void prefetch_line_l2(const void* ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr) : "memory");
+// Touch one line with a load whose value is discarded: the address
+// translation (and the line) are then cached for the loads that follow.  The
+// value may be stale (callers touch before their PDL wait) and is never used;
+// nothing waits for the load to return.
+__device__ __forceinline__ void touch_line(const void* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  asm volatile("" ::"r"(v));
 }
 
 // Bring one box of a 2-D tensor map into L2 (x aligned as for tma_load_2d).

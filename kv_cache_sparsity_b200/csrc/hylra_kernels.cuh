@@ -54,7 +54,7 @@ constexpr int NTHR_BF16 = NT_BF16 + 32;  // + one producer warp
 constexpr int NW_F32 = 4;                // warps of the fp32 kernel (32 tokens each)
 constexpr int NT_F32 = NW_F32 * 32;
 constexpr int NWMAX = 8;
-constexpr int NT_MERGE = 512;              // threads of the merge kernel
+constexpr int NT_MERGE = 256;              // threads of a merge CTA
 constexpr int NCOMB = 4;                 // per-warp states merged at a segment end
 constexpr int NSTAGE = 3;
 constexpr int BOX_BYTES = 64 * 2 * BLK;       // 64 bf16 columns x 128 rows
@@ -1471,20 +1471,33 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 
 // ------------------------------------------------------------ merge kernel
 //
-// Runs after decode_bf16_kernel (as its programmatic dependent): one CTA per
-// (sequence, KV head).  The kernel boundary makes the streaming kernel's
-// partials visible; no fence or ticket is needed.  Two independent halves
-// run side by side so that neither waits for the other:
-//   warps 0-7   merge the contributors' partial rows into the output;
-//   warps 8-15  (reset layers) derive each head's max and sum straight from
-//               the contributors' (m, Z) pairs, score the blocks and select
-//               the top-k; (reuse layers) check the index list for repeats.
-constexpr int MERGE_HALF = NT_MERGE / 2;
-constexpr int BAR_OUT = 2;   // named barrier of warps 0-7
-constexpr int BAR_TOPK = 3;  // named barrier of warps 8-15
+// Runs after decode_bf16_kernel (as its programmatic dependent).  The kernel
+// boundary makes the streaming kernel's partials visible; no fence or ticket
+// is needed.  Grid (B*Hkv, 1 + merge_out_ctas(..)): for each (sequence, KV
+// head) independent CTAs run side by side so that none waits for another and
+// each SM loads only its share of the partials:
+//   y = 0      (reset layers) derives each head's max and sum straight from
+//              the contributors' (m, Z) pairs, scores the blocks and selects
+//              the top-k; (reuse layers) checks the index list for repeats;
+//   y = 1..    each merges the contributors' partial rows of its heads into
+//              the output.
+constexpr int BAR_TOPK = 3;           // named barrier of the selection CTA
+
+// Output CTAs per (b, h): one per head up to four when the grid stays
+// within one wave of SMs (few sequences and heads: each SM then loads a
+// smaller share of the partials), else one.  Heads [g0, g1) of output CTA
+// `part` (1..n).
+__host__ __device__ constexpr int merge_out_ctas(int r, long long nbh, int sms) {
+  return nbh * (1 + (r < 4 ? r : 4)) <= sms ? (r < 4 ? r : 4) : 1;
+}
+__device__ __forceinline__ void merge_out_heads(int r, int n, int part, int& g0, int& g1) {
+  const int per = (r + n - 1) / n;
+  g0 = min(r, (part - 1) * per);
+  g1 = min(r, g0 + per);
+}
 
 struct SmemMerge {
-  float4 red[MERGE_HALF];  // per-group partial rows, [group][float4 column]
+  float4 red[NT_MERGE];    // per-group partial rows, [group][float4 column]
   float rm[NWMAX][GMAX];   // per-group running max and sum
   float rz[NWMAX][GMAX];
   SmemCommon c;            // prefix sums; head statistics, keys and top-k scratch
@@ -1497,8 +1510,11 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   SmemCommon& c = sm.c;
   const int tid = threadIdx.x;
   const int bh = (int)blockIdx.x;
+  const int part = (int)blockIdx.y;  // 0: statistics and top-k; 1..: output heads
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int r = p.r;
+  int g0 = 0, g1 = 0;
+  if (part > 0) merge_out_heads(r, (int)gridDim.y - 1, part, g0, g1);
   // The next layer's kernel may launch now: it reads nothing of this layer
   // and writes nothing before its own wait, which returns only after this
   // kernel, and so the streaming kernel, has completed.  Its CTAs take the
@@ -1506,7 +1522,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   griddep_launch_dependents();
   if (tid == 0) {
     c.trace_n = 0;
-    c.trace_cta = 160 + bh;
+    c.trace_cta = 160 + bh * 8 + part;
     HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 30 << 8);
   }
   // everything that does not depend on the streaming kernel's output first
@@ -1529,43 +1545,51 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int nb = (seqlen + BLK - 1) / BLK;
   const int kp = min(p.k, nb);
   const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
-  if (U > 0 && tid < 8) {
+  float* out_bh = p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD;
+  if (U > 0 && tid < 6) {
     // Before the wait: a line at each end of every range read or written
     // after it, so that their address translations are cached when it
-    // returns (hints only; no data is used before the wait).
+    // returns (values discarded: nothing is used before the wait).
     const int32_t* idx_row = (FULL ? p.topk_out : p.topk_in) + (size_t)bh * p.k;
-    const float* out_row = p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD;
-    const float* bs0 = FULL ? p.bstat + bstat_at(p, bh, 0, 0) : pbase;
-    const float* bs1 = FULL ? p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1 : pbase;
-    const void* ptr = tid == 0   ? (const void*)pbase
-                      : tid == 1 ? (const void*)(pbase + (size_t)nc * SLOT_FLOATS - 1)
-                      : tid == 2 ? (const void*)bs0
-                      : tid == 3 ? (const void*)bs1
-                      : tid == 4 ? (const void*)out_row
-                      : tid == 5 ? (const void*)(out_row + r * HD - 1)
-                      : tid == 6 ? (const void*)idx_row
-                                 : (const void*)(idx_row + max(p.k - 1, 0));
-    prefetch_line_l2(ptr);
+    const void* ptr;
+    if (part == 0) {
+      const float* bs0 = FULL ? p.bstat + bstat_at(p, bh, 0, 0) : pbase;
+      const float* bs1 = FULL ? p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1 : pbase;
+      ptr = tid == 0 ? (const void*)bs0
+          : tid == 1 ? (const void*)bs1
+          : tid == 2 ? (const void*)idx_row
+          : tid == 3 ? (const void*)(idx_row + max(p.k - 1, 0))
+          : tid == 4 ? (const void*)(pbase + GMAX * HD)
+                     : (const void*)(pbase + (size_t)nc * SLOT_FLOATS - 1);
+    } else {
+      ptr = tid == 0 ? (const void*)pbase
+          : tid == 1 ? (const void*)(pbase + (size_t)nc * SLOT_FLOATS - 1)
+          : tid == 2 ? (const void*)(out_bh + g0 * HD)
+          : tid == 3 ? (const void*)(out_bh + g1 * HD - 1)
+          : tid == 4 ? (const void*)(pbase + (size_t)(nc / 2) * SLOT_FLOATS)
+                     : (const void*)(pbase + (size_t)(nc - 1) * SLOT_FLOATS);
+    }
+    touch_line(ptr);
   }
   griddep_wait();  // the streaming kernel has completed: partials are visible
   if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 31 << 8);
   if (U == 0) {
     // a sequence without units: zero output (and no indices)
-    for (int i = tid; i < r * HD; i += NT_MERGE)
-      p.out[((size_t)b * p.Hq + (size_t)h * r) * HD + i] = 0.f;
-    if (FULL)
+    if (part > 0)
+      for (int i = g0 * HD + tid; i < g1 * HD; i += NT_MERGE) out_bh[i] = 0.f;
+    else if (FULL)
       for (int i = tid; i < p.k; i += NT_MERGE) p.topk_out[(size_t)bh * p.k + i] = -1;
     return;
   }
 
-  if (tid < MERGE_HALF) {
-    // ------------------------------------------------ output rows (LSE merge)
+  if (part > 0) {
+    // ------------------------------------------ output rows g0..g1-1 (LSE merge)
     constexpr int CB = 10;  // contributors per thread and batch of loads
-    const int ncol = r * (HD / 4);  // float4 columns
-    const int GA = ncol >= MERGE_HALF ? 1 : min(NWMAX, MERGE_HALF / ncol);
-    for (int t = tid; t < GA * ncol; t += MERGE_HALF) {
+    const int ncol = (g1 - g0) * (HD / 4);  // float4 columns
+    const int GA = ncol >= NT_MERGE ? 1 : min(NWMAX, NT_MERGE / ncol);
+    for (int t = tid; t < GA * ncol; t += NT_MERGE) {
       const int q = t / ncol, col = t - q * ncol;
-      const int g = col / (HD / 4), d4 = col - g * (HD / 4);
+      const int g = g0 + col / (HD / 4), d4 = col % (HD / 4);
       float M = -INFINITY, Z = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int j0 = q; j0 < nc; j0 += GA * CB) {
@@ -1573,7 +1597,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
         float4 ov[CB];
 #pragma unroll
         for (int u = 0; u < CB; ++u) {
-          const int j = j0 + u * GA;
+          const int j = j0 + u * GA;  // the same in every lane of a warp
           mv[u] = -INFINITY;
           if (j < nc) {
             const float* sl = pbase + (size_t)j * SLOT_FLOATS;
@@ -1611,11 +1635,10 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
         sm.rz[q][g] = Z;
       }
     }
-    if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 23 << 8);
-    named_bar_sync(BAR_OUT, MERGE_HALF);
+    __syncthreads();
     if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 24 << 8);
-    for (int col = tid; col < ncol; col += MERGE_HALF) {
-      const int g = col / (HD / 4), d4 = col - g * (HD / 4);
+    for (int col = tid; col < ncol; col += NT_MERGE) {
+      const int g = g0 + col / (HD / 4), d4 = col % (HD / 4);
       float M = -INFINITY;
       for (int q = 0; q < GA; ++q) M = fmaxf(M, sm.rm[q][g]);
       float Z = 0.f;
@@ -1635,29 +1658,33 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       }
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
       if (Z > 0.f) o = make_float4(acc.x / Z, acc.y / Z, acc.z / Z, acc.w / Z);
-      *reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + (size_t)h * r + g) * HD + 4 * d4) = o;
+      *reinterpret_cast<float4*>(out_bh + g * HD + 4 * d4) = o;
     }
     if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 17 << 8);
     return;
   }
 
-  const int tb = tid - MERGE_HALF;  // 0..255
+  const int tb = tid;  // 0..NT_MERGE-1
   const int wb = tb >> 5, lane = tb & 31;
   if (FULL) {
     // --------------------------------------------- block scores and top-k
     // block records of this thread's first SPT blocks (tb, tb + 256, ...),
     // all loaded up front, together with the head statistics below
+    // (the conditions are the same in every lane of a warp and lanes past
+    // the last block reload it, so no load result selects against a
+    // default, which would wait for that load on the spot; entries g >= r
+    // and blocks past nb are never read)
     constexpr int SPT = 4;
     float2 sv0[SPT][GMAX];
 #pragma unroll
     for (int u = 0; u < SPT; ++u) {
-      const int beta = tb + u * MERGE_HALF;
+      if (u * NT_MERGE + wb * 32 < nb) {
+        const int beta = min(tb + u * NT_MERGE, nb - 1);
 #pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        sv0[u][g] = make_float2(0.f, -INFINITY);
-        if (beta < nb && g < r)
-          sv0[u][g] = __ldcg(reinterpret_cast<const float2*>(
-              p.bstat + bstat_at(p, bh, g, beta)));
+        for (int g = 0; g < GMAX; ++g)
+          if (g < r)
+            sv0[u][g] =
+                __ldcg(reinterpret_cast<const float2*>(p.bstat + bstat_at(p, bh, g, beta)));
       }
     }
     // head g's max and sum, straight from the contributors' (m, Z): warp g
@@ -1668,13 +1695,17 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       float M = -INFINITY;
 #pragma unroll
       for (int u = 0; u < MAX_CTAS / 32; ++u) {
-        const int j = u * 32 + lane;
-        mj[u] = -INFINITY;
-        zj[u] = 0.f;
-        if (j < nc) {
-          const float* sl = pbase + (size_t)j * SLOT_FLOATS;
+        if (u * 32 < nc) {  // warp-uniform; lanes past nc reload the last one
+          const float* sl = pbase + (size_t)min(u * 32 + lane, nc - 1) * SLOT_FLOATS;
           mj[u] = __ldcg(sl + GMAX * HD + g);
           zj[u] = __ldcg(sl + GMAX * HD + GMAX + g);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < MAX_CTAS / 32; ++u) {
+        if (u * 32 + lane >= nc) {
+          mj[u] = -INFINITY;
+          zj[u] = 0.f;
         }
         M = fmaxf(M, mj[u]);
       }
@@ -1695,7 +1726,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
         c.rzg[g] = Z > 0.f ? 1.f / Z : 0.f;
       }
     }
-    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    named_bar_sync(BAR_TOPK, NT_MERGE);
     if (tb == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 18 << 8);
     // score of block beta: its attention mass summed over the r heads
     uint32_t* keys = reinterpret_cast<uint32_t*>(&c.comb_o[0][0][0]);
@@ -1716,10 +1747,10 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     };
 #pragma unroll
     for (int u = 0; u < SPT; ++u) {
-      const int beta = tb + u * MERGE_HALF;
+      const int beta = tb + u * NT_MERGE;
       if (beta < nb) keys[beta] = score_key(sv0[u]);
     }
-    for (int beta = tb + SPT * MERGE_HALF; beta < nb; beta += MERGE_HALF) {
+    for (int beta = tb + SPT * NT_MERGE; beta < nb; beta += NT_MERGE) {
       float2 sv[GMAX];
 #pragma unroll
       for (int g = 0; g < GMAX; ++g)
@@ -1729,12 +1760,12 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       keys[beta] = score_key(sv);
     }
     if (nonfinite) atomicOr(p.status, HYLRA_STATUS_NONFINITE);
-    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    named_bar_sync(BAR_TOPK, NT_MERGE);
     if (tb == 0) {
       HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 12 << 8);
       HYLRA_TRACE_VAL(c.trace_n, c.trace_cta, 43 << 8, HYLRA_CLOCK());
     }
-    topk_select<MERGE_HALF, BAR_TOPK>(p, c, bh, nb, tb);
+    topk_select<NT_MERGE, BAR_TOPK>(p, c, bh, nb, tb);
     if (tb == 0) {
       HYLRA_TRACE_VAL(c.trace_n, c.trace_cta, 44 << 8, HYLRA_CLOCK());
       HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
@@ -1744,10 +1775,10 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     // a reused list naming one block twice counts that block twice: flag it
     const int32_t* idx = p.topk_in + (size_t)bh * p.k;
     int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
-    for (int e = tb; e < kp; e += MERGE_HALF) sidx[e] = __ldcg(idx + e);
-    named_bar_sync(BAR_TOPK, MERGE_HALF);
+    for (int e = tb; e < kp; e += NT_MERGE) sidx[e] = __ldcg(idx + e);
+    named_bar_sync(BAR_TOPK, NT_MERGE);
     bool dup = false;
-    for (int e = tb; e < kp; e += MERGE_HALF) {
+    for (int e = tb; e < kp; e += NT_MERGE) {
       const int32_t v = sidx[e];
       if (v < 0) continue;
       for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
@@ -1914,8 +1945,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     const int32_t* idx = p.topk_in + (size_t)bh * p.k;
     bool waited = false;
     if (p.idx_wait) {
-      // warm the index row's address translation (a hint) before the wait
-      if (lane == 0) prefetch_line_l2(idx + j0);
+      // warm the index row's address translation before the wait
+      if (lane == 0) touch_line(idx + j0);
       griddep_wait();  // indices written by the preceding kernel
       waited = true;
     }
@@ -2045,8 +2076,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     // first phase of the cluster barrier (every CTA has started), needed
     // before the stores into CTA 0; taken now, while the data is on its way
     cluster_wait_acquire();
-    if (rank == 0 && ct == 0)  // the output row's address translation (a hint)
-      prefetch_line_l2(p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD);
+    if (rank == 0 && ct == 0)  // the output row's address translation
+      touch_line(p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD);
     // Blocks go in pairs (one 256-token step each) when every block has its
     // own stage; with refills, one at a time so each freed stage reloads
     // early.  A stage is released only when a refill follows.
@@ -2056,21 +2087,15 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       const uint32_t ph0 = (uint32_t)((i / nst) & 1), ph1 = (uint32_t)(((i + 1) / nst) & 1);
       mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag);
       mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag);
-      if (ct == 0) {
-        HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
-        HYLRA_TRACE_VAL(tn, tcta, 47 << 8, HYLRA_CLOCK());
-      }
+      if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
-      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 48 << 8, HYLRA_CLOCK());
       const int blk0 = sm.meta_blk[s0], blk1 = sm.meta_blk[s1];
       const int nv0 = sm.meta_nvalid[s0], nv1 = sm.meta_nvalid[s1];
       if (blk0 == nb - 1) patch_newest(s0, ph0);
       if (blk1 == nb - 1) patch_newest(s1, ph1);
-      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 45 << 8, HYLRA_CLOCK());
       wa.block2(stages + (size_t)s0 * STAGE_BYTES, nv0, &sm.fullV_bar[s0], ph0,
                 stages + (size_t)s1 * STAGE_BYTES, nv1, &sm.fullV_bar[s1], ph1, p.scale_log2,
                 abort_flag);
-      if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 46 << 8, HYLRA_CLOCK());
     }
     for (; i < nu; ++i) {
       const int s = i % nst;
@@ -2092,16 +2117,12 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
       }
     }
-    if (ct == 0) {
-      HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
-      HYLRA_TRACE_VAL(tn, tcta, 49 << 8, HYLRA_CLOCK());
-    }
+    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 4 << 8);
     // this CTA's state: the eight warp states merged into one and sent to
     // slot `rank` of CTA 0's gather area (st.async: the bytes complete CTA
     // 0's gather barrier, so no cluster barrier is needed afterwards)
     wa.store_state(comb_o + cw * r * RC_LD, RC_LD, comb_m + cw * GMAX, comb_z + cw * GMAX, r);
     named_bar_sync(BAR_CONS, NT_BF16);
-    if (ct == 0) HYLRA_TRACE_VAL(tn, tcta, 50 << 8, HYLRA_CLOCK());
     const uint32_t dst = mapa_shared(smem_u32(gather), 0u) + (uint32_t)((int)rank * slot) * 4u;
     const uint32_t gbar = mapa_shared(smem_u32(&sm.gather_bar), 0u);
     for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {
@@ -2126,10 +2147,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       st_async_f32x2(dst + (uint32_t)(g * HD + col) * 4u, o0, o1, gbar);
       if (col == 0) st_async_f32x2(dst + (uint32_t)(r * HD + 2 * g) * 4u, M, Z, gbar);
     }
-    if (ct == 0) {
-      HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
-      HYLRA_TRACE_VAL(tn, tcta, 52 << 8, HYLRA_CLOCK());
-    }
+    if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
     if (rank == 0) {
       // ----------------------------------------------- merge (CTA rank 0)
       mbar_wait_cluster_bounded(&sm.gather_bar, 0u, abort_flag);
