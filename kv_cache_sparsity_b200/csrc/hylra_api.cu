@@ -511,7 +511,7 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
 // outputs and indices of every OUT_CHUNK layers go back as soon as those
 // layers are done; the caller's stream joins the copy stream at the end.
 // The stream and events are per host thread and device.
-constexpr int OUT_CHUNK = 4;
+constexpr int OUT_CHUNK = 8;
 
 struct HostPipe {
   cudaStream_t main = nullptr, copy = nullptr;
