@@ -146,19 +146,30 @@ int prepare_bf16_kernels() {
 // pipeline stages.
 struct RCPlan {
   int cs, upc, nst;
+  bool comb_in_stage;
   size_t smem;
 };
 
 // Stages: one per block of the CTA up to NST_MAX_RC, as many as fit beside
-// the gather area (0: this cluster size does not fit).
+// the gather area (0: this cluster size does not fit); when blocks outnumber
+// the stages that fit, the warp states move into stage 0 at the end if that
+// makes room for one more.
 RCPlan rc_plan_for(int cs, int kmax, int r, int nst_cap = NST_MAX_RC) {
   RCPlan pl{};
   pl.cs = cs;
   pl.upc = (kmax + cs - 1) / cs;
-  const size_t fixed = rc_smem_bytes(cs, r, 0) + 1024;
-  const int fit = fixed >= kSmemMax ? 0 : (int)((kSmemMax - fixed) / STAGE_BYTES);
-  pl.nst = std::min(std::min(pl.upc, nst_cap), fit);
-  pl.smem = rc_smem_bytes(cs, r, pl.nst) + 1024;
+  const int want = std::min(pl.upc, nst_cap);
+  for (int alias = 0; alias < 2; ++alias) {
+    const size_t fixed = rc_smem_bytes(cs, r, 0, alias != 0) + 1024;
+    const int fit = fixed >= kSmemMax ? 0 : (int)((kSmemMax - fixed) / STAGE_BYTES);
+    const int nst = std::min(want, fit);
+    if (alias == 0 || nst > pl.nst) {
+      pl.nst = nst;
+      pl.comb_in_stage = alias != 0;
+    }
+    if (pl.nst >= want) break;
+  }
+  pl.smem = rc_smem_bytes(cs, r, pl.nst, pl.comb_in_stage) + 1024;
   return pl;
 }
 
@@ -340,6 +351,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
       if (plan_reuse_cluster(s, &pl)) {
         p.upc = pl.upc;
         p.nst = pl.nst;
+        p.comb_in_stage = pl.comb_in_stage ? 1 : 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(pl.cs, nbh);
         cfg.blockDim = dim3(NTHR_BF16);

@@ -131,6 +131,7 @@ struct Params {
   int late_deficit;  // still held by the preceding kernel) and take this many units fewer
   int q_wait;        // q and each sequence's newest K/V row come from the preceding kernel
   int upc, nst;      // cluster reuse kernel: blocks per CTA, pipeline stages
+  int comb_in_stage; // cluster reuse kernel: the warp states go to stage 0 at the end
   int trace_slot;    // trace builds: which per-launch region of the trace buffer
   float scale_log2;  // log2(e) / sqrt(d)
 };
@@ -1836,8 +1837,12 @@ __host__ __device__ constexpr size_t rc_gather_bytes(int cs, int r) {
 __host__ __device__ constexpr size_t rc_comb_bytes(int r) {
   return rc_align((size_t)NW_BF16 * (r * RC_LD + 2 * GMAX) * 4);
 }
-__host__ __device__ constexpr size_t rc_smem_bytes(int cs, int r, int nst) {
-  return rc_header_bytes() + rc_gather_bytes(cs, r) + rc_comb_bytes(r) +
+// With comb_in_stage the warp states go to stage 0, which every consumer
+// warp is done with by then (a barrier first); that leaves room for one more
+// stage when blocks outnumber stages.
+__host__ __device__ constexpr size_t rc_smem_bytes(int cs, int r, int nst,
+                                                   bool comb_in_stage = false) {
+  return rc_header_bytes() + rc_gather_bytes(cs, r) + (comb_in_stage ? 0 : rc_comb_bytes(r)) +
          (size_t)nst * STAGE_BYTES;
 }
 
@@ -1885,10 +1890,11 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   const int CS = (int)gridDim.x;
   const int r = p.r;
   float* gather = reinterpret_cast<float*>(base + rc_header_bytes());
-  float* comb_o = reinterpret_cast<float*>(base + rc_header_bytes() + rc_gather_bytes(CS, r));
+  uint8_t* after_gather = base + rc_header_bytes() + rc_gather_bytes(CS, r);
+  uint8_t* stages = after_gather + (p.comb_in_stage ? 0 : rc_comb_bytes(r));
+  float* comb_o = reinterpret_cast<float*>(p.comb_in_stage ? stages : after_gather);
   float* comb_m = comb_o + NW_BF16 * r * RC_LD;  // [warp][GMAX]
   float* comb_z = comb_m + NW_BF16 * GMAX;
-  uint8_t* stages = base + rc_header_bytes() + rc_gather_bytes(CS, r) + rc_comb_bytes(r);
   const uint32_t rank = cluster_ctarank();
   const int bh = (int)blockIdx.y;
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
@@ -2121,6 +2127,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     // this CTA's state: the eight warp states merged into one and sent to
     // slot `rank` of CTA 0's gather area (st.async: the bytes complete CTA
     // 0's gather barrier, so no cluster barrier is needed afterwards)
+    if (p.comb_in_stage) named_bar_sync(BAR_CONS, NT_BF16);  // stage 0 no longer read
     wa.store_state(comb_o + cw * r * RC_LD, RC_LD, comb_m + cw * GMAX, comb_z + cw * GMAX, r);
     named_bar_sync(BAR_CONS, NT_BF16);
     const uint32_t dst = mapa_shared(smem_u32(gather), 0u) + (uint32_t)((int)rank * slot) * 4u;

@@ -166,6 +166,22 @@ def test_reuse_with_every_block_equals_full(dtype):
     assert torch.allclose(out_r, out_f, atol=tol, rtol=0)
 
 
+def test_reuse_many_blocks_per_cta():
+    """k = 64 of 128 blocks over 8 KV heads: each cluster CTA takes several
+    blocks with refills (the plan that also puts the warp states into a
+    stage at the end to fit a third stage)."""
+    w = W.custom("reuse_k64", batch=1, layers=2, seqlens=(128 * 128 - 5,), num_q_heads=32,
+                 num_kv_heads=8, topk=64, seed=31)
+    run = T.Runner(w)
+    q0, K0, V0 = _layer(w, 0)
+    q1, K1, V1 = _layer(w, 1)
+    _, tk = run.full(q0, K0, V0)
+    out = run.reuse(q1, K1, V1, tk).cpu().numpy()
+    assert run.status() == 0
+    ref = T.oracle_reuse(w, q1, K1, V1, 0, tk.cpu().numpy()[0])
+    T.check_out(out[0], ref, "bf16", "reuse_k64")
+
+
 def test_reuse_skips_minus_one_and_flags_bad_indices():
     w = W.custom("badidx", batch=1, seqlens=(1000,), num_q_heads=8, num_kv_heads=2, topk=4,
                  seed=16)
