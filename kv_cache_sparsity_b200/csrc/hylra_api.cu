@@ -519,9 +519,10 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
 
 // hylra_decode_step_host: a second stream carries the copies so that they
 // overlap the step.  Layer 0's query goes first on the caller's stream, the
-// other layers' queries on the copy stream (layer 1 waits for them), and the
-// outputs and indices of every OUT_CHUNK layers go back as soon as those
-// layers are done; the caller's stream joins the copy stream at the end.
+// other layers' queries on the copy stream (layer 1 waits for them), the
+// outputs of every OUT_CHUNK layers go back as soon as those layers are done
+// and the indices once the last reset layer is; the caller's stream joins
+// the copy stream at the end.
 // The stream and events are per host thread and device.
 constexpr int OUT_CHUNK = 8;
 
@@ -538,6 +539,7 @@ struct HostPipe {
   int32_t* topk_host = nullptr;
   size_t topk_layer = 0;
   int num_layers = 0, copied = 0;
+  int last_reset = 0;  // the indices are final once this layer is done
 };
 
 int host_pipe_resources(HostPipe* hp) {
@@ -566,25 +568,29 @@ int host_pipe_resources(HostPipe* hp) {
   return HYLRA_OK;
 }
 
-// the outputs (and indices) of layers [copied, upto) back to the host
-int host_pipe_copy_out(HostPipe* hp, int upto) {
-  if (upto <= hp->copied) return HYLRA_OK;
-  const int l0 = hp->copied, n = upto - l0;
+// After layer `done - 1`: the outputs of layers [copied, upto) back to the
+// host and, once the last reset layer is done, all layers' indices (the
+// step writes no others) in one copy.
+int host_pipe_copy_out(HostPipe* hp, int upto, bool topk) {
+  const bool out = upto > hp->copied && hp->out_host;
+  topk = topk && hp->topk_host;
+  if (!out && !topk) return HYLRA_OK;
   if (cudaEventRecord(hp->ev_out, hp->main) != cudaSuccess ||
       cudaStreamWaitEvent(hp->copy, hp->ev_out, 0) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  if (hp->out_host &&
-      cudaMemcpyAsync(hp->out_host + l0 * hp->out_layer_floats,
-                      hp->out_dev + l0 * hp->out_layer_floats,
-                      n * hp->out_layer_floats * sizeof(float), cudaMemcpyDeviceToHost,
-                      hp->copy) != cudaSuccess)
+  if (topk && cudaMemcpyAsync(hp->topk_host, hp->topk_dev,
+                              hp->num_layers * hp->topk_layer * sizeof(int32_t),
+                              cudaMemcpyDeviceToHost, hp->copy) != cudaSuccess)
     return HYLRA_ERR_CUDA;
-  if (hp->topk_host &&
-      cudaMemcpyAsync(hp->topk_host + l0 * hp->topk_layer, hp->topk_dev + l0 * hp->topk_layer,
-                      n * hp->topk_layer * sizeof(int32_t), cudaMemcpyDeviceToHost,
-                      hp->copy) != cudaSuccess)
-    return HYLRA_ERR_CUDA;
-  hp->copied = upto;
+  if (out) {
+    const int l0 = hp->copied, n = upto - l0;
+    if (cudaMemcpyAsync(hp->out_host + l0 * hp->out_layer_floats,
+                        hp->out_dev + l0 * hp->out_layer_floats,
+                        n * hp->out_layer_floats * sizeof(float), cudaMemcpyDeviceToHost,
+                        hp->copy) != cudaSuccess)
+      return HYLRA_ERR_CUDA;
+    hp->copied = upto;
+  }
   return HYLRA_OK;
 }
 
@@ -599,7 +605,9 @@ int host_pipe_before(void* ctx, int layer) {
 int host_pipe_after(void* ctx, int layer) {
   HostPipe* hp = static_cast<HostPipe*>(ctx);
   const int done = layer + 1;
-  if (done % OUT_CHUNK == 0 && done < hp->num_layers) return host_pipe_copy_out(hp, done);
+  const bool chunk = done % OUT_CHUNK == 0 && done < hp->num_layers;
+  if (chunk || layer == hp->last_reset)
+    return host_pipe_copy_out(hp, chunk ? done : hp->copied, layer == hp->last_reset);
   return HYLRA_OK;
 }
 
@@ -723,6 +731,8 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
   hp.topk_host = topk_host;
   hp.topk_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
   hp.num_layers = num_layers;
+  for (int l = 0; l < num_layers; ++l)
+    if (policy && policy[l]) hp.last_reset = l;
   std::vector<const void*> qp(num_layers);
   std::vector<float*> op(num_layers);
   for (int l = 0; l < num_layers; ++l) {
@@ -745,7 +755,7 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
   rc = run_step(shape, num_layers, policy, qp.data(), K, V, nullptr, seqlens, op.data(), topk_dev,
                 nullptr, nullptr, workspace, workspace_bytes, hp.main, &hooks);
   // the copy stream always rejoins the caller's stream (also after an error)
-  const int rc_out = rc ? rc : host_pipe_copy_out(&hp, num_layers);
+  const int rc_out = rc ? rc : host_pipe_copy_out(&hp, num_layers, false);
   if (cudaEventRecord(hp.ev_join, hp.copy) != cudaSuccess ||
       cudaStreamWaitEvent(hp.main, hp.ev_join, 0) != cudaSuccess)
     return HYLRA_ERR_CUDA;
