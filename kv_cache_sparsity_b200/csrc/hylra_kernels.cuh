@@ -1488,8 +1488,11 @@ constexpr int BAR_TOPK = 3;           // named barrier of the selection CTA
 // within one wave of SMs (few sequences and heads: each SM then loads a
 // smaller share of the partials), else one.  Heads [g0, g1) of output CTA
 // `part` (1..n).
+__host__ __device__ constexpr int merge_out_split(int r) {  // up to 4 CTAs, none empty
+  return (r + (r + 3) / 4 - 1) / ((r + 3) / 4);
+}
 __host__ __device__ constexpr int merge_out_ctas(int r, long long nbh, int sms) {
-  return nbh * (1 + (r < 4 ? r : 4)) <= sms ? (r < 4 ? r : 4) : 1;
+  return nbh * (1 + merge_out_split(r)) <= sms ? merge_out_split(r) : 1;
 }
 __device__ __forceinline__ void merge_out_heads(int r, int n, int part, int& g0, int& g1) {
   const int per = (r + n - 1) / n;
@@ -1515,7 +1518,10 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int r = p.r;
   int g0 = 0, g1 = 0;
-  if (part > 0) merge_out_heads(r, (int)gridDim.y - 1, part, g0, g1);
+  if (part > 0) {
+    merge_out_heads(r, (int)gridDim.y - 1, part, g0, g1);
+    if (g0 >= g1) return;  // no heads left for this part (not launched so)
+  }
   // The next layer's kernel may launch now: it reads nothing of this layer
   // and writes nothing before its own wait, which returns only after this
   // kernel, and so the streaming kernel, has completed.  Its CTAs take the

@@ -55,6 +55,9 @@ CASES = [
     W.custom("group1", seqlens=(2000,), num_q_heads=4, num_kv_heads=4, topk=6, seed=5),
     W.custom("group2", seqlens=(3000,), num_q_heads=8, num_kv_heads=4, topk=6, seed=6),
     W.custom("group8", seqlens=(2500,), num_q_heads=16, num_kv_heads=2, topk=6, seed=7),
+    W.custom("group5", batch=2, seqlens=(2200, 700), num_q_heads=10, num_kv_heads=2, topk=6,
+             seed=32),
+    W.custom("group7", seqlens=(1900,), num_q_heads=14, num_kv_heads=2, topk=5, seed=33),
     W.custom("iid_bf16", seqlens=(6000,), num_q_heads=8, num_kv_heads=2, topk=8,
              structure="iid", seed=8),
     W.custom("many_heads", batch=2, seqlens=(9000, 7000), num_q_heads=64, num_kv_heads=16,
@@ -130,8 +133,9 @@ def test_capacity_larger_than_longest_sequence():
     _full_and_check(w, kv_capacity=cap, inputs=(q, K2, V2))
 
 
-@pytest.mark.parametrize("w", CASES[:3] + [W.custom("fp32r", seqlens=(1500, 4000), batch=2,
-                                                    dtype="fp32", structure="iid", seed=14)],
+@pytest.mark.parametrize("w", CASES[:3] + [CASES[6], CASES[7]] +
+                         [W.custom("fp32r", seqlens=(1500, 4000), batch=2,
+                                   dtype="fp32", structure="iid", seed=14)],
                          ids=lambda w: w.name)
 def test_reuse_layer_matches_oracle(w):
     """Reuse with the indices the full kernel produced for another layer."""
