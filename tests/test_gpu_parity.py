@@ -272,13 +272,14 @@ def test_equal_scores_rank_by_block_index(nblocks):
     (2000, 32, "bf16", "iid"),
     (200, 30, "fp32", "iid"),
     (400, 32, "fp32", "salient"),
+    (300, 40, "fp32", "iid"),
     (513, 33, "bf16", "salient"),
     (1024, 64, "bf16", "iid"),
 ])
 def test_selection_paths_match_oracle(nblocks, topk, dtype, structure):
     """More blocks than selection threads: the merge tree of per-warp sorted
     lists for k' <= 32 (bf16: 256 threads, fp32: 128), the radix select
-    above; each with a ragged last block."""
+    above (both kernels); each with a ragged last block."""
     w = W.custom(f"sel_{nblocks}_{topk}_{dtype}", batch=1, seqlens=(128 * nblocks - 37,),
                  num_q_heads=8, num_kv_heads=2, topk=topk, dtype=dtype, structure=structure,
                  seed=60 + nblocks % 17)
