@@ -188,3 +188,21 @@ def test_pooled_profiling_steps(lib):
     assert H.similarity(np.concatenate([steps[0]] * 3, axis=1)).tobytes() == one.tobytes()
     mixed = np.concatenate(steps, axis=1)
     assert H.similarity(mixed).tobytes() == O.similarity_matrix(mixed).tobytes()
+
+
+def test_trace_build_compiles_and_exports_its_hooks(tmp_path):
+    """The documented trace build (-DHYLRA_TRACE: globaltimer events, plan and
+    late-start overrides) still compiles for sm_100a and exports its hooks."""
+    import ctypes
+    import subprocess
+    from kv_cache_sparsity_b200 import build as hbuild
+    out = tmp_path / "libhylra_trace.so"
+    cmd = [hbuild.nvcc_path(), "-DHYLRA_TRACE", "-gencode", hbuild.GENCODE, "-O3", "-std=c++17",
+           "-Xcompiler", "-fPIC", "-shared", "-I", hbuild.INCLUDE, "-I", hbuild.CSRC,
+           "-o", str(out)] + hbuild.SOURCES
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr[-3000:]
+    tl = ctypes.CDLL(str(out))
+    for name in ("hylra_trace_set", "hylra_plan_override", "hylra_late_override",
+                 "hylra_decode_step"):
+        assert hasattr(tl, name), name
