@@ -162,7 +162,7 @@ struct alignas(16) SmemCommon {
   float cf[NCOMB][GMAX];  // segment-end scale factors
   int prefix[HYLRA_MAX_BATCH + 1];  // units before sequence b (all heads)
   int hist[256];
-  int misc[8];  // 1: radix digit, 2: remaining, 3: list size, 4: abort
+  int misc[8];  // 1: radix digit, 2: remaining, 3: list size, 4: abort, 5: digit count
   int warp_sums[NT_MERGE / 32];
   StageMeta segs[MAX_SEGS];  // segments whose partial is stored but not yet ticketed
   int seg_last[MAX_SEGS];
@@ -550,11 +550,15 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     return;
   }
 
-  // Radix select of the kp-th largest key, 8 bits per pass.
+  // Radix select of the kp-th largest key, 8 bits per pass.  A pass whose
+  // chosen digit holds exactly the `remain` keys still wanted ends the
+  // search: every key whose bits above `shift` reach the prefix is taken.
   uint32_t prefix = 0;
   int remain = kp;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  int shift = 0;
+  bool whole = false;  // the last digit's keys are all taken
+  for (int pass = 0; pass < 4 && !whole; ++pass) {
+    shift = 24 - 8 * pass;
     for (int i = ct; i < 256; i += NT) c.hist[i] = 0;
     if (ct == 0) c.misc[3] = 0;
     named_bar_sync(BAR, NT);
@@ -591,6 +595,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
           if (acc + cnt[i] >= remain) {
             c.misc[1] = 255 - 8 * lane - i;
             c.misc[2] = remain - acc;
+            c.misc[5] = cnt[i];  // keys with this digit
             break;
           }
           acc += cnt[i];
@@ -600,15 +605,18 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     named_bar_sync(BAR, NT);
     prefix |= (uint32_t)c.misc[1] << shift;
     remain = c.misc[2];
+    whole = c.misc[5] == remain;
   }
-  const uint32_t tau = prefix;  // the kp-th largest score; take `remain` of its copies
+  // tau: the kp-th largest key's bits from `shift` up.  Keep every key whose
+  // bits from `shift` up exceed tau's, and of those equal to it all of them
+  // (whole digit) or the lowest-index `remain` (ties after the last pass).
+  const uint32_t tau = prefix >> shift;
 
-  // Keep every key above tau and the lowest-index `remain` keys equal to it.
   uint2* rlist = reinterpret_cast<uint2*>(keys + MAX_NB);
   const int per = (nb + NT - 1) / NT;
   const int b0 = min(nb, ct * per), b1 = min(nb, b0 + per);
   int eq = 0;
-  for (int beta = b0; beta < b1; ++beta) eq += keys[beta] == tau;
+  for (int beta = b0; beta < b1; ++beta) eq += (keys[beta] >> shift) == tau;
   int incl = eq;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -623,9 +631,9 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     if (w < wid) before += c.warp_sums[w];
   for (int beta = b0; beta < b1; ++beta) {
     const uint32_t key = keys[beta];
-    bool sel = key > tau;
-    if (key == tau) {
-      sel = before < remain;
+    bool sel = (key >> shift) > tau;
+    if ((key >> shift) == tau) {
+      sel = whole || before < remain;
       ++before;
     }
     if (sel) {
