@@ -2091,6 +2091,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       uint8_t* dst = stages + (size_t)s * STAGE_BYTES + (lane < 16 ? 0 : 2 * BOX_BYTES) +
                      (c >> 3) * BOX_BYTES + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
       if (!*abort_flag) *reinterpret_cast<uint4*>(dst) = __ldcg(reinterpret_cast<const uint4*>(src));
+      // the stage may be released and refilled by TMA (async proxy) later:
+      // order this generic-proxy write before any such refill
+      fence_proxy_async_smem();
       __syncwarp();
     };
     // first phase of the cluster barrier (every CTA has started), needed

@@ -161,6 +161,28 @@ def full_layer(q, K, V, n: int, k: int):
     return out, S32, topk
 
 
+def layer_topk(q, K, n: int, k: int):
+    """The ranking half of ``full_layer``: fp32 block scores and top-k of a
+    reset layer without its attention output (no V is read).  Used for
+    profiling runs, where only the index sets feed the overlap matrix
+    (HyLRA summary §2.2, "Similarity Matrix Construction").
+
+    Returns (S32 [Hkv, NB] float32, topk [Hkv, k] int32), the same values as
+    ``full_layer(q, K, V, n, k)[1:]``.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    Hkv = K.shape[0]
+    r = Hq // Hkv
+    probs = np.zeros((Hq, n), dtype=np.float64)
+    if n > 0:
+        for g in range(Hq):
+            probs[g] = attention_probs(q[g], K[g // r, :n])
+    S32 = round_scores_fp32(block_scores(probs, Hkv))
+    topk = np.stack([topk_blocks(S32[h], k) for h in range(Hkv)])
+    return S32, topk
+
+
 def topk_gap(S32_h: np.ndarray, k: int) -> float:
     """Smallest relative gap between consecutive ranks 1..k'+1 of one head.
 

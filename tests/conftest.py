@@ -8,3 +8,13 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Top-k gap certificates and near-tie swap counts of the parity tests."""
+    lib = sys.modules.get("hylra_testlib")
+    lines = lib.certificate_lines() if lib is not None else []
+    if lines:
+        terminalreporter.write_sep("-", "top-k gap certificates (oracle fp32 scores)")
+        for line in lines:
+            terminalreporter.write_line(line)

@@ -137,3 +137,54 @@ def check_topk(got: np.ndarray, ref: np.ndarray, S32: np.ndarray, what=""):
 
 def min_gap(S32_rows, k) -> float:
     return min((O.topk_gap(r, k) for r in S32_rows), default=math.inf)
+
+
+# Gap certificates of the top-k checks, per configuration, printed at the end
+# of the session (conftest.pytest_terminal_summary): for each index set the
+# oracle's smallest relative gap between consecutive fp32 scores of ranks
+# 1..k'+1 (oracle.topk_gap).  A set whose gap is below NEAR_TIE_REL is a
+# near tie: the kernel's fp32 sums (another summation order) may swap those
+# ranks, so such a set is reported as "near-tie, unpinned".
+CERTIFICATES: dict = {}
+
+
+def check_topk_certified(config: str, got, ref, S32_h, k: int, what=""):
+    """check_topk plus the set's gap certificate, recorded under `config`.
+    A swap is accepted only inside a near tie; returns the swap count."""
+    swaps = check_topk(got, ref, S32_h, what)
+    gap = O.topk_gap(S32_h, k)
+    assert swaps == 0 or gap < NEAR_TIE_REL, f"{what}: swap with certificate {gap}"
+    c = CERTIFICATES.setdefault(config, {"sets": 0, "min_gap": math.inf, "near_ties": 0,
+                                         "swaps": 0})
+    c["sets"] += 1
+    c["min_gap"] = min(c["min_gap"], gap)
+    c["near_ties"] += int(gap < NEAR_TIE_REL)
+    c["swaps"] += swaps
+    return swaps
+
+
+def certificate_lines():
+    out = []
+    for name in sorted(CERTIFICATES):
+        c = CERTIFICATES[name]
+        state = ("near-tie, unpinned" if c["near_ties"] else "pinned")
+        out.append(f"{name}: {c['sets']} index sets, min relative gap {c['min_gap']:.3g}, "
+                   f"{c['near_ties']} near-tie sets, {c['swaps']} swaps ({state})")
+    return out
+
+
+class SequenceLayers:
+    """The layers of one sequence b as the fp64 arrays oracle.decode_step
+    takes (q [1, Hq, d], K and V [1, Hkv, n_b, d]), converted when a layer is
+    read, so that only one layer is held in host memory at a time."""
+
+    def __init__(self, w: W.Workload, layers, b: int):
+        self.w, self.layers, self.b = w, layers, b
+
+    def __len__(self):
+        return len(self.layers)
+
+    def __getitem__(self, l):
+        q, K, V = self.layers[l]
+        return (q[self.b:self.b + 1].double().cpu().numpy(), seq_arrays(self.w, K, self.b)[None],
+                seq_arrays(self.w, V, self.b)[None])

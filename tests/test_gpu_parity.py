@@ -42,7 +42,8 @@ def _full_and_check(w, layer=0, kv_capacity=None, inputs=None):
         o_ref, S32, tk_ref = T.oracle_full(w, q, K, V, b)
         T.check_out(out[b], o_ref, w.dtype, f"{w.name} b={b}")
         for h in range(w.num_kv_heads):
-            swaps += T.check_topk(tk[b, h], tk_ref[h], S32[h], f"{w.name} b={b} h={h}")
+            swaps += T.check_topk_certified(w.name, tk[b, h], tk_ref[h], S32[h], w.topk,
+                                            f"{w.name} b={b} h={h}")
     return run, (q, K, V), out, tk, swaps
 
 
@@ -90,7 +91,8 @@ def test_tiny_fp32_config_step_matches_oracle():
         if w.policy[l]:
             _, S32, _ = T.oracle_full(w, *layers[l], 0)
             for h in range(w.num_kv_heads):
-                assert T.check_topk(tk[l, 0, h], tk_ref[l][0, h], S32[h], f"tiny l={l}") == 0
+                assert T.check_topk_certified("tiny", tk[l, 0, h], tk_ref[l][0, h], S32[h], w.topk,
+                                              f"tiny l={l}") == 0
 
 
 def test_fp32_ragged_packed():
@@ -184,6 +186,37 @@ def test_reuse_many_blocks_per_cta():
     assert run.status() == 0
     ref = T.oracle_reuse(w, q1, K1, V1, 0, tk.cpu().numpy()[0])
     T.check_out(out[0], ref, "bf16", "reuse_k64")
+
+
+def test_step_reuse_refills_the_stage_of_an_early_newest_block():
+    """Inside a step a reuse layer rereads the newest cache row after its
+    wait and writes it into the staged block.  Here the newest block ranks
+    first (so it sits in the first stage of the first CTA) and every CTA has
+    more blocks than stages, so that stage is refilled by TMA after the row
+    was rewritten: the refill must land after the rewrite."""
+    n = 128 * 100 - 37  # partial newest block
+    w = W.custom("newest_first", batch=1, layers=2, seqlens=(n,), num_q_heads=8,
+                 num_kv_heads=2, topk=64, seed=41)
+    q0, K0, V0 = W.layer_inputs(w, 0, device="cpu")
+    u = W.structure(w).u  # [B, Hkv, d] salient directions the queries follow
+    last = (n - 1) // 128 * 128
+    K0[0, :, last:n] = (K0[0, :, last:n].float() + 9.0 * u[0][:, None, :]).to(K0.dtype)
+    layers = [(q0.cuda(), K0.cuda(), V0.cuda()), _layer(w, 1)]
+    run = T.Runner(w)
+    policy = (1, 0)
+    topk = torch.full((2, 1, 2, 64), -7, dtype=torch.int32, device="cuda")
+    outs = [run.new_out() for _ in range(2)]
+    for _ in range(3):
+        H.decode_step(run.shape, policy, [l[0] for l in layers], [l[1] for l in layers],
+                      [l[2] for l in layers], run.seqlens, outs, topk, run.ws)
+        assert run.status() == 0
+        tk = topk.cpu().numpy()
+        assert np.all(tk[0, 0, :, 0] == (n - 1) // 128), "newest block not ranked first"
+        np_layers = [tuple(t.double().cpu().numpy() for t in l) for l in layers]
+        o_ref, tk_ref = O.decode_step(policy, np_layers, w.seqlens, w.topk)
+        assert np.array_equal(tk[0], tk_ref[0])
+        for l in range(2):
+            T.check_out(outs[l].cpu().numpy(), o_ref[l], "bf16", f"newest-first layer {l}")
 
 
 def test_reuse_skips_minus_one_and_flags_bad_indices():

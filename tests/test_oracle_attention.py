@@ -175,3 +175,32 @@ def test_topk_gap_certificate():
     S = np.array([4.0, 3.0, 2.0, 1.0], dtype=np.float32)
     assert O.topk_gap(S, 2) == pytest.approx(0.25)   # min((4-3)/4, (3-2)/3)
     assert O.topk_gap(np.array([1.0], dtype=np.float32), 4) == math.inf
+
+
+# ------------------------------------------------------ ranking without output
+
+@pytest.mark.parametrize("n,hq,hkv", [(0, 4, 2), (1, 4, 1), (300, 8, 2), (1000, 8, 8),
+                                      (2049, 16, 4)])
+def test_layer_topk_equals_full_layer_ranking(n, hq, hkv):
+    """layer_topk (no V read) gives exactly full_layer's scores and indices."""
+    rng = np.random.default_rng(n + 7 * hq)
+    q = rng.standard_normal((hq, 64))
+    K = rng.standard_normal((hkv, max(n, 1), 64))
+    V = rng.standard_normal((hkv, max(n, 1), 64))
+    _, S_full, tk_full = O.full_layer(q, K, V, n, 5)
+    S, tk = O.layer_topk(q, K, n, 5)
+    assert S.dtype == np.float32 and S.tobytes() == S_full.tobytes()
+    assert np.array_equal(tk, tk_full)
+
+
+def test_layer_topk_dominant_keys_rank_their_blocks_first():
+    """One key per chosen block aligned with the query dominates: those
+    blocks come first, in decreasing order of their logit bump."""
+    d, n = 32, 128 * 10
+    q = np.zeros((2, d))
+    q[:, 0] = math.sqrt(d)
+    K = np.zeros((1, n, d))
+    for beta, bump in ((7, 30.0), (2, 25.0), (9, 20.0)):
+        K[0, beta * 128 + 5, 0] = bump   # logit = bump on that one token
+    _, tk = O.layer_topk(q, K, n, 3)
+    assert list(tk[0]) == [7, 2, 9]
