@@ -302,6 +302,40 @@ def similarity_matrix(topk: np.ndarray) -> np.ndarray:
     return M
 
 
+def overlap_counts(topk: np.ndarray):
+    """The two integer sums behind ``similarity_matrix``.
+
+    topk: int array [L, S, k] as for similarity_matrix.  Returns
+    (inter [L, L] int64, total [L] int64): inter[t][s] = sum_u |I_s[u] & I_t[u]|
+    for s <= t (0 above the diagonal), total[t] = sum_u |I_t[u]|.  Both are
+    sums over the index sets u, so the counts of disjoint groups of sets (for
+    example the KV heads held by different GPUs) add up to the counts of all
+    of them.
+    """
+    topk = np.asarray(topk)
+    L, S = topk.shape[0], topk.shape[1]
+    sets = [[frozenset(int(x) for x in topk[l, u] if x >= 0) for u in range(S)]
+            for l in range(L)]
+    inter = np.zeros((L, L), dtype=np.int64)
+    total = np.zeros(L, dtype=np.int64)
+    for t in range(L):
+        total[t] = sum(len(sets[t][u]) for u in range(S))
+        for s in range(t + 1):
+            inter[t, s] = sum(len(sets[s][u] & sets[t][u]) for u in range(S))
+    return inter, total
+
+
+def similarity_from_counts(inter: np.ndarray, total: np.ndarray) -> np.ndarray:
+    """M[t][s] = inter[t][s] / total[t] (s <= t; 0 where total[t] is 0)."""
+    inter = np.asarray(inter)
+    L = inter.shape[0]
+    M = np.zeros((L, L), dtype=np.float64)
+    for t in range(L):
+        for s in range(t + 1):
+            M[t, s] = int(inter[t, s]) / int(total[t]) if total[t] else 0.0
+    return M
+
+
 # ---------------------------------------------------------------------------
 # Policy search (HyLRA summary §2.2, "Dynamic Programming")
 # ---------------------------------------------------------------------------

@@ -102,3 +102,37 @@ def test_static_policy_closed_form(L, period):
     assert len(pol) == L and pol[0] == O.RESET
     assert R == -(-L // period) == sum(pol)
     assert [i for i, x in enumerate(pol) if x == O.RESET] == list(range(0, L, period))
+
+
+def test_overlap_counts_hand_worked():
+    g = _load("similarity_3layer.json")
+    inter, total = O.overlap_counts(np.array(g["topk"]))
+    assert inter.tolist() == g["inter"] and total.tolist() == g["total"]
+    assert O.similarity_from_counts(inter, total).tolist() == g["M"]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_overlap_counts_add_over_disjoint_groups_of_sets(seed):
+    """Counts of two disjoint groups of index sets add up to the counts of
+    all of them, and the ratio of the sums is the pooled matrix exactly."""
+    rng = np.random.default_rng(seed)
+    L, S, k, nb = 6, 10, 5, 12
+    topk = np.full((L, S, k), -1, dtype=np.int32)
+    for l in range(L):
+        for u in range(S):
+            m = int(rng.integers(0, k + 1))
+            topk[l, u, :m] = rng.choice(nb, size=m, replace=False)
+    i_all, t_all = O.overlap_counts(topk)
+    cut = int(rng.integers(1, S))
+    i_a, t_a = O.overlap_counts(topk[:, :cut])
+    i_b, t_b = O.overlap_counts(topk[:, cut:])
+    assert np.array_equal(i_a + i_b, i_all) and np.array_equal(t_a + t_b, t_all)
+    M = O.similarity_from_counts(i_a + i_b, t_a + t_b)
+    assert M.tobytes() == O.similarity_matrix(topk).tobytes()
+    # brute force on the definition: one set at a time
+    for t in range(L):
+        assert t_all[t] == sum(int((topk[t, u] >= 0).sum()) for u in range(S))
+        for s in range(t + 1):
+            brute = sum(len(set(topk[s, u][topk[s, u] >= 0]) & set(topk[t, u][topk[t, u] >= 0]))
+                        for u in range(S))
+            assert i_all[t, s] == brute
