@@ -7,14 +7,26 @@ a reset layer running full attention + block scoring + top-k, a reuse layer
 attending over the blocks the most recent reset layer selected, under the
 policy the DP derives from a profiling run (all layers full) of the same
 synthetic workload.  Inputs are resident in HBM before timing starts; each
-step streams more bytes than the 126 MB L2 holds.
+step streams more bytes than the 126 MB L2 holds.  The default workload is
+the largest one that fits one GPU (ragged16: 16 sequences of 8K-128K tokens,
+all 32 layer caches resident).
 
-value      = device time per hybrid decode step (us), max over ranks
-e2e        = the same step through the C-ABI host-buffer entry point
-             (q copied host->device, outputs device->host, inside the timing)
-roofline   = the full (reset-layer) kernel: K+V bytes of one layer per launch
-             over its average duration in the all-full step
-cpu_baseline / --impl reference = the fp64 oracle on the host cores
+With N GPUs (torchrun), rank r holds the KV heads shard(Hkv, r, N) of every
+sequence: one fixed workload split N ways ("scaling": "strong"), no
+collective in the step; the profiled overlap matrix is pooled exactly over
+the ranks (integer counts, one all-reduce), so every rank runs the policy a
+single GPU derives.
+
+value        = device time per hybrid decode step (us), max over ranks
+e2e          = the same step through the C-ABI host-buffer entry point
+               (q copied host->device, outputs device->host, inside the timing)
+roofline     = the reset layer (streaming + merge kernels): K+V bytes of one
+               layer on this GPU over its average time in the all-reset step
+reuse_layer  = a reuse layer's K+V bytes over its average time in a step of one
+               reset layer followed by reuse layers
+cpu_baseline / --impl reference = the fp64 oracle, single-threaded on the host,
+               on a bounded sample (one reset and one reuse layer of one KV head
+               of every sequence), scaled to a whole step
 """
 
 from __future__ import annotations
@@ -149,28 +161,31 @@ def _num(x):
 # ----------------------------------------------------------------- our arm
 
 class Model:
-    """All layers of one synthetic workload resident on this GPU."""
+    """All layers of one synthetic workload resident on this GPU: the KV
+    heads ``heads`` of every sequence (all of them on one GPU)."""
 
-    def __init__(self, w: W.Workload, H, resident_layers: int):
-        self.w, self.H = w, H
+    def __init__(self, w: W.Workload, H, resident_layers: int, heads: range):
+        self.w, self.H, self.heads = w, H, heads
         dev = "cuda"
+        self.nkv = len(heads)
+        self.nq = self.nkv * w.group
         self.seqlens = torch.tensor(w.seqlens, dtype=torch.int32, device=dev)
         self.offs = (torch.tensor(W.seq_offsets(w)[:-1], dtype=torch.int64, device=dev)
                      if w.packed else None)
         dtype = H.BF16 if w.dtype == "bf16" else H.FP32
         if w.packed:
-            self.shape = H.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.topk,
-                                      w.max_seqlen, dtype=dtype, total_tokens=w.total_tokens,
+            self.shape = H.make_shape(w.batch, self.nq, self.nkv, w.topk, w.max_seqlen,
+                                      dtype=dtype, total_tokens=w.total_tokens,
                                       seq_offsets=self.offs)
         else:
-            self.shape = H.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.topk,
-                                      w.max_seqlen, dtype=dtype, kv_capacity=w.max_seqlen)
+            self.shape = H.make_shape(w.batch, self.nq, self.nkv, w.topk, w.max_seqlen,
+                                      dtype=dtype, kv_capacity=w.max_seqlen)
         self.ws = torch.empty(H.workspace_bytes(self.shape), dtype=torch.uint8, device=dev)
         H.workspace_init(self.ws)
         self.resident = resident_layers
         self.q, self.K, self.V = [], [], []
         for l in range(w.layers):
-            q, K, V = W.layer_inputs(w, l, device=dev)
+            q, K, V = W.layer_inputs(w, l, device=dev, heads=heads)
             self.q.append(q)
             if l < resident_layers:
                 self.K.append(K)
@@ -180,14 +195,23 @@ class Model:
         torch.cuda.synchronize()
         self.Ks = [self.K[l % resident_layers] for l in range(w.layers)]
         self.Vs = [self.V[l % resident_layers] for l in range(w.layers)]
-        self.outs = [torch.empty(w.batch, w.num_q_heads, w.head_dim, device=dev)
+        self.outs = [torch.empty(w.batch, self.nq, w.head_dim, device=dev)
                      for _ in range(w.layers)]
-        self.topk = torch.full((w.layers, w.batch, w.num_kv_heads, w.topk), -1,
+        self.topk = torch.full((w.layers, w.batch, self.nkv, w.topk), -1,
                                dtype=torch.int32, device=dev)
 
+    def full_bytes(self) -> int:
+        """K+V bytes of one reset layer on this GPU."""
+        return self.w.kv_bytes_per_layer() * self.nkv // self.w.num_kv_heads
+
+    def reuse_bytes(self) -> int:
+        """K+V bytes one reuse layer touches on this GPU."""
+        return self.w.kv_bytes_reuse_layer() * self.nkv // self.w.num_kv_heads
+
     def step(self, policy, stream=None):
-        self.H.decode_step(self.shape, policy, self.q, self.Ks, self.Vs, self.seqlens,
-                           self.outs, self.topk, self.ws, stream=stream)
+        L = len(policy)
+        self.H.decode_step(self.shape, policy, self.q[:L], self.Ks[:L], self.Vs[:L],
+                           self.seqlens, self.outs[:L], self.topk[:L], self.ws, stream=stream)
 
     def graph(self, policy):
         s = torch.cuda.Stream()
@@ -227,14 +251,34 @@ def policy_rule(args, w) -> str:
     return f"dp theta={theta:g} profile_steps={max(1, args.profile_steps)}"
 
 
+def step_bytes(w: W.Workload, policy) -> int:
+    """K+V bytes one hybrid step touches over the whole workload."""
+    R = sum(policy)
+    return R * w.kv_bytes_per_layer() + (w.layers - R) * w.kv_bytes_reuse_layer()
+
+
+def config_of(w: W.Workload, policy, args, world: int) -> dict:
+    """The workload as both arms name it (the same keys and values)."""
+    return {
+        "workload": workload_desc(w),
+        "policy": "".join("R" if x else "U" for x in policy),
+        "policy_rule": policy_rule(args, w),
+        "resets": int(sum(policy)),
+        "l2": "inputs larger than L2: a step streams %.2f GB" % (step_bytes(w, policy) / 1e9),
+        "parallelism": f"kv-head shards x{world}",
+    }
+
+
 def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int = 1):
     """The step's reset/reuse policy.
 
     dp: profiling run(s) with every layer full -> overlap matrix -> DP policy
     (HyLRA summary §2.2).  With profile_steps P > 1 the index sets of P decode
-    steps (fresh queries, same cache) are pooled into one matrix.  A workload
-    with a fixed policy keeps it.  jump3: a reset every third layer (the
-    static baseline of §4)."""
+    steps (fresh queries, same cache) are pooled into one matrix.  Over
+    several ranks the matrix is pooled from every rank's index sets (integer
+    counts summed over ranks), so all ranks derive the single-GPU policy.  A
+    workload with a fixed policy keeps it.  jump3: a reset every third layer
+    (the static baseline of §4)."""
     w = m.w
     if rule == "jump3":
         pol, _ = H.static_policy(w.layers, 3)
@@ -246,12 +290,12 @@ def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int 
     q0 = list(m.q)
     for p in range(max(1, profile_steps)):
         if p > 0:
-            m.q = [W.step_query(w, l, p, device="cuda") for l in range(w.layers)]
+            m.q = [W.step_query(w, l, p, device="cuda", heads=m.heads) for l in range(w.layers)]
         m.step(allfull)
         torch.cuda.synchronize()
-        sets.append(m.topk.cpu().numpy().reshape(w.layers, w.batch * w.num_kv_heads, w.topk))
+        sets.append(m.topk.cpu().numpy().reshape(w.layers, w.batch * m.nkv, w.topk))
     m.q = q0
-    M = H.similarity(np.concatenate(sets, axis=1))
+    M = D.pooled_similarity(H, np.concatenate(sets, axis=1), device="cuda")
     pol, R, S = H.dp_policy(M, w.theta if theta is None else theta)
     return pol, M
 
@@ -293,9 +337,9 @@ def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
     w = m.w
     q_host = torch.stack([q.cpu() for q in m.q]).pin_memory()
     q_dev = torch.empty_like(q_host, device="cuda")
-    out_dev = torch.empty(w.layers, w.batch, w.num_q_heads, w.head_dim, device="cuda")
+    out_dev = torch.empty(w.layers, w.batch, m.nq, w.head_dim, device="cuda")
     out_host = torch.empty(out_dev.shape, dtype=torch.float32).pin_memory()
-    tk_dev = torch.full((w.layers, w.batch, w.num_kv_heads, w.topk), -1, dtype=torch.int32,
+    tk_dev = torch.full((w.layers, w.batch, m.nkv, w.topk), -1, dtype=torch.int32,
                         device="cuda")
     tk_host = torch.empty(tk_dev.shape, dtype=torch.int32).pin_memory()
 
@@ -315,22 +359,9 @@ def e2e_step_time(m: Model, H, policy, steps, warmup, dist_on):
     with torch.cuda.graph(g, stream=s):
         call(stream=torch.cuda.current_stream())
 
-    def one():
-        g.replay()
-
     for _ in range(warmup):
-        one()
-    D.barrier()
-    torch.cuda.synchronize()
-    st = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(steps):
-        one()
-    e1.record(st)
-    torch.cuda.synchronize()
-    D.barrier()
-    ms = e0.elapsed_time(e1) / steps
+        g.replay()
+    ms = timed_replays(g, steps, dist_on)
     h2d = q_host.numel() * q_host.element_size()
     d2h = out_host.numel() * 4 + tk_host.numel() * 4
     del g
@@ -345,7 +376,6 @@ def offload_measure(m: Model, H, policy, steps, warmup, dist_on):
     w = m.w
     offloaded = tuple(0 if x else 1 for x in policy)
     Ko, Vo = [], []
-    host_bytes = 0
     for l in range(w.layers):
         if offloaded[l]:
             Ko.append(m.Ks[l].cpu().pin_memory())
@@ -372,8 +402,7 @@ def offload_measure(m: Model, H, policy, steps, warmup, dist_on):
     ms = timed_replays(g, steps, dist_on)
     # bytes that cross the link per step: k' blocks of K and V per (b, h) per
     # offloaded layer
-    per_layer = w.kv_bytes_reuse_layer()
-    host_bytes = per_layer * sum(offloaded)
+    host_bytes = m.reuse_bytes() * sum(offloaded)
     # a plain pinned-host-to-device copy of those bytes, for the link's rate
     src = torch.empty(host_bytes, dtype=torch.uint8).pin_memory()
     dst = torch.empty(host_bytes, dtype=torch.uint8, device="cuda")
@@ -392,48 +421,55 @@ def offload_measure(m: Model, H, policy, steps, warmup, dist_on):
             "host_link_bytes_per_step": int(host_bytes),
             "host_link_gbs": round(host_bytes / (ms * 1e-3) / 1e9, 1),
             "plain_copy_gbs": round(host_bytes / (copy_ms * 1e-3) / 1e9, 1),
-            "device_cache_bytes_moved_to_host": int(w.kv_bytes_per_layer() * sum(offloaded))}
+            "device_cache_bytes_moved_to_host": int(m.full_bytes() * sum(offloaded))}
 
 
-def oracle_sample(w: W.Workload, m: Model, policy, heads=(0,), reps=1):
-    """Time the fp64 oracle on a bounded sample of one decode step: all
-    layers under ``policy`` for the KV heads ``heads`` of every sequence.
-    Returns (seconds per full step scaled to all heads, sample text, threads)."""
-    from oracle import hylra_oracle as O
+def oracle_sample_data(w: W.Workload, reset_layer, reuse_layer, head=0):
+    """The inputs of the oracle's bounded sample, as fp64 host arrays: KV
+    head `head` of every sequence (its query rows, keys and values) in one
+    reset layer and one reuse layer.  reset_layer / reuse_layer: (q, K, V)
+    tensors (any device) holding at least KV head `head`; reuse_layer may be
+    None (a policy without reuse layers)."""
     r = w.group
-    data = []
-    for l in range(w.layers):
-        q = m.q[l].double().cpu().numpy()
-        K, V = m.Ks[l], m.Vs[l]
-        per_b = []
+
+    def prep(layer):
+        q, K, V = layer
+        out = []
         for b in range(w.batch):
-            kb = W.per_sequence(w, K, b)
-            vb = W.per_sequence(w, V, b)
-            per_b.append((q[b][[g for h in heads for g in range(h * r, (h + 1) * r)]],
-                          kb[list(heads)].double().cpu().numpy(),
-                          vb[list(heads)].double().cpu().numpy()))
-        data.append(per_b)
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        current = [None] * w.batch
-        for l in range(w.layers):
-            for b in range(w.batch):
-                qb, kb, vb = data[l][b]
-                n = w.seqlens[b]
-                if policy[l]:
-                    _, _, current[b] = O.full_layer(qb, kb, vb, n, w.topk)
-                else:
-                    O.reuse_attention(qb, kb, vb, n, current[b])
-    dt = (time.perf_counter() - t0) / reps
-    scale = w.num_kv_heads / len(heads)
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    sample = (f"{reps} decode step(s) of all {w.layers} layers under the bench policy for "
-              f"KV head(s) {list(heads)} of {w.num_kv_heads} of every sequence, scaled x{scale:g}")
-    return dt * scale, sample, threads
+            out.append((q[b, head * r:(head + 1) * r].double().cpu().numpy(),
+                        W.per_sequence(w, K, b)[head:head + 1].double().cpu().numpy(),
+                        W.per_sequence(w, V, b)[head:head + 1].double().cpu().numpy()))
+        return out
+
+    return head, prep(reset_layer), (prep(reuse_layer) if reuse_layer is not None else None)
+
+
+def oracle_sample(w: W.Workload, data, policy):
+    """Time the fp64 oracle, single-threaded, on a bounded sample of one
+    decode step (oracle_sample_data): the sampled KV head of every sequence
+    through one reset layer (full attention, block scores, top-k) and one
+    reuse layer (attention over the blocks that reset layer selected).  A
+    step is R reset and L - R reuse layers over all Hkv heads, so the two
+    times scale to it exactly (the oracle's cost per layer does not depend on
+    which layer it is).  Returns (seconds per step, sample text, threads)."""
+    from oracle import hylra_oracle as O
+    from threadpoolctl import threadpool_limits
+    head, d_reset, d_reuse = data
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        idx = [O.full_layer(qb, kb, vb, w.seqlens[b], w.topk)[2]
+               for b, (qb, kb, vb) in enumerate(d_reset)]
+        t1 = time.perf_counter()
+        if d_reuse is not None:
+            for b, (qb, kb, vb) in enumerate(d_reuse):
+                O.reuse_attention(qb, kb, vb, w.seqlens[b], idx[b])
+        t2 = time.perf_counter()
+    R = sum(policy)
+    sec = w.num_kv_heads * (R * (t1 - t0) + (w.layers - R) * (t2 - t1))
+    sample = (f"KV head {head} of every sequence through one reset and one reuse layer, "
+              f"single-threaded; scaled to {w.num_kv_heads} KV heads x ({R} reset + "
+              f"{w.layers - R} reuse layers)")
+    return sec, sample, 1
 
 
 def run_ours(args, rank, world, dist_on):
@@ -441,20 +477,27 @@ def run_ours(args, rank, world, dist_on):
     hbuild.build()
     H.load()
     w = W.config(args.config)
+    heads = D.shard(w.num_kv_heads, rank, world)
+    if len(heads) == 0:
+        raise SystemExit(f"{world} ranks for {w.num_kv_heads} KV heads: a rank would hold none")
     free = torch.cuda.mem_get_info()[0]
-    per_layer = w.kv_bytes_per_layer()  # K and V bytes of one layer
+    per_layer = w.kv_bytes_per_layer() * len(heads) // w.num_kv_heads  # K and V on this GPU
     resident = w.layers
     if per_layer * w.layers > free * 0.85:
         resident = max(1, int(free * 0.85 // per_layer))
-    m = Model(w, H, resident)
+    m = Model(w, H, resident, heads)
     policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps)
-    allfull = (1,) * w.layers
+    L = w.layers
+    allfull = (1,) * L
+    one_then_reuse = (1,) + (0,) * (L - 1)
     R = sum(policy)
     g_h = m.graph(policy)
     g_f = m.graph(allfull)
+    g_u = m.graph(one_then_reuse)
+    g_1 = m.graph((1,))
     for _ in range(args.warmup):
-        g_h.replay()
-        g_f.replay()
+        for g in (g_h, g_f, g_u, g_1):
+            g.replay()
     torch.cuda.synchronize()
     assert H.read_status(m.ws) == 0, "device status set during warm-up"
 
@@ -465,15 +508,19 @@ def run_ours(args, rank, world, dist_on):
     clk.start()
     ms_h = timed_replays(g_h, args.steps, dist_on)
     ms_f = timed_replays(g_f, args.steps, dist_on)
+    ms_u = timed_replays(g_u, args.steps, dist_on)
+    ms_1 = timed_replays(g_1, args.steps, dist_on)
     # keep the GPU busy long enough for the sampler when the timed region is short
     fill = 0.0 if args.no_clock_fill else 0.6
-    t_end = time.time() + max(0.0, fill - (ms_h + ms_f) * args.steps / 1000.0)
+    t_end = time.time() + max(0.0, fill - (ms_h + ms_f + ms_u + ms_1) * args.steps / 1000.0)
     while time.time() < t_end:
         g_h.replay()
         torch.cuda.synchronize()
     clocks = clk.stop()
     ms_h = max_over_ranks(ms_h, dist_on)
     ms_f = max_over_ranks(ms_f, dist_on)
+    ms_u = max_over_ranks(ms_u, dist_on)
+    ms_1 = max_over_ranks(ms_1, dist_on)
     status = H.read_status(m.ws)
 
     e2e_ms, h2d, d2h = e2e_step_time(m, H, policy, max(3, args.steps // 4), args.warmup,
@@ -482,18 +529,25 @@ def run_ours(args, rank, world, dist_on):
     g_launches = g_h.kernel_nodes
     errs = output_error_vs_full(m, g_h, g_f)
     reuse_errs = [e for e, x in zip(errs, policy) if not x] or [0.0]
-    del g_h, g_f
+    del g_h, g_f, g_u, g_1
     offload = (offload_measure(m, H, policy, max(3, args.steps // 4), args.warmup, dist_on)
                if args.offload else None)
 
-    full_b = w.kv_bytes_per_layer()
-    reuse_b = w.kv_bytes_reuse_layer()
-    step_bytes = R * full_b + (w.layers - R) * reuse_b
-    us_h = ms_h * 1000.0
-    kv_gbs = step_bytes / (ms_h * 1e-3) / 1e9
-    full_launch_us = ms_f * 1000.0 / w.layers
-    achieved = full_b / (full_launch_us * 1e-6) / 1e9
     peak, peak_kind = measured_hbm_peak()
+    job_bytes = step_bytes(w, policy)
+    us_h = ms_h * 1000.0
+    kv_gbs = job_bytes / (ms_h * 1e-3) / 1e9
+    full_b, reuse_b = m.full_bytes(), m.reuse_bytes()
+    reset_us = ms_f * 1000.0 / L
+    reuse_us = (ms_u - ms_1) * 1000.0 / max(1, L - 1)
+    achieved = full_b / (reset_us * 1e-6) / 1e9
+
+    def layer_rate(nbytes, us):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": round(us, 3), "kv_bytes": int(nbytes), "gbs": round(gbs, 1),
+                "frac_of_measured": round(gbs / peak, 4),
+                "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
+
     line = {
         "metric": METRIC,
         "value": round(us_h, 3),
@@ -503,28 +557,26 @@ def run_ours(args, rank, world, dist_on):
         "warmup": args.warmup,
         "ms_per_step": round(ms_h, 6),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong",
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
-        "config": {
-            "workload": workload_desc(w),
-            "policy": "".join("R" if x else "U" for x in policy),
-            "policy_rule": policy_rule(args, w),
-            "resets": R,
-            "resident_layer_caches": m.resident,
-            "l2": "inputs larger than L2: a step streams %.2f GB" % (step_bytes / 1e9),
-            "replicas": "each rank runs its own copy of the workload" if world > 1 else None,
-        },
-        "kv_bytes_per_step": step_bytes,
+        "config": config_of(w, policy, args, world),
+        "kv_heads_per_gpu": len(heads),
+        "resident_layer_caches": m.resident,
+        "kv_bytes_per_step": job_bytes,
         "kv_gbs": round(kv_gbs, 1),
         "kv_frac_of_8tbs": round(kv_gbs / NOMINAL_HBM_GBS, 4),
         "full_us_per_step": round(ms_f * 1000.0, 3),
         "speedup_vs_full": round(ms_f / ms_h, 4),
-        "sequences_per_s_all_ranks": round(world * w.batch / (ms_h * 1e-3), 1),
+        "sequences_per_s": round(w.batch / (ms_h * 1e-3), 1),
+        "reset_layer": layer_rate(full_b, reset_us),
+        "reuse_layer": dict(layer_rate(reuse_b, reuse_us),
+                            how="(one reset + %d reuse layers) - (one reset layer), per reuse "
+                                "layer, graph-replayed" % (L - 1)),
         "roofline": {
             "bound": "hbm",
-            "kernel": "decode_bf16_kernel<full> (reset layer)",
+            "kernel": "reset layer (streaming + merge kernels, the step's dominant work)",
             "achieved": round(achieved, 1),
             "peak": peak,
             "peak_kind": peak_kind,
@@ -532,7 +584,7 @@ def run_ours(args, rank, world, dist_on):
             "frac": round(achieved / peak, 4),
             "traffic": ncu_traffic("full_kernel", w.name),
             "algorithmic_bytes_per_launch": full_b,
-            "avg_launch_us": round(full_launch_us, 3),
+            "avg_launch_us": round(reset_us, 3),
         },
         "e2e": {"value": round(e2e_ms * 1000.0, 3), "unit": "us/step",
                 "how": "hylra_decode_step_host captured in a CUDA graph, copies included",
@@ -545,7 +597,12 @@ def run_ours(args, rank, world, dist_on):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sec, sample, threads = oracle_sample(w, m, policy, heads=(0,), reps=1)
+        first_reuse = next((l for l in range(L) if not policy[l]), None)
+        data = oracle_sample_data(
+            w, (m.q[0], m.Ks[0], m.Vs[0]),
+            None if first_reuse is None else (m.q[first_reuse], m.Ks[first_reuse],
+                                              m.Vs[first_reuse]))
+        sec, sample, threads = oracle_sample(w, data, policy)
         line["cpu_baseline"] = {"value": round(sec * 1e6, 1), "unit": "us/step",
                                 "cores": threads, "kind": "oracle", "sample": sample}
     return line
@@ -553,56 +610,57 @@ def run_ours(args, rank, world, dist_on):
 
 # ----------------------------------------------------------- reference arm
 
-def run_reference(args):
+def oracle_policy(w: W.Workload, args, gen: str):
+    """The policy the oracle derives from its own profiling run: every layer
+    a reset layer (oracle.layer_topk on every layer, sequence and KV head),
+    its overlap matrix, its DP.  Inputs are drawn layer by layer on `gen` and
+    copied to the host."""
+    from oracle import hylra_oracle as O
+    if args.policy == "jump3":
+        return O.static_policy(w.layers, 3)[0]
+    if w.policy is not None:
+        return tuple(w.policy)
+    P = max(1, args.profile_steps)
+    Hkv, k = w.num_kv_heads, w.topk
+    sets = np.full((w.layers, P * w.batch * Hkv, k), -1, dtype=np.int32)
+    for l in range(w.layers):
+        q, K, _ = W.layer_inputs(w, l, device=gen)
+        K = K.cpu()
+        for p in range(P):
+            qp = (q if p == 0 else W.step_query(w, l, p, device=gen)).cpu()
+            for b in range(w.batch):
+                _, tk = O.layer_topk(qp[b].double().numpy(),
+                                     W.per_sequence(w, K, b).double().numpy(), w.seqlens[b], k)
+                sets[l, (p * w.batch + b) * Hkv:(p * w.batch + b + 1) * Hkv] = tk
+        del q, K
+        if gen == "cuda":
+            torch.cuda.empty_cache()
+    M = O.similarity_matrix(sets)
+    return O.dp_policy(M, w.theta if args.theta is None else args.theta)[0]
+
+
+def run_reference(args, world):
     """The fp64 oracle, as it stands, on the host cores (no GPU needed; with
     one, only to draw the same inputs as our arm)."""
-    from oracle import hylra_oracle as O
     w = W.config(args.config)
-    heads = (0,)  # bounded sample: one KV head of every sequence, scaled to all heads
-
-    class _M:
-        pass
-
-    m = _M()
-    m.q, m.Ks, m.Vs = [], [], []
     # the same values as our arm: torch's generator differs between CPU and
     # GPU, so the inputs are drawn on the GPU when there is one (and only
     # then copied to the host, where all the timed work runs)
     gen = "cuda" if torch.cuda.is_available() else "cpu"
-    for l in range(w.layers):
-        q, K, V = (t.cpu() for t in W.layer_inputs(w, l, device=gen))
-        m.q.append(q)
-        m.Ks.append(K)
-        m.Vs.append(V)
+    policy = oracle_policy(w, args, gen)
+    first_reuse = next((l for l in range(w.layers) if not policy[l]), None)
+    data = oracle_sample_data(
+        w, W.layer_inputs(w, 0, device=gen),
+        W.layer_inputs(w, first_reuse, device=gen) if first_reuse is not None else None)
     if gen == "cuda":
         torch.cuda.empty_cache()
-    # policy: the oracle's own profiling + DP on this sample (every layer full)
-    if args.policy == "jump3":
-        policy, _ = O.static_policy(w.layers, 3)
-    elif w.policy is not None:
-        policy = tuple(w.policy)
-    else:
-        sets = []
-        for l in range(w.layers):
-            per = []
-            for p in range(max(1, args.profile_steps)):
-                ql = m.q[l] if p == 0 else W.step_query(w, l, p, device=gen).cpu()
-                for b in range(w.batch):
-                    kb = W.per_sequence(w, m.Ks[l], b).double().numpy()
-                    vb = W.per_sequence(w, m.Vs[l], b).double().numpy()
-                    _, _, tk = O.full_layer(ql[b].double().numpy(), kb, vb, w.seqlens[b],
-                                            w.topk)
-                    per.extend(list(tk))
-            sets.append(per)
-        M = O.similarity_matrix(np.array(sets))
-        policy, _, _ = O.dp_policy(M, w.theta if args.theta is None else args.theta)
-    times = []
     for _ in range(args.warmup):
-        oracle_sample(w, m, policy, heads=heads, reps=1)
+        oracle_sample(w, data, policy)
+    times = []
     sample = ""
     threads = 1
     for _ in range(args.steps):
-        sec, sample, threads = oracle_sample(w, m, policy, heads=heads, reps=1)
+        sec, sample, threads = oracle_sample(w, data, policy)
         times.append(sec)
     us = statistics.mean(times) * 1e6
     return {
@@ -615,13 +673,11 @@ def run_reference(args):
         "warmup": args.warmup,
         "ms_per_step": round(us / 1000.0, 3),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
-        "config": {"workload": workload_desc(w),
-                   "policy": "".join("R" if x else "U" for x in policy),
-                   "policy_rule": policy_rule(args, w)},
+        "config": config_of(w, policy, args, world),
         "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(us, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
@@ -636,7 +692,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="llama8b_32k", choices=W.CONFIG_NAMES)
+    ap.add_argument("--config", default="ragged16", choices=W.CONFIG_NAMES,
+                    help="workload (default: the largest that fits one GPU)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--policy", default="dp", choices=["dp", "jump3"],
@@ -657,7 +714,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return 0
 
     dist_on = world > 1

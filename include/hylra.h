@@ -20,7 +20,9 @@
  *   §2.2 Offline policy: a lower-triangular overlap matrix M of top-k indices
  *        between source and target layers, and a dynamic program over states
  *        (i, j) with reset jumps and vertical moves gated by theta.
- *                                          -> hylra_similarity, hylra_dp_policy
+ *                                          -> hylra_similarity, hylra_dp_policy,
+ *                                             hylra_overlap_counts,
+ *                                             hylra_similarity_from_counts
  *   §4   The Jump3 baseline (a reset every third layer).
  *                                          -> hylra_static_policy
  *
@@ -216,6 +218,25 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers,
 int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k,
                      const int32_t* topk, double* M);
 
+/* The two integer sums behind hylra_similarity (same topk argument):
+ * inter: HOST int64 [num_layers][num_layers], inter[t][s] =
+ * sum_u |I_s(u) & I_t(u)| for s <= t (0 above the diagonal); total: HOST
+ * int64 [num_layers], total[t] = sum_u |I_t(u)|.  Both are sums over the
+ * index sets, so the counts of disjoint groups of sets (for example the KV
+ * heads profiled on different GPUs) add up exactly to the counts of all of
+ * them; hylra_similarity_from_counts then gives the same M as
+ * hylra_similarity over all the sets, bit for bit.  Synchronous. */
+int hylra_overlap_counts(int32_t num_layers, int32_t num_sets, int32_t k,
+                         const int32_t* topk, int64_t* inter, int64_t* total);
+
+/* M[t][s] = inter[t][s] / total[t] for s <= t (0 where total[t] == 0, and
+ * above the diagonal); counts as written by hylra_overlap_counts (or their
+ * sums over groups of sets).  HYLRA_ERR_INVALID for counts no set of index
+ * lists can give (negative, inter[t][s] > total[t], nonzero above the
+ * diagonal).  Synchronous. */
+int hylra_similarity_from_counts(int32_t num_layers, const int64_t* inter,
+                                 const int64_t* total, double* M);
+
 /* Policy (HyLRA summary §2.2 "Dynamic Programming").  States (i, j): layer j
  * uses the indices of reset layer i; layer 0 is a reset.  Reset jump
  * (i, j) -> (j+1, j+1); vertical move (i, j) -> (i, j+1) allowed when
@@ -255,6 +276,19 @@ int hylra_static_policy(int32_t num_layers, int32_t period, uint8_t* policy,
 int hylra_decode_full_noalloc(const hylra_shape_t* shape, const void* q, const void* K,
                               const void* V, const int32_t* seqlens, float* out,
                               int32_t* topk_out, uint32_t* status_out, hylra_stream_t stream);
+
+/* Failure detection.  Every wait inside the kernels (for a TMA copy, a
+ * pipeline stage, a peer CTA's data) gives up after a limit of SM clocks,
+ * 2^31 (about a second) by default; the kernel then stops issuing copies,
+ * waits (bounded) for the copies it already issued, finishes without trusting
+ * the data it did not get, and sets HYLRA_STATUS_TIMEOUT in the workspace
+ * status word (hylra_read_status).  Its outputs are then meaningless; the
+ * workspace, cleared with hylra_read_status(..., clear = 1), serves the next
+ * call as before.  This sets the limit for launches made after the call
+ * (process-wide; a CUDA graph keeps the limit it was captured with);
+ * cycles <= 0 restores the default.  A short limit makes a watchdog fire on a
+ * healthy GPU: tests use that to exercise the path.  Always HYLRA_OK. */
+int hylra_set_wait_limit(int64_t cycles);
 
 /* Copy the workspace status word to *status (synchronises the stream); when
  * clear != 0 the word is reset to 0 afterwards. */

@@ -211,6 +211,9 @@ int rc_max_active(const RCPlan& pl) {
   return v;
 }
 
+// Limit of the kernels' bounded waits, in SM clocks (hylra_set_wait_limit).
+std::atomic<long long> g_wait_limit{WAIT_LIMIT_DEFAULT};
+
 #if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
 int g_plan_cs = 0, g_plan_nst = 0;  // tuning builds: force a plan
 int g_late_deficit = -1;            // tuning builds: force the late-start deficit
@@ -334,6 +337,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.q_wait = pdl ? 1 : 0;
   p.trace_slot = trace_slot;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
 
   if (s->dtype == HYLRA_BF16) {
     if ((rc = prepare_bf16_kernels())) return rc;
@@ -784,6 +788,12 @@ int hylra_trace_set(void* buf) {
                                                                           : HYLRA_ERR_CUDA;
 }
 #endif
+
+int hylra_set_wait_limit(int64_t cycles) {
+  g_wait_limit.store(cycles > 0 ? (long long)cycles : WAIT_LIMIT_DEFAULT,
+                     std::memory_order_relaxed);
+  return HYLRA_OK;
+}
 
 int hylra_read_status(void* workspace, uint32_t* status, int clear, hylra_stream_t stream) {
   if (!workspace || !status) return HYLRA_ERR_INVALID;

@@ -51,11 +51,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^31 SM clocks (about a second), records
-// the failure in *abort (shared) and returns false.  Once *abort is set every
-// later wait returns at once, so all warps still reach the same barriers.
+// Default limit of a bounded wait: ~2^31 SM clocks (about a second).
+constexpr long long WAIT_LIMIT_DEFAULT = 1ll << 31;
+// Limit of a drain (waiting for a CTA's own copies in flight before it exits).
+constexpr long long DRAIN_LIMIT = 1ll << 31;
+
+// Bounded wait: gives up after `limit` SM clocks, records the failure in
+// *abort (shared) and returns false.  Once *abort is set every later wait
+// returns at once; the kernels keep their barrier sequences independent of
+// the data a failed wait would have delivered, so all warps still reach the
+// same barriers and loop counts.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort,
+                                                  long long limit = WAIT_LIMIT_DEFAULT) {
   if (*abort) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -63,11 +71,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (clock64() - t0 > (1ll << 31)) {
+      if (clock64() - t0 > limit) {
         *abort = 1;
         return false;
       }
     }
+  }
+}
+
+// Drain: wait (bounded by DRAIN_LIMIT, whatever *abort says) until the phase
+// that an issued copy completes has completed, so that the CTA never exits
+// with a copy into its shared memory still in flight.  False if it gave up.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && clock64() - t0 > DRAIN_LIMIT) return false;
   }
 }
 
@@ -275,18 +295,29 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
-                                                          volatile int* abort) {
+                                                          volatile int* abort,
+                                                          long long limit = WAIT_LIMIT_DEFAULT) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (clock64() - t0 > (1ll << 31)) {
+      if (clock64() - t0 > limit) {
         *abort = 1;
         return false;
       }
     }
+  }
+}
+
+// Drain of a phase completed by other CTAs' stores (see mbar_drain).
+__device__ __forceinline__ bool mbar_drain_cluster(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0u && clock64() - t0 > DRAIN_LIMIT) return false;
   }
 }
 

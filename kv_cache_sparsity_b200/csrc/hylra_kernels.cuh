@@ -134,6 +134,7 @@ struct Params {
   int comb_in_stage; // cluster reuse kernel: the warp states go to stage 0 at the end
   int trace_slot;    // trace builds: which per-launch region of the trace buffer
   float scale_log2;  // log2(e) / sqrt(d)
+  long long wait_limit;  // SM clocks after which a bounded wait gives up
 };
 
 struct StageMeta {
@@ -951,7 +952,8 @@ struct WarpAttn {
   // to that max) of this warp's tokens for heads A and B.
   __device__ __forceinline__ void block(uint8_t* stage, int nvalid, float scale_log2,
                                         uint64_t* fullV, uint32_t ph, volatile int* abort_flag,
-                                        float& mxA, float& mxB, float& sA, float& sB) {
+                                        long long lim, float& mxA, float& mxB, float& sA,
+                                        float& sB) {
     const uint32_t kbase = smem_u32(stage);
     const uint32_t vbase = kbase + 2 * BOX_BYTES;
     const bool partial = nvalid < BLK;
@@ -977,7 +979,7 @@ struct WarpAttn {
         x[e] = v;
       }
     }
-    mbar_wait_bounded(fullV, ph, abort_flag);
+    mbar_wait_bounded(fullV, ph, abort_flag, lim);
     if (partial) {
       // rows past the sequence end may hold anything (even NaN): zero V
       for (int idx = lane; idx < 16 * 16; idx += 32) {
@@ -1066,7 +1068,7 @@ struct WarpAttn {
   // pair costs little more than one block.
   __device__ __forceinline__ void block2(uint8_t* st0, int nv0, uint64_t* fullV0, uint32_t ph0,
                                          uint8_t* st1, int nv1, uint64_t* fullV1, uint32_t ph1,
-                                         float scale_log2, volatile int* abort_flag) {
+                                         float scale_log2, volatile int* abort_flag, long long lim) {
     float x0[4], x1[4];
     {
       float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1089,8 +1091,8 @@ struct WarpAttn {
         x1[e] = tok < nv1 ? (b0[e] + b1[e]) * scale_log2 : -INFINITY;
       }
     }
-    mbar_wait_bounded(fullV0, ph0, abort_flag);
-    mbar_wait_bounded(fullV1, ph1, abort_flag);
+    mbar_wait_bounded(fullV0, ph0, abort_flag, lim);
+    mbar_wait_bounded(fullV1, ph1, abort_flag, lim);
     if (nv0 < BLK) zero_tail_v(st0, nv0);
     if (nv1 < BLK) zero_tail_v(st1, nv1);
     // max and sums over the pair's tokens for heads A and B
@@ -1316,12 +1318,14 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     // With q_wait, the first stages' K/V tiles are requested before the wait
     // and their q rows after it (qpend: stages whose q load is deferred).
     uint32_t qpend = 0u;
+    // (a deferred q load is issued even after a failed wait: its bytes are
+    // counted in its stage's phase, which the drain below waits for)
     auto wait_and_flush = [&]() {
       if (waited) return;
       griddep_wait();
       waited = true;
       for (int t = 0; t < NSTAGE; ++t) {
-        if (!(qpend & (1u << t)) || *abort_flag) continue;
+        if (!(qpend & (1u << t))) continue;
         const StageMeta& mt = sm.meta[t];
         bulk_load(sm.qslot[t], qbase + ((size_t)mt.b * p.Hq + (size_t)mt.h * p.r) * HD * 2,
                   qbytes, &sm.fullK_bar[t]);
@@ -1332,7 +1336,11 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 #ifdef HYLRA_TRACE
     int tn = 0;  // trace events of the producer thread
 #endif
+    int issued = 0;  // units 0 .. issued-1 have started their stage's phase
     for (int i = 0; i < n; ++i) {
+      // after a failed wait nothing more is issued: the consumers no longer
+      // wait for stages, so a refill could land in a stage still being read
+      if (*abort_flag) break;
       UnitIter nx = it;
       nx.advance(c, p);
       // reuse: fetch the next unit's index now, use it next iteration
@@ -1346,7 +1354,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
       // a stage is refilled only after the consumers used it, which needs q
       if (p.q_wait && i >= NSTAGE) wait_and_flush();
-      mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
+      if (!mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag, p.wait_limit)) break;
       HYLRA_TRACE_EV(tn, 256, (2 << 8) | (i & 0xff));
       const StageMeta m =
           describe_unit<FULL>(p, c, it, i, n, T, G, seqlen, FULL ? it.j : idx_cur, true);
@@ -1354,9 +1362,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (p.q_wait && m.blk >= 0 && m.blk == m.nb - 1) wait_and_flush();
       sm.meta[s] = m;
       const bool seg_start = (m.flags & F_SEG_START) != 0;
-      uint32_t bytesK = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? 2u * BOX_BYTES : 0u);
-      uint32_t bytesV = m.blk >= 0 ? 2u * BOX_BYTES : 0u;
-      if (*abort_flag) bytesK = bytesV = 0u;
+      const uint32_t bytesK = (seg_start ? qbytes : 0u) + (m.blk >= 0 ? 2u * BOX_BYTES : 0u);
+      const uint32_t bytesV = m.blk >= 0 ? 2u * BOX_BYTES : 0u;
+      issued = i + 1;
       const int row = p.staged ? (int)(((long long)(m.b * p.Hkv + m.h) * p.k + m.pos) * BLK)
                                : (int)(row0 + (long long)m.h * hstride + (long long)m.blk * BLK);
       uint8_t* st = sm.stage[s];
@@ -1388,6 +1396,13 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       idx_cur = idx_next;
     }
     if (p.q_wait) wait_and_flush();
+    // never exit with a copy into this CTA's shared memory in flight
+    for (int t = 0; t < NSTAGE && t < issued; ++t) {
+      const int last = t + (issued - 1 - t) / NSTAGE * NSTAGE;  // last unit of stage t
+      const uint32_t ph = (uint32_t)((last / NSTAGE) & 1);
+      if (!mbar_drain(&sm.fullK_bar[t], ph) || !mbar_drain(&sm.fullV_bar[t], ph)) *abort_flag = 1;
+    }
+    if (*abort_flag) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
     return;
   }
 
@@ -1402,7 +1417,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     // zero query, result discarded (brings the code into the instruction
     // cache)
     float d0, d1, d2, d3;
-    wa.block(sm.stage[0], BLK, p.scale_log2, &sm.fullV_bar[0], 0u, abort_flag, d0, d1, d2, d3);
+    wa.block(sm.stage[0], BLK, p.scale_log2, &sm.fullV_bar[0], 0u, abort_flag, p.wait_limit, d0,
+             d1, d2, d3);
     wa.reset();
   }
   bool waited = false;  // griddep_wait done (needed before the first global write)
@@ -1413,21 +1429,30 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     }
   };
   if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 1 << 8);
+  // The consumers walk the units themselves for the segment boundaries (the
+  // same walk as the producer's): every named barrier below then depends only
+  // on the split, never on a stage description, so all consumer warps meet
+  // the same barriers even after a failed wait left a description unwritten.
+  UnitIter cit;
+  if (n > 0) cit.seek(c, p, lo);
 
   for (int i = 0; i < n; ++i) {
     const int s = i % NSTAGE;
     const uint32_t ph = (uint32_t)((i / NSTAGE) & 1);
-    mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
+    const bool seg_start = i == 0 || cit.j == 0;
+    const bool seg_end = i == n - 1 || cit.j == cit.U - 1;
+    cit.advance(c, p);
+    mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag, p.wait_limit);
     if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, (3 << 8) | (i & 0xff));
     const StageMeta m = sm.meta[s];
-    if (m.flags & F_SEG_START) {
+    if (seg_start) {
       wa.reset();
       wa.load_q(sm.qslot[s], p.r);
     }
     if (m.blk >= 0) {
       float mxA, mxB, sA, sB;
-      wa.block(sm.stage[s], m.nvalid, p.scale_log2, &sm.fullV_bar[s], ph, abort_flag, mxA, mxB,
-               sA, sB);
+      wa.block(sm.stage[s], m.nvalid, p.scale_log2, &sm.fullV_bar[s], ph, abort_flag,
+               p.wait_limit, mxA, mxB, sA, sB);
       if (FULL && wa.g4 == 0) {
         sm.bst_s[s][cw][2 * wa.c4] = sA;
         sm.bst_s[s][cw][2 * wa.c4 + 1] = sB;
@@ -1435,7 +1460,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
         sm.bst_m[s][cw][2 * wa.c4 + 1] = mxB;
       }
     } else {
-      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);  // keep the phase in step
+      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag, p.wait_limit);  // keep the phase in step
     }
     if (FULL && m.blk >= 0) {
       // the last warp to finish this block merges the eight shares
@@ -1463,7 +1488,7 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, (4 << 8) | (i & 0xff));
     if (lane == 0) mbar_arrive(&sm.empty_bar[s]);
 
-    if (m.flags & F_SEG_END) {
+    if (seg_end) {
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
       ensure_waited();
       wa.to_comb(c.comb_o, c.comb_m, c.comb_z, cw);  // eight warp states -> four
@@ -1920,6 +1945,10 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       mbar_init(&sm.fullK_bar[s], 1);
       mbar_init(&sm.fullV_bar[s], 1);
       mbar_init(&sm.empty_bar[s], NW_BF16);
+      // a consumer that gave up waiting reads a description that the
+      // producer may not have written: start from "no block"
+      sm.meta_blk[s] = -1;
+      sm.meta_nvalid[s] = 0;
     }
     if (rank == 0) {
       // completes once every CTA's slot has landed (st.async transactions)
@@ -2007,9 +2036,12 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       tma_prefetch_l2_2d(&tmV, 64, row);
     }
     int qpend = 0;
+    int issued = 0;  // blocks 0 .. issued-1 have started their stage's phase
     for (int i = 0; i < nu; ++i) {
       const int s = i % nst;
       const uint32_t ph = (uint32_t)((i / nst) & 1);
+      // after a failed wait nothing more is issued (the whole warp stops)
+      if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
       int blk = i < 32 ? __shfl_sync(0xffffffffu, my_blk, i) : 0;
       if (lane != 0) continue;
       if (i >= 32) blk = __ldcg(idx + j0 + i);
@@ -2020,18 +2052,20 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       // a stage is refilled only after the consumers used it, which needs q
       // (the block holding the newest token is staged early like the rest:
       // its consumer warp rewrites the newest row after the wait)
+      // (a deferred q load is issued even after a failed wait: its bytes are
+      // counted in stage 0's first phase, which the drain below waits for)
       if (p.q_wait && !waited && i >= nst) {
         griddep_wait();
         waited = true;
-        if (qpend && !*abort_flag) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
+        if (qpend) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
         qpend = 0;
       }
-      mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag);
+      if (!mbar_wait_bounded(&sm.empty_bar[s], ph ^ 1u, abort_flag, p.wait_limit)) continue;
       sm.meta_blk[s] = blk;
       sm.meta_nvalid[s] = blk >= 0 ? min(BLK, seqlen - blk * BLK) : 0;
-      uint32_t bytesK = (i == 0 ? qbytes : 0u) + (blk >= 0 ? 2u * BOX_BYTES : 0u);
-      uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
-      if (*abort_flag) bytesK = bytesV = 0u;
+      const uint32_t bytesK = (i == 0 ? qbytes : 0u) + (blk >= 0 ? 2u * BOX_BYTES : 0u);
+      const uint32_t bytesV = blk >= 0 ? 2u * BOX_BYTES : 0u;
+      issued = i + 1;
       uint8_t* st = stages + (size_t)s * STAGE_BYTES;
       const int row = unit_row(i, blk);
       if (bytesK) {
@@ -2060,7 +2094,16 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     }
     if (lane == 0 && p.q_wait && !waited) {
       griddep_wait();
-      if (qpend && !*abort_flag) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
+      if (qpend) bulk_load(sm.qbuf, qsrc, qbytes, &sm.fullK_bar[0]);
+    }
+    // never exit with a copy into this CTA's shared memory in flight
+    if (lane == 0) {
+      for (int t = 0; t < nst && t < issued; ++t) {
+        const int last = t + (issued - 1 - t) / nst * nst;  // last block of stage t
+        const uint32_t ph = (uint32_t)((last / nst) & 1);
+        if (!mbar_drain(&sm.fullK_bar[t], ph) || !mbar_drain(&sm.fullV_bar[t], ph))
+          *abort_flag = 1;
+      }
     }
     __syncwarp();
   } else {
@@ -2080,9 +2123,11 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     auto patch_newest = [&](int s, uint32_t ph) {
       const int blk = sm.meta_blk[s];
       if (!p.q_wait || p.staged || blk < 0 || blk != nb - 1) return;
-      const int rr = sm.meta_nvalid[s] - 1;  // the newest row within the block
+      // the newest row within the block, from the length itself (not from the
+      // stage description, which a failed wait may leave half written)
+      const int rr = seqlen - 1 - blk * BLK;
       if ((rr >> 4) != cw) return;
-      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);  // V landed (K: fullK)
+      mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag, p.wait_limit);  // V landed (K: fullK)
       griddep_wait();
       const int c = lane & 15;
       const long long grow = row0c + (long long)blk * BLK + rr;
@@ -2108,8 +2153,8 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     for (; nu <= nst && i + 1 < nu; i += 2) {
       const int s0 = i % nst, s1 = (i + 1) % nst;
       const uint32_t ph0 = (uint32_t)((i / nst) & 1), ph1 = (uint32_t)(((i + 1) / nst) & 1);
-      mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag);
-      mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag);
+      mbar_wait_bounded(&sm.fullK_bar[s0], ph0, abort_flag, p.wait_limit);
+      mbar_wait_bounded(&sm.fullK_bar[s1], ph1, abort_flag, p.wait_limit);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
       const int blk0 = sm.meta_blk[s0], blk1 = sm.meta_blk[s1];
@@ -2118,12 +2163,12 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (blk1 == nb - 1) patch_newest(s1, ph1);
       wa.block2(stages + (size_t)s0 * STAGE_BYTES, nv0, &sm.fullV_bar[s0], ph0,
                 stages + (size_t)s1 * STAGE_BYTES, nv1, &sm.fullV_bar[s1], ph1, p.scale_log2,
-                abort_flag);
+                abort_flag, p.wait_limit);
     }
     for (; i < nu; ++i) {
       const int s = i % nst;
       const uint32_t ph = (uint32_t)((i / nst) & 1);
-      mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag);
+      mbar_wait_bounded(&sm.fullK_bar[s], ph, abort_flag, p.wait_limit);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 3 << 8);
       if (i == 0) wa.load_q(sm.qbuf, r);
       const int blk = sm.meta_blk[s];
@@ -2131,9 +2176,9 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (blk >= 0) {
         float mxA, mxB, sA, sB;
         wa.block(stages + (size_t)s * STAGE_BYTES, sm.meta_nvalid[s], p.scale_log2,
-                 &sm.fullV_bar[s], ph, abort_flag, mxA, mxB, sA, sB);
+                 &sm.fullV_bar[s], ph, abort_flag, p.wait_limit, mxA, mxB, sA, sB);
       } else {
-        mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag);
+        mbar_wait_bounded(&sm.fullV_bar[s], ph, abort_flag, p.wait_limit);
       }
       if (i + nst < nu) {
         __syncwarp();
@@ -2174,7 +2219,11 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
     if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 5 << 8);
     if (rank == 0) {
       // ----------------------------------------------- merge (CTA rank 0)
-      mbar_wait_cluster_bounded(&sm.gather_bar, 0u, abort_flag);
+      // every CTA sends its slot whatever happened to its waits, so the
+      // phase completes: after a failed wait, drain it before leaving (the
+      // other CTAs' stores must not land in an exited CTA)
+      if (!mbar_wait_cluster_bounded(&sm.gather_bar, 0u, abort_flag, p.wait_limit))
+        mbar_drain_cluster(&sm.gather_bar, 0u);
       if (ct == 0) HYLRA_TRACE_CTA(tn, tcta, 6 << 8);
       bool waited = false;
       for (int pr = ct; pr < r * (HD / 2); pr += NT_BF16) {

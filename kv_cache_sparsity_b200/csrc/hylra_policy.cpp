@@ -67,9 +67,9 @@ bool preferred(int r1, double s1, const std::vector<uint8_t>& p1, const Path& b)
 
 extern "C" {
 
-int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k, const int32_t* topk,
-                     double* M) {
-  if (num_layers < 1 || num_sets < 0 || k < 1 || !M || (num_sets > 0 && !topk))
+int hylra_overlap_counts(int32_t num_layers, int32_t num_sets, int32_t k, const int32_t* topk,
+                         int64_t* inter, int64_t* total) {
+  if (num_layers < 1 || num_sets < 0 || k < 1 || !inter || !total || (num_sets > 0 && !topk))
     return HYLRA_ERR_INVALID;
   const int L = num_layers, S = num_sets;
   std::vector<std::vector<int32_t>> sets((size_t)L * S);
@@ -77,21 +77,47 @@ int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k, const int3
     for (int u = 0; u < S; ++u)
       sets[(size_t)l * S + u] = index_set(topk + ((size_t)l * S + u) * k, k);
   for (int t = 0; t < L; ++t) {
+    long long tot = 0;
+    for (int u = 0; u < S; ++u) tot += (long long)sets[(size_t)t * S + u].size();
+    total[t] = tot;
     for (int s = 0; s < L; ++s) {
-      double v = 0.0;
-      if (s <= t) {
-        long long inter = 0, total = 0;
-        for (int u = 0; u < S; ++u) {
-          const auto& target = sets[(size_t)t * S + u];
-          total += (long long)target.size();
-          inter += intersection_size(sets[(size_t)s * S + u], target);
-        }
-        v = total ? (double)inter / (double)total : 0.0;
-      }
-      M[(size_t)t * L + s] = v;
+      long long n = 0;
+      if (s <= t)
+        for (int u = 0; u < S; ++u)
+          n += intersection_size(sets[(size_t)s * S + u], sets[(size_t)t * S + u]);
+      inter[(size_t)t * L + s] = n;
     }
   }
   return HYLRA_OK;
+}
+
+int hylra_similarity_from_counts(int32_t num_layers, const int64_t* inter, const int64_t* total,
+                                 double* M) {
+  if (num_layers < 1 || !inter || !total || !M) return HYLRA_ERR_INVALID;
+  const int L = num_layers;
+  for (int t = 0; t < L; ++t) {
+    if (total[t] < 0) return HYLRA_ERR_INVALID;
+    for (int s = 0; s < L; ++s) {
+      const int64_t n = inter[(size_t)t * L + s];
+      if (n < 0 || n > total[t] || (s > t && n != 0)) return HYLRA_ERR_INVALID;
+    }
+  }
+  for (int t = 0; t < L; ++t)
+    for (int s = 0; s < L; ++s)
+      M[(size_t)t * L + s] = (s <= t && total[t] > 0)
+                                 ? (double)inter[(size_t)t * L + s] / (double)total[t]
+                                 : 0.0;
+  return HYLRA_OK;
+}
+
+int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k, const int32_t* topk,
+                     double* M) {
+  if (num_layers < 1 || num_sets < 0 || k < 1 || !M || (num_sets > 0 && !topk))
+    return HYLRA_ERR_INVALID;
+  std::vector<int64_t> inter((size_t)num_layers * num_layers), total(num_layers);
+  int rc = hylra_overlap_counts(num_layers, num_sets, k, topk, inter.data(), total.data());
+  if (rc) return rc;
+  return hylra_similarity_from_counts(num_layers, inter.data(), total.data(), M);
 }
 
 int hylra_dp_policy(int32_t num_layers, const double* M, double theta, uint8_t* policy,

@@ -1,14 +1,21 @@
 """Host-side helpers for running one process per GPU.
 
-The decode path shards by sequence and KV head with no exchange step, so the
-only cross-rank traffic is timing: every rank measures its own copy of the
-work on its own GPU and the slowest rank's time is the job's time.
+The decode path splits by KV head with no exchange step in the data path:
+every (sequence, KV head) pair is independent through full attention, block
+scoring, top-k and reuse attention, so rank r holds the KV heads
+``shard(Hkv, r, world)`` of every sequence (and their query heads) and runs
+the whole step on them.  The only data crossing ranks is in the offline
+profiling: the overlap matrix is a ratio of two integer sums over index sets
+(hylra_overlap_counts), so the ranks add their counts with one integer
+all-reduce and every rank derives the same matrix, and the same policy, as a
+single GPU holding every head.  Timing is max-reduced over ranks.
 """
 
 from __future__ import annotations
 
 import os
 
+import numpy as np
 import torch
 
 
@@ -43,3 +50,32 @@ def shard(n: int, rank: int, world: int) -> range:
     lo = n * rank // world
     hi = n * (rank + 1) // world
     return range(lo, hi)
+
+
+def sum_over_ranks(*arrays: np.ndarray, device="cpu"):
+    """Element-wise integer sums of int64 host arrays over all ranks (the
+    arrays themselves when not distributed); exact, in one all-reduce."""
+    if not dist_on():
+        return tuple(np.asarray(a, dtype=np.int64) for a in arrays)
+    flat = np.concatenate([np.asarray(a, dtype=np.int64).ravel() for a in arrays])
+    t = torch.from_numpy(flat).to(device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    flat = t.cpu().numpy()
+    out, off = [], 0
+    for a in arrays:
+        n = int(np.asarray(a).size)
+        out.append(flat[off:off + n].reshape(np.asarray(a).shape))
+        off += n
+    return tuple(out)
+
+
+def pooled_similarity(H, sets: np.ndarray, device="cpu") -> np.ndarray:
+    """Overlap matrix of the index sets held by every rank together.
+
+    sets: this rank's profiled index sets, int32 [L, S_rank, k].  Each rank
+    counts its own sets with the library (H.overlap_counts), the counts are
+    summed over ranks, and the library turns the sums into M: the same matrix,
+    bit for bit, as H.similarity over all ranks' sets in one process."""
+    inter, total = H.overlap_counts(sets)
+    inter, total = sum_over_ranks(inter, total, device=device)
+    return H.similarity_from_counts(inter, total)

@@ -42,7 +42,8 @@ EXPORTS = ("hylra_workspace_bytes", "hylra_workspace_init", "hylra_decode_full",
            "hylra_similarity", "hylra_dp_policy", "hylra_read_status", "hylra_strerror",
            "hylra_version", "hylra_decode_full_noalloc", "hylra_static_policy",
            "hylra_stage_bytes", "hylra_gather_blocks", "hylra_decode_reuse_staged",
-           "hylra_decode_step_offload")
+           "hylra_decode_step_offload", "hylra_overlap_counts",
+           "hylra_similarity_from_counts", "hylra_set_wait_limit")
 
 
 class HylraError(RuntimeError):
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
         "hylra_decode_step": [SP, I32, P, P, P, P, P, P, P, P, S, P],
         "hylra_decode_step_host": [SP, I32, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "hylra_similarity": [I32, I32, I32, P, P],
+        "hylra_overlap_counts": [I32, I32, I32, P, P, P],
+        "hylra_similarity_from_counts": [I32, P, P, P],
         "hylra_dp_policy": [I32, P, ctypes.c_double, P, ctypes.POINTER(I32),
                             ctypes.POINTER(ctypes.c_double)],
         "hylra_read_status": [P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P],
@@ -102,6 +105,7 @@ def load() -> ctypes.CDLL:
         "hylra_gather_blocks": [SP, P, P, P, P, P, P, P],
         "hylra_decode_reuse_staged": [SP, P, P, P, P, P, P, P, S, P],
         "hylra_decode_step_offload": [SP, I32, P, P, P, P, P, P, P, P, P, P, P, S, P],
+        "hylra_set_wait_limit": [I64],
         "hylra_strerror": [ctypes.c_int],
         "hylra_version": [],
     }
@@ -204,6 +208,12 @@ def decode_full_noalloc(shape: Shape, q, K, V, seqlens, out, topk_out, status_ou
            "hylra_decode_full_noalloc")
 
 
+def set_wait_limit(cycles: int):
+    """Limit (SM clocks) of the kernels' bounded waits for later launches;
+    cycles <= 0 restores the default."""
+    _check(load().hylra_set_wait_limit(int(cycles)), "hylra_set_wait_limit")
+
+
 def read_status(ws, clear: bool = True, stream=None) -> int:
     v = ctypes.c_uint32(0)
     _check(load().hylra_read_status(_ptr(ws), ctypes.byref(v), int(clear), _stream(stream)),
@@ -217,6 +227,28 @@ def similarity(topk: np.ndarray) -> np.ndarray:
     L, S, k = t.shape
     M = np.zeros((L, L), dtype=np.float64)
     _check(load().hylra_similarity(L, S, k, t.ctypes.data, M.ctypes.data), "hylra_similarity")
+    return M
+
+
+def overlap_counts(topk: np.ndarray):
+    """topk: int32 [L, S, k] host array -> (inter [L, L] int64, total [L] int64)."""
+    t = np.ascontiguousarray(topk, dtype=np.int32)
+    L, S, k = t.shape
+    inter = np.zeros((L, L), dtype=np.int64)
+    total = np.zeros(L, dtype=np.int64)
+    _check(load().hylra_overlap_counts(L, S, k, t.ctypes.data, inter.ctypes.data,
+                                       total.ctypes.data), "hylra_overlap_counts")
+    return inter, total
+
+
+def similarity_from_counts(inter: np.ndarray, total: np.ndarray) -> np.ndarray:
+    """(inter [L, L], total [L]) int64 host arrays -> M [L, L] float64."""
+    i = np.ascontiguousarray(inter, dtype=np.int64)
+    t = np.ascontiguousarray(total, dtype=np.int64)
+    L = t.shape[0]
+    M = np.zeros((L, L), dtype=np.float64)
+    _check(load().hylra_similarity_from_counts(L, i.ctypes.data, t.ctypes.data, M.ctypes.data),
+           "hylra_similarity_from_counts")
     return M
 
 

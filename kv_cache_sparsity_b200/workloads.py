@@ -178,11 +178,15 @@ def _gen(device, seed: int) -> torch.Generator:
     return g
 
 
-def step_query(w: Workload, layer: int, step: int, device="cpu"):
+def step_query(w: Workload, layer: int, step: int, device="cpu", heads=None):
     """The query of one layer at decode step `step` ([B][Hq][d]); step 0 is the
     query of layer_inputs.  Later steps draw fresh noise around the same
     salient directions (the cache is left as it is: over a few profiled steps
-    its growth by one token each is negligible)."""
+    its growth by one token each is negligible).  ``heads``: only the query
+    heads of those KV heads."""
+    if heads is not None:
+        q = step_query(w, layer, step, device)
+        return q[:, heads.start * w.group:heads.stop * w.group].contiguous()
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     B, Hq, d = w.batch, w.num_q_heads, w.head_dim
     base = (w.seed * 1000003 + layer * 101) * 4
@@ -198,11 +202,23 @@ def step_query(w: Workload, layer: int, step: int, device="cpu"):
     return q.to(dt)
 
 
-def layer_inputs(w: Workload, layer: int, device="cpu"):
+def layer_inputs(w: Workload, layer: int, device="cpu", heads=None):
     """(q, K, V) of one layer, in the workload's dtype and layout, on ``device``.
 
     The same (workload, layer, device type) always gives the same values.
+    ``heads`` (a range of KV heads) keeps only those KV heads and their query
+    heads, with the values they have in the whole layer.
     """
+    if heads is not None:
+        q, K, V = layer_inputs(w, layer, device)
+        h0, h1 = heads.start, heads.stop
+        r = w.group
+        q = q[:, h0 * r:h1 * r].contiguous()
+        if w.packed:
+            K, V = K[h0:h1].contiguous(), V[h0:h1].contiguous()
+        else:
+            K, V = K[:, h0:h1].contiguous(), V[:, h0:h1].contiguous()
+        return q, K, V
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     B, Hq, H, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
     base = (w.seed * 1000003 + layer * 101) * 4

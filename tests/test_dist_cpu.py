@@ -1,10 +1,13 @@
 """World-size-2 checks of the per-rank host logic, on CPU with gloo: the
-slowest rank's time is reported by every rank, barriers pair up, and the
-sequence shards of a batch cover it exactly once."""
+slowest rank's time is reported by every rank, barriers pair up, the KV-head
+shards cover the heads exactly once, and the overlap matrix pooled over the
+ranks' index sets (integer counts, one all-reduce) equals the single-process
+matrix bit for bit."""
 
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -50,6 +53,57 @@ def test_two_ranks_max_and_shards():
     assert [g for _, g, _ in res] == [3.75, 3.75]
     covered = res[0][2] + res[1][2]
     assert sorted(covered) == list(range(7))
+
+
+def _profiled_sets(L=7, B=3, Hkv=4, k=6, nb=20, seed=5):
+    """Synthetic profiled index sets [L, B, Hkv, k] with some -1 padding."""
+    rng = np.random.default_rng(seed)
+    t = np.full((L, B, Hkv, k), -1, dtype=np.int32)
+    for l in range(L):
+        for b in range(B):
+            for h in range(Hkv):
+                m = k - (b == 2) * 2
+                t[l, b, h, :m] = rng.choice(nb, size=m, replace=False)
+    return t
+
+
+def _pool_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from kv_cache_sparsity_b200 import hylra as H
+        H.load()
+        sets = _profiled_sets()
+        L, B, Hkv, k = sets.shape
+        heads = D.shard(Hkv, rank, world)
+        mine = sets[:, :, heads.start:heads.stop].reshape(L, -1, k)
+        M = D.pooled_similarity(H, mine)
+        q.put((rank, list(heads), M.tobytes()))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_two_ranks_pool_the_overlap_matrix_exactly():
+    from kv_cache_sparsity_b200 import build as hbuild
+    from kv_cache_sparsity_b200 import hylra as H
+    from oracle import hylra_oracle as O
+    hbuild.build()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_pool_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    sets = _profiled_sets()
+    L, B, Hkv, k = sets.shape
+    assert sorted(res[0][1] + res[1][1]) == list(range(Hkv))
+    whole = O.similarity_matrix(sets.reshape(L, -1, k))
+    assert res[0][2] == res[1][2] == whole.tobytes()
 
 
 def test_single_process_fallbacks():

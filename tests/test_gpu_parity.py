@@ -530,3 +530,55 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(H.HylraError) as e:
         H.decode_full(run.shape, q, K, V, run.seqlens, run.new_out(), run.new_topk(), small)
     assert e.value.code == -4
+
+
+def test_bounded_waits_give_up_and_the_workspace_recovers():
+    """Failure detection without a fault: with a wait limit of one SM clock
+    the kernels' waits for their TMA copies (and the reuse cluster's wait for
+    its peers) give up.  Each kernel then stops issuing, waits for the copies
+    it already issued, finishes, and sets HYLRA_STATUS_TIMEOUT.  With the
+    default limit back, the same workspace (status cleared) gives exactly the
+    results of a run that never timed out."""
+    w = W.custom("timeout", batch=2, layers=4, seqlens=(20000, 9000), num_q_heads=32,
+                 num_kv_heads=8, topk=16, seed=51)
+    run = T.Runner(w)
+    layers = [_layer(w, l) for l in range(w.layers)]
+    args = ([l[0] for l in layers], [l[1] for l in layers], [l[2] for l in layers])
+    policy = (1, 0, 0, 1)
+
+    def step():
+        topk = torch.full((w.layers, 2, 8, 16), -7, dtype=torch.int32, device="cuda")
+        outs = [run.new_out() for _ in range(w.layers)]
+        H.decode_step(run.shape, policy, *args, run.seqlens, outs, topk, run.ws)
+        return outs, topk
+
+    def single_layers():
+        out, tk = run.full(*layers[0])
+        return [out, run.reuse(*layers[1], tk)], tk
+
+    good = step()
+    assert run.status() == 0
+    good_single = single_layers()
+    assert run.status() == 0
+    seen = {}
+    try:
+        H.set_wait_limit(1)
+        for name, fn in (("step", step), ("single", single_layers)):
+            for _ in range(5):  # a wait gives up unless its data was already there
+                fn()
+                st = run.status()  # reads and clears
+                # (a layer that gave up computes on whatever its stages held, so its
+                # block scores may also be flagged as non-finite)
+                assert st & ~(H.STATUS_TIMEOUT | H.STATUS_NONFINITE) == 0, f"{name}: {st:#x}"
+                if st & H.STATUS_TIMEOUT:
+                    seen[name] = True
+                    break
+    finally:
+        H.set_wait_limit(0)
+    assert seen == {"step": True, "single": True}, seen
+    for fn, ref in ((step, good), (single_layers, good_single)):
+        outs, tk = fn()
+        assert run.status() == 0
+        for a, b in zip(outs, ref[0]):
+            assert torch.equal(a, b)
+        assert torch.equal(tk, ref[1])

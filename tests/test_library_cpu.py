@@ -108,6 +108,35 @@ def test_similarity_matches_oracle_bitwise(lib, seed):
     assert M.tobytes() == Mo.tobytes()
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_overlap_counts_match_oracle(lib, seed):
+    rng = np.random.default_rng(50 + seed)
+    L, S, k = int(rng.integers(1, 10)), int(rng.integers(1, 16)), int(rng.integers(1, 9))
+    nb = int(rng.integers(k, 3 * k + 2))
+    topk = np.full((L, S, k), -1, dtype=np.int32)
+    for l in range(L):
+        for u in range(S):
+            kp = int(rng.integers(0, k + 1))
+            topk[l, u, :kp] = rng.permutation(nb)[:kp]
+    inter, total = H.overlap_counts(topk)
+    io, to = O.overlap_counts(topk)
+    assert np.array_equal(inter, io) and np.array_equal(total, to)
+    M = H.similarity_from_counts(inter, total)
+    assert M.tobytes() == O.similarity_from_counts(io, to).tobytes()
+    assert M.tobytes() == H.similarity(topk).tobytes()
+
+
+def test_similarity_from_counts_rejects_impossible_counts(lib):
+    inter = np.array([[2, 0], [3, 2]], dtype=np.int64)
+    with pytest.raises(H.HylraError):
+        H.similarity_from_counts(inter, np.array([2, 2], dtype=np.int64))  # 3 > total 2
+    with pytest.raises(H.HylraError):
+        H.similarity_from_counts(np.array([[2, 1], [1, 2]], dtype=np.int64),
+                                 np.array([2, 2], dtype=np.int64))  # above the diagonal
+    M = H.similarity_from_counts(np.zeros((2, 2), dtype=np.int64), np.zeros(2, dtype=np.int64))
+    assert np.all(M == 0.0)
+
+
 def _dyadic(L, rng, denom=64):
     M = np.zeros((L, L))
     for t in range(L):
