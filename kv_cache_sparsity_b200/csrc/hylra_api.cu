@@ -237,6 +237,7 @@ bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return false;
 #if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
+  if (g_plan_cs < 0) return false;  // the stream-K split over every SM instead
   if (g_plan_cs > 0) {
     const RCPlan pl = rc_plan_for(std::min(g_plan_cs, kmax), kmax, r, g_plan_nst);
     if (pl.nst < 1 || rc_max_active(pl) < 1) return false;
@@ -767,7 +768,8 @@ int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const
 }
 
 #if defined(HYLRA_TRACE) || defined(HYLRA_TUNE)
-// Tuning and trace builds only: force the reuse cluster plan (cs = 0: automatic).
+// Tuning and trace builds only: force the reuse cluster plan (cs = 0: automatic,
+// cs < 0: no cluster kernel).
 int hylra_plan_override(int cs, int nst) {
   g_plan_cs = cs;
   g_plan_nst = nst;

@@ -183,6 +183,40 @@ def layer_topk(q, K, n: int, k: int):
     return S32, topk
 
 
+def token_scores(probs: np.ndarray, num_kv_heads: int) -> np.ndarray:
+    """fp64 attention mass of every token, per KV head: S[h, t] = sum over
+    the r q-heads g of KV head h of p[g, t].  The token-level counterpart of
+    ``block_scores`` for a profiling run that records top-k *token* indices
+    (HyLRA summary §2.2, "Similarity Matrix Construction", speaks of top-k
+    token indices; the block version follows §2.4)."""
+    Hq, n = probs.shape
+    r = Hq // num_kv_heads
+    S = np.zeros((num_kv_heads, n), dtype=np.float64)
+    for h in range(num_kv_heads):
+        for g in range(h * r, (h + 1) * r):
+            S[h] += probs[g]
+    return S
+
+
+def layer_token_topk(q, K, n: int, k_tokens: int):
+    """Top-k tokens of a reset layer, per KV head: fp32 token scores (fp64
+    mass rounded once) ranked by score descending, lower token index first
+    among equal scores, padded with -1.  Returns (S32 [Hkv, n] float32,
+    topk [Hkv, k_tokens] int32)."""
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    Hkv = K.shape[0]
+    r = Hq // Hkv
+    probs = np.zeros((Hq, n), dtype=np.float64)
+    if n > 0:
+        for g in range(Hq):
+            probs[g] = attention_probs(q[g], K[g // r, :n])
+    S32 = round_scores_fp32(token_scores(probs, Hkv))
+    # the ranking rule is the blocks' one, applied to tokens
+    topk = np.stack([topk_blocks(S32[h], k_tokens) for h in range(Hkv)])
+    return S32, topk
+
+
 def topk_gap(S32_h: np.ndarray, k: int) -> float:
     """Smallest relative gap between consecutive ranks 1..k'+1 of one head.
 

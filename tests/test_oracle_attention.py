@@ -204,3 +204,58 @@ def test_layer_topk_dominant_keys_rank_their_blocks_first():
         K[0, beta * 128 + 5, 0] = bump   # logit = bump on that one token
     _, tk = O.layer_topk(q, K, n, 3)
     assert list(tk[0]) == [7, 2, 9]
+
+
+# ---------------------------------------------------------- token-level top-k
+
+@pytest.mark.parametrize("n", [1, 5, 300, 1024])
+def test_token_scores_sum_to_group_size_and_match_block_sums(n):
+    q = _rand((8, 32), 21)
+    K = _rand((2, n, 32), 22)
+    V = _rand((2, n, 32), 23)
+    _, probs = O.full_attention(q, K, V, n)
+    St = O.token_scores(probs, 2)
+    np.testing.assert_allclose(St.sum(axis=1), 4.0, rtol=0, atol=1e-11)
+    Sb = O.block_scores(probs, 2)
+    for beta in range(O.num_blocks(n)):
+        lo, hi = 128 * beta, min(128 * beta + 128, n)
+        np.testing.assert_allclose(St[:, lo:hi].sum(axis=1), Sb[:, beta], rtol=1e-13, atol=0)
+
+
+def test_token_topk_hand_worked():
+    """One KV head, two q-heads, five tokens; query along axis 0, keys with
+    logits ln(1), ln(4), ln(2), ln(4), ln(3) for both heads: masses
+    proportional to 1, 4, 2, 4, 3 (the two 4s tie: lower index first)."""
+    d = 4
+    q = np.zeros((2, d))
+    q[:, 0] = math.sqrt(d)
+    K = np.zeros((1, 5, d))
+    K[0, :, 0] = np.log([1.0, 4.0, 2.0, 4.0, 3.0])
+    S32, tk = O.layer_token_topk(q, K, 5, 3)
+    np.testing.assert_allclose(S32[0], 2 * np.array([1, 4, 2, 4, 3]) / 14, rtol=1e-6)
+    assert list(tk[0]) == [1, 3, 4]
+    _, tk6 = O.layer_token_topk(q, K, 5, 6)
+    assert list(tk6[0]) == [1, 3, 4, 2, 0, -1]
+
+
+def test_token_topk_reduces_to_blocks_for_block_constant_keys():
+    """Keys constant inside each 128-token block: every token of a block has
+    the same score, so the top k*128 tokens are exactly the tokens of the top
+    k blocks, and the token-level overlap matrix equals the block-level one."""
+    d, hq, hkv, nb, k = 16, 4, 2, 12, 3
+    rng = np.random.default_rng(5)
+    sets_b, sets_t = [], []
+    for layer in range(4):
+        q = rng.standard_normal((hq, d))
+        blockkeys = rng.standard_normal((hkv, nb, d)) * 2.0
+        K = np.repeat(blockkeys, 128, axis=1)
+        _, tkb = O.layer_topk(q, K, 128 * nb, k)
+        _, tkt = O.layer_token_topk(q, K, 128 * nb, 128 * k)
+        for h in range(hkv):
+            want = sorted(t for beta in tkb[h] for t in range(128 * beta, 128 * beta + 128))
+            assert sorted(tkt[h].tolist()) == want
+        sets_b.append(tkb)
+        sets_t.append(tkt)
+    Mb = O.similarity_matrix(np.array(sets_b))
+    Mt = O.similarity_matrix(np.array(sets_t))
+    assert Mt.tobytes() == Mb.tobytes()
