@@ -32,6 +32,7 @@ cpu_baseline / --impl reference = the fp64 oracle, single-threaded on the host,
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -248,7 +249,18 @@ def policy_rule(args, w) -> str:
     if w.policy is not None:
         return "fixed by the workload"
     theta = w.theta if args.theta is None else args.theta
-    return f"dp theta={theta:g} profile_steps={max(1, args.profile_steps)}"
+    rule = f"dp theta={theta:g} profile_steps={max(1, args.profile_steps)}"
+    if args.profile_seeds > 1:
+        rule += f" profile_seeds={args.profile_seeds}"
+    if args.token_topk > 0:
+        rule += f" token_topk={args.token_topk}"
+    return rule
+
+
+def seed_variant(w: W.Workload, s: int) -> W.Workload:
+    """Workload s of a multi-seed profiling run: the same shapes and lengths,
+    its own salient structure and noise (s = 0: the benchmarked workload)."""
+    return w if s == 0 else dataclasses.replace(w, seed=w.seed + 7919 * s)
 
 
 def step_bytes(w: W.Workload, policy) -> int:
@@ -269,14 +281,34 @@ def config_of(w: W.Workload, policy, args, world: int) -> dict:
     }
 
 
-def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int = 1):
+def profile_layer_sets(m: Model, H, q, K, V, token_topk: int) -> np.ndarray:
+    """Index sets of one layer run as a reset layer, one per (sequence, KV
+    head): its top-k blocks, or with token_topk > 0 its top-`token_topk`
+    tokens (token scores on the GPU, selection on the host)."""
+    w = m.w
+    out = torch.empty(w.batch, m.nq, w.head_dim, device="cuda")
+    tk = torch.empty(w.batch, m.nkv, w.topk, dtype=torch.int32, device="cuda")
+    if token_topk <= 0:
+        H.decode_full(m.shape, q, K, V, m.seqlens, out, tk, m.ws)
+        return tk.cpu().numpy().reshape(w.batch * m.nkv, w.topk)
+    scores = torch.empty(w.batch, m.nkv, max(1, w.max_seqlen), device="cuda")
+    H.token_scores(m.shape, q, K, V, m.seqlens, out, tk, scores, m.ws)
+    sc = scores.cpu().numpy().reshape(w.batch * m.nkv, -1)
+    lengths = np.repeat(np.array(w.seqlens, dtype=np.int32), m.nkv)
+    return H.token_topk(sc, token_topk, lengths)
+
+
+def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int = 1,
+                  profile_seeds: int = 1, token_topk: int = 0):
     """The step's reset/reuse policy.
 
     dp: profiling run(s) with every layer full -> overlap matrix -> DP policy
     (HyLRA summary §2.2).  With profile_steps P > 1 the index sets of P decode
-    steps (fresh queries, same cache) are pooled into one matrix.  Over
-    several ranks the matrix is pooled from every rank's index sets (integer
-    counts summed over ranks), so all ranks derive the single-GPU policy.  A
+    steps (fresh queries, same cache) are pooled into one matrix; with
+    profile_seeds S > 1 those of S workloads that differ only by seed; with
+    token_topk > 0 the sets are top-k tokens instead of blocks.  Over several
+    ranks the matrix is pooled from every rank's index sets (integer counts
+    summed over ranks), so all ranks derive the single-GPU policy.  A
     workload with a fixed policy keeps it.  jump3: a reset every third layer
     (the static baseline of §4)."""
     w = m.w
@@ -291,10 +323,23 @@ def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int 
     for p in range(max(1, profile_steps)):
         if p > 0:
             m.q = [W.step_query(w, l, p, device="cuda", heads=m.heads) for l in range(w.layers)]
-        m.step(allfull)
-        torch.cuda.synchronize()
-        sets.append(m.topk.cpu().numpy().reshape(w.layers, w.batch * m.nkv, w.topk))
+        if token_topk > 0:
+            sets.append(np.stack([profile_layer_sets(m, H, m.q[l], m.Ks[l], m.Vs[l], token_topk)
+                                  for l in range(w.layers)]))
+        else:
+            m.step(allfull)  # the step's own launch configuration
+            torch.cuda.synchronize()
+            sets.append(m.topk.cpu().numpy().reshape(w.layers, w.batch * m.nkv, w.topk))
     m.q = q0
+    for s in range(1, max(1, profile_seeds)):
+        ws = seed_variant(w, s)
+        per_layer = []
+        for l in range(w.layers):
+            q, K, V = W.layer_inputs(ws, l, device="cuda", heads=m.heads)
+            per_layer.append(profile_layer_sets(m, H, q, K, V, token_topk))
+            del q, K, V
+        sets.append(np.stack(per_layer))
+        torch.cuda.empty_cache()
     M = D.pooled_similarity(H, np.concatenate(sets, axis=1), device="cuda")
     pol, R, S = H.dp_policy(M, w.theta if theta is None else theta)
     return pol, M
@@ -486,7 +531,8 @@ def run_ours(args, rank, world, dist_on):
     if per_layer * w.layers > free * 0.85:
         resident = max(1, int(free * 0.85 // per_layer))
     m = Model(w, H, resident, heads)
-    policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps)
+    policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps,
+                              args.profile_seeds, args.token_topk)
     L = w.layers
     allfull = (1,) * L
     one_then_reuse = (1,) + (0,) * (L - 1)
@@ -621,20 +667,26 @@ def oracle_policy(w: W.Workload, args, gen: str):
     if w.policy is not None:
         return tuple(w.policy)
     P = max(1, args.profile_steps)
-    Hkv, k = w.num_kv_heads, w.topk
-    sets = np.full((w.layers, P * w.batch * Hkv, k), -1, dtype=np.int32)
+    S = max(1, args.profile_seeds)
+    Hkv = w.num_kv_heads
+    k = args.token_topk if args.token_topk > 0 else w.topk
+    rank_fn = O.layer_token_topk if args.token_topk > 0 else O.layer_topk
+    sets = np.full((w.layers, (P + S - 1) * w.batch * Hkv, k), -1, dtype=np.int32)
+    # the sets in our arm's order: steps 0..P-1 of the workload, then seeds 1..S-1
+    runs = [(0, p) for p in range(P)] + [(s, 0) for s in range(1, S)]
     for l in range(w.layers):
-        q, K, _ = W.layer_inputs(w, l, device=gen)
-        K = K.cpu()
-        for p in range(P):
-            qp = (q if p == 0 else W.step_query(w, l, p, device=gen)).cpu()
+        for j, (s, p) in enumerate(runs):
+            ws = seed_variant(w, s)
+            q, K, _ = W.layer_inputs(ws, l, device=gen)
+            K = K.cpu()
+            qp = (q if p == 0 else W.step_query(ws, l, p, device=gen)).cpu()
             for b in range(w.batch):
-                _, tk = O.layer_topk(qp[b].double().numpy(),
-                                     W.per_sequence(w, K, b).double().numpy(), w.seqlens[b], k)
-                sets[l, (p * w.batch + b) * Hkv:(p * w.batch + b + 1) * Hkv] = tk
-        del q, K
-        if gen == "cuda":
-            torch.cuda.empty_cache()
+                _, tk = rank_fn(qp[b].double().numpy(), W.per_sequence(w, K, b).double().numpy(),
+                                w.seqlens[b], k)
+                sets[l, (j * w.batch + b) * Hkv:(j * w.batch + b + 1) * Hkv] = tk
+            del q, K, qp
+            if gen == "cuda":
+                torch.cuda.empty_cache()
     M = O.similarity_matrix(sets)
     return O.dp_policy(M, w.theta if args.theta is None else args.theta)[0]
 
@@ -704,6 +756,10 @@ def main():
                     help="also time the step with the reuse layers' caches in host memory")
     ap.add_argument("--profile-steps", type=int, default=1,
                     help="decode steps pooled into the profiled overlap matrix")
+    ap.add_argument("--profile-seeds", type=int, default=1,
+                    help="synthetic workloads (seeds) pooled into the profiled overlap matrix")
+    ap.add_argument("--token-topk", type=int, default=0,
+                    help="profile top-k tokens (this many per head) instead of top-k blocks")
     ap.add_argument("--no-clock-fill", action="store_true",
                     help="skip the extra busy window for the clock sampler (profiler runs)")
     args = ap.parse_args()

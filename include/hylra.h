@@ -237,6 +237,30 @@ int hylra_overlap_counts(int32_t num_layers, int32_t num_sets, int32_t k,
 int hylra_similarity_from_counts(int32_t num_layers, const int64_t* inter,
                                  const int64_t* total, double* M);
 
+/* Token-level profiling (HyLRA summary §2.2 "Similarity Matrix Construction"
+ * speaks of top-k *token* indices; the decode path selects 128-token blocks,
+ * §2.4).  A reset layer exactly as hylra_decode_full (out and topk_out are
+ * written the same way), plus the attention mass of every cached token
+ * summed over the r q-heads of its KV head: scores[b][h][t] =
+ * sum_g p_{g,t} for t < n_b, 0 for n_b <= t < max_seqlen.  scores: device
+ * fp32 [B][Hkv][max_seqlen].  For profiling runs (CUDA cores, two extra
+ * kernels that re-read K), not for the decode step.  B * Hkv <= 65535. */
+int hylra_token_scores(const hylra_shape_t* shape, const void* q, const void* K,
+                       const void* V, const int32_t* seqlens, float* out,
+                       int32_t* topk_out, float* scores, void* workspace,
+                       size_t workspace_bytes, hylra_stream_t stream);
+
+/* Top-k entries of each of num_lists score lists (host): scores HOST fp32
+ * [num_lists][n], lengths HOST int32 [num_lists] (entries 0..lengths[u]-1 of
+ * list u are valid; NULL: all n), topk HOST int32 [num_lists][k]: indices in
+ * rank order (score descending, lower index first among equal scores),
+ * padded with -1.  Scores must be finite and >= 0 (HYLRA_ERR_INVALID
+ * otherwise, nothing written).  With hylra_token_scores' output this gives
+ * the token-level index sets; hylra_similarity takes them as it takes block
+ * sets.  Synchronous. */
+int hylra_token_topk(int32_t num_lists, int32_t n, const float* scores,
+                     const int32_t* lengths, int32_t k, int32_t* topk);
+
 /* Policy (HyLRA summary §2.2 "Dynamic Programming").  States (i, j): layer j
  * uses the indices of reset layer i; layer 0 is a reset.  Reset jump
  * (i, j) -> (j+1, j+1); vertical move (i, j) -> (i, j+1) allowed when

@@ -674,6 +674,54 @@ int hylra_decode_step(const hylra_shape_t* shape, int32_t num_layers, const uint
                   nullptr, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
+int hylra_token_scores(const hylra_shape_t* shape, const void* q, const void* K, const void* V,
+                       const int32_t* seqlens, float* out, int32_t* topk_out, float* scores,
+                       void* workspace, size_t workspace_bytes, hylra_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!scores || !aligned(scores, 4)) return HYLRA_ERR_INVALID;
+  const int nbh = shape->batch * shape->num_kv_heads;
+  const int nbmax = std::max(1, (shape->max_seqlen + BLK - 1) / BLK);
+  if (nbh > 65535) return HYLRA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the reset layer itself: its block records stay in the workspace
+  if ((rc = launch(shape, true, q, K, V, seqlens, nullptr, out, topk_out, workspace,
+                   workspace_bytes, st)))
+    return rc;
+  int G = 0;
+  if ((rc = sm_count(&G))) return rc;
+  const Layout L = make_layout(shape, G);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  Params p{};
+  p.q = q;
+  p.K = K;
+  p.V = V;
+  p.seqlens = seqlens;
+  p.seq_off = shape->kv_capacity > 0 ? nullptr : shape->seq_offsets;
+  p.status = reinterpret_cast<uint32_t*>(w + L.status);
+  p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.bstat = reinterpret_cast<float*>(w + L.bstat);
+  p.cap = shape->kv_capacity;
+  p.total = shape->kv_capacity > 0 ? 0 : shape->total_tokens;
+  p.B = shape->batch;
+  p.Hq = shape->num_q_heads;
+  p.Hkv = shape->num_kv_heads;
+  p.r = shape->num_q_heads / shape->num_kv_heads;
+  p.k = shape->topk;
+  p.max_seqlen = shape->max_seqlen;
+  p.nbmax = L.nbmax;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
+  // the partials are consumed by the merge: their space holds the head statistics
+  float2* stats = reinterpret_cast<float2*>(p.partials);
+  head_stats_kernel<<<nbh, NT_TOKEN, 0, st>>>(p, stats);
+  const dim3 grid(nbmax, nbh);
+  if (shape->dtype == HYLRA_BF16)
+    token_scores_kernel<__nv_bfloat16><<<grid, NT_TOKEN, 0, st>>>(p, stats, scores);
+  else
+    token_scores_kernel<float><<<grid, NT_TOKEN, 0, st>>>(p, stats, scores);
+  return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
+}
+
 int hylra_stage_bytes(const hylra_shape_t* shape, size_t* bytes) {
   int rc = check_shape(shape);
   if (rc) return rc;

@@ -2297,6 +2297,101 @@ __global__ void __launch_bounds__(NT_GATHER) gather_blocks_kernel(const __grid_c
   }
 }
 
+// ------------------------------------------------ token-level profiling
+//
+// A profiling run may record top-k *token* indices instead of blocks (HyLRA
+// summary §2.2 speaks of top-k token indices).  After a reset layer
+// (decode_bf16_kernel<true> / decode_f32_kernel<true> + merge) the workspace
+// holds every block's record (its max and its sum relative to it, per
+// q-head).  head_stats_kernel reduces them to each head's max M_g and sum Z_g
+// (log2 domain) and token_scores_kernel recomputes every token's logits and
+// writes its attention mass summed over the group,
+// score[t] = sum_g 2^(x_gt - M_g) / Z_g.  CUDA cores: this is profiling, not
+// the decode path.
+constexpr int NT_TOKEN = 128;  // one token per thread, one block per CTA
+
+// Per (b, h): (M_g, Z_g) of its r heads into stats[bh][g] (float2).
+__global__ void __launch_bounds__(NT_TOKEN) head_stats_kernel(const __grid_constant__ Params p,
+                                                             float2* stats) {
+  __shared__ float red_m[NT_TOKEN / 32][GMAX], red_z[NT_TOKEN / 32][GMAX];
+  const int bh = (int)blockIdx.x, b = bh / p.Hkv;
+  const int tid = (int)threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nb = (valid_seqlen(p, b, false) + BLK - 1) / BLK;
+  for (int g = 0; g < p.r; ++g) {
+    float M = -INFINITY, Z = 0.f;
+    for (int beta = tid; beta < nb; beta += NT_TOKEN) {
+      const float2 rec = *reinterpret_cast<const float2*>(p.bstat + bstat_at(p, bh, g, beta));
+      if (rec.y == -INFINITY) continue;  // a block without valid tokens
+      if (rec.y > M) {
+        Z = Z * (M == -INFINITY ? 0.f : exp2f(M - rec.y));
+        M = rec.y;
+      }
+      Z += rec.x * exp2f(rec.y - M);
+    }
+    // warp then CTA merge of (M, Z)
+    for (int off = 16; off > 0; off >>= 1) {
+      const float Mo = __shfl_xor_sync(0xffffffffu, M, off);
+      const float Zo = __shfl_xor_sync(0xffffffffu, Z, off);
+      const float Mn = fmaxf(M, Mo);
+      Z = (Mn == -INFINITY) ? 0.f
+                            : (M == -INFINITY ? 0.f : Z * exp2f(M - Mn)) +
+                                  (Mo == -INFINITY ? 0.f : Zo * exp2f(Mo - Mn));
+      M = Mn;
+    }
+    if (lane == 0) {
+      red_m[wid][g] = M;
+      red_z[wid][g] = Z;
+    }
+  }
+  __syncthreads();
+  if (tid < p.r) {
+    const int g = tid;
+    float M = -INFINITY;
+    for (int w = 0; w < NT_TOKEN / 32; ++w) M = fmaxf(M, red_m[w][g]);
+    float Z = 0.f;
+    if (M != -INFINITY)
+      for (int w = 0; w < NT_TOKEN / 32; ++w)
+        if (red_m[w][g] != -INFINITY) Z += red_z[w][g] * exp2f(red_m[w][g] - M);
+    stats[(size_t)bh * GMAX + g] = make_float2(M, Z);
+  }
+}
+
+// Grid (nbmax, B * Hkv): token t = 128 * blockIdx.x + threadIdx.x of (b, h);
+// scores [B][Hkv][max_seqlen], 0 past the sequence end.
+template <typename T>
+__global__ void __launch_bounds__(NT_TOKEN) token_scores_kernel(const __grid_constant__ Params p,
+                                                               const float2* stats,
+                                                               float* scores) {
+  __shared__ float qs[GMAX][HD];
+  __shared__ float2 st[GMAX];
+  const int bh = (int)blockIdx.y, b = bh / p.Hkv, h = bh - b * p.Hkv;
+  const int tid = (int)threadIdx.x;
+  const int n = valid_seqlen(p, b, false);
+  const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.r) * HD;
+  for (int e = tid; e < p.r * HD; e += NT_TOKEN) qs[e / HD][e % HD] = (float)qg[e];
+  if (tid < p.r) st[tid] = stats[(size_t)bh * GMAX + tid];
+  __syncthreads();
+  const int t = (int)blockIdx.x * BLK + tid;
+  if (t >= p.max_seqlen) return;
+  float score = 0.f;
+  if (t < n) {
+    const T* krow = static_cast<const T*>(p.K) + (row_base(p, b, h) + t) * HD;
+    float acc[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) acc[g] = 0.f;
+    for (int d = 0; d < HD; ++d) {
+      const float kv = (float)krow[d];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g)
+        if (g < p.r) acc[g] = fmaf(kv, qs[g][d], acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g)
+      if (g < p.r && st[g].y > 0.f) score += exp2f(acc[g] * p.scale_log2 - st[g].x) / st[g].y;
+  }
+  scores[(size_t)bh * p.max_seqlen + t] = score;
+}
+
 // ------------------------------------------------------------ fp32 kernel
 
 template <bool FULL>

@@ -120,6 +120,35 @@ int hylra_similarity(int32_t num_layers, int32_t num_sets, int32_t k, const int3
   return hylra_similarity_from_counts(num_layers, inter.data(), total.data(), M);
 }
 
+int hylra_token_topk(int32_t num_lists, int32_t n, const float* scores, const int32_t* lengths,
+                     int32_t k, int32_t* topk) {
+  if (num_lists < 0 || n < 0 || k < 1 || !topk || (num_lists > 0 && n > 0 && !scores))
+    return HYLRA_ERR_INVALID;
+  for (int u = 0; u < num_lists; ++u) {
+    const int len = lengths ? lengths[u] : n;
+    if (len < 0 || len > n) return HYLRA_ERR_INVALID;
+    for (int t = 0; t < len; ++t) {
+      const float v = scores[(size_t)u * n + t];
+      if (!std::isfinite(v) || v < 0.f) return HYLRA_ERR_INVALID;
+    }
+  }
+  std::vector<int32_t> order;
+  for (int u = 0; u < num_lists; ++u) {
+    const int len = lengths ? lengths[u] : n;
+    const float* sc = scores + (size_t)u * n;
+    const int kp = std::min(k, len);
+    order.resize(len);
+    for (int t = 0; t < len; ++t) order[t] = t;
+    // score descending, lower index first among equal scores
+    std::partial_sort(order.begin(), order.begin() + kp, order.end(), [sc](int32_t a, int32_t b) {
+      return sc[a] != sc[b] ? sc[a] > sc[b] : a < b;
+    });
+    int32_t* dst = topk + (size_t)u * k;
+    for (int e = 0; e < k; ++e) dst[e] = e < kp ? order[e] : -1;
+  }
+  return HYLRA_OK;
+}
+
 int hylra_dp_policy(int32_t num_layers, const double* M, double theta, uint8_t* policy,
                     int32_t* num_resets, double* cum_similarity) {
   if (num_layers < 1 || !M || !policy || std::isnan(theta)) return HYLRA_ERR_INVALID;

@@ -43,7 +43,8 @@ EXPORTS = ("hylra_workspace_bytes", "hylra_workspace_init", "hylra_decode_full",
            "hylra_version", "hylra_decode_full_noalloc", "hylra_static_policy",
            "hylra_stage_bytes", "hylra_gather_blocks", "hylra_decode_reuse_staged",
            "hylra_decode_step_offload", "hylra_overlap_counts",
-           "hylra_similarity_from_counts", "hylra_set_wait_limit")
+           "hylra_similarity_from_counts", "hylra_set_wait_limit", "hylra_token_scores",
+           "hylra_token_topk")
 
 
 class HylraError(RuntimeError):
@@ -106,6 +107,8 @@ def load() -> ctypes.CDLL:
         "hylra_decode_reuse_staged": [SP, P, P, P, P, P, P, P, S, P],
         "hylra_decode_step_offload": [SP, I32, P, P, P, P, P, P, P, P, P, P, P, S, P],
         "hylra_set_wait_limit": [I64],
+        "hylra_token_scores": [SP, P, P, P, P, P, P, P, P, S, P],
+        "hylra_token_topk": [I32, I32, P, P, I32, P],
         "hylra_strerror": [ctypes.c_int],
         "hylra_version": [],
     }
@@ -219,6 +222,26 @@ def read_status(ws, clear: bool = True, stream=None) -> int:
     _check(load().hylra_read_status(_ptr(ws), ctypes.byref(v), int(clear), _stream(stream)),
            "hylra_read_status")
     return v.value
+
+
+def token_scores(shape: Shape, q, K, V, seqlens, out, topk_out, scores, ws, stream=None):
+    """Reset layer + per-token attention mass (scores: device fp32 [B][Hkv][max_seqlen])."""
+    _check(load().hylra_token_scores(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V),
+                                     _ptr(seqlens), _ptr(out), _ptr(topk_out), _ptr(scores),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hylra_token_scores")
+
+
+def token_topk(scores: np.ndarray, k: int, lengths=None) -> np.ndarray:
+    """scores: fp32 [U, n] host array (lengths: int32 [U] valid entries or None)
+    -> int32 [U, k] indices in rank order, -1 padded."""
+    sc = np.ascontiguousarray(scores, dtype=np.float32)
+    U, n = sc.shape
+    ln = None if lengths is None else np.ascontiguousarray(lengths, dtype=np.int32)
+    out = np.zeros((U, k), dtype=np.int32)
+    _check(load().hylra_token_topk(U, n, sc.ctypes.data, None if ln is None else ln.ctypes.data,
+                                   int(k), out.ctypes.data), "hylra_token_topk")
+    return out
 
 
 def similarity(topk: np.ndarray) -> np.ndarray:

@@ -144,7 +144,9 @@ def min_gap(S32_rows, k) -> float:
 # oracle's smallest relative gap between consecutive fp32 scores of ranks
 # 1..k'+1 (oracle.topk_gap).  A set whose gap is below NEAR_TIE_REL is a
 # near tie: the kernel's fp32 sums (another summation order) may swap those
-# ranks, so such a set is reported as "near-tie, unpinned".
+# ranks, so such a set is reported as "near-tie, unpinned".  A gap of exactly
+# 0 is a tie the tests build on purpose (identical blocks): the kernel then
+# computes identical scores and the tie rule (lower block first) decides.
 CERTIFICATES: dict = {}
 
 
@@ -155,10 +157,11 @@ def check_topk_certified(config: str, got, ref, S32_h, k: int, what=""):
     gap = O.topk_gap(S32_h, k)
     assert swaps == 0 or gap < NEAR_TIE_REL, f"{what}: swap with certificate {gap}"
     c = CERTIFICATES.setdefault(config, {"sets": 0, "min_gap": math.inf, "near_ties": 0,
-                                         "swaps": 0})
+                                         "exact_ties": 0, "swaps": 0})
     c["sets"] += 1
     c["min_gap"] = min(c["min_gap"], gap)
-    c["near_ties"] += int(gap < NEAR_TIE_REL)
+    c["near_ties"] += int(0.0 < gap < NEAR_TIE_REL)
+    c["exact_ties"] += int(gap == 0.0)
     c["swaps"] += swaps
     return swaps
 
@@ -167,9 +170,11 @@ def certificate_lines():
     out = []
     for name in sorted(CERTIFICATES):
         c = CERTIFICATES[name]
-        state = ("near-tie, unpinned" if c["near_ties"] else "pinned")
+        state = "near-tie, unpinned" if c["near_ties"] else "pinned"
+        ties = (f", {c['exact_ties']} sets with exactly equal scores (tie rule)"
+                if c["exact_ties"] else "")
         out.append(f"{name}: {c['sets']} index sets, min relative gap {c['min_gap']:.3g}, "
-                   f"{c['near_ties']} near-tie sets, {c['swaps']} swaps ({state})")
+                   f"{c['near_ties']} near-tie sets{ties}, {c['swaps']} swaps ({state})")
     return out
 
 

@@ -582,3 +582,50 @@ def test_bounded_waits_give_up_and_the_workspace_recovers():
         for a, b in zip(outs, ref[0]):
             assert torch.equal(a, b)
         assert torch.equal(tk, ref[1])
+
+
+TOKEN_CASES = [
+    W.custom("tok_dense", batch=2, seqlens=(3000, 700), num_q_heads=8, num_kv_heads=2, topk=6,
+             seed=61),
+    W.custom("tok_packed_r1", batch=3, seqlens=(1300, 129, 2500), num_q_heads=4, num_kv_heads=4,
+             topk=5, packed=True, seed=62),
+    W.custom("tok_fp32", batch=1, seqlens=(1000,), num_q_heads=8, num_kv_heads=2, topk=4,
+             dtype="fp32", structure="iid", seed=63),
+]
+# Token masses: fp32 logits of 128 products (absolute error ~1e-5 in the
+# log2 domain, i.e. ~1e-5 relative in the probability), a head sum built from
+# the blocks' fp32 records and a hardware exp2: 1e-4 relative is ten times that.
+TOKEN_RTOL = 1e-4
+
+
+@pytest.mark.parametrize("w", TOKEN_CASES, ids=lambda w: w.name)
+def test_token_scores_match_oracle(w):
+    """Token-level profiling: per-token attention mass against the oracle;
+    the host selection on the GPU's scores against the oracle's ranking rule
+    (exact), and the selected tokens valid against the oracle's own scores."""
+    run = T.Runner(w)
+    q, K, V = _layer(w, 0)
+    out_ref, tk_ref = run.full(q, K, V)
+    assert run.status() == 0
+    out, tk = run.new_out(), run.new_topk()
+    scores = torch.full((w.batch, w.num_kv_heads, w.max_seqlen), float("nan"), device="cuda")
+    H.token_scores(run.shape, q, K, V, run.seqlens, out, tk, scores, run.ws)
+    assert run.status() == 0
+    assert torch.equal(out, out_ref) and torch.equal(tk, tk_ref)
+    sc = scores.cpu().numpy()
+    ktok = 128 * w.topk
+    for b in range(w.batch):
+        n = w.seqlens[b]
+        S32, _ = O.layer_token_topk(q[b].double().cpu().numpy(), T.seq_arrays(w, K, b), n, ktok)
+        assert np.all(sc[b, :, n:] == 0.0)
+        np.testing.assert_allclose(sc[b, :, :n], S32, rtol=TOKEN_RTOL, atol=1e-12)
+        got = H.token_topk(sc[b, :, :n], ktok)
+        for h in range(w.num_kv_heads):
+            assert np.array_equal(got[h], O.topk_blocks(sc[b, h, :n], ktok))
+            # valid against the oracle: no chosen token scores clearly below a
+            # token left out
+            kp = min(ktok, n)
+            chosen = S32[h][got[h][:kp]].astype(np.float64)
+            left = np.delete(S32[h], got[h][:kp]).astype(np.float64)
+            if left.size:
+                assert chosen.min() >= left.max() * (1 - 2 * TOKEN_RTOL)

@@ -235,3 +235,30 @@ def test_trace_build_compiles_and_exports_its_hooks(tmp_path):
     for name in ("hylra_trace_set", "hylra_plan_override", "hylra_late_override",
                  "hylra_decode_step"):
         assert hasattr(tl, name), name
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_token_topk_matches_oracle_ranking(lib, seed):
+    """Host token selection against the oracle's ranking rule on the same
+    fp32 scores (many exact ties: scores drawn from a few values)."""
+    rng = np.random.default_rng(70 + seed)
+    U, n, k = 6, 300, int(rng.integers(1, 40))
+    scores = rng.choice(np.array([0.0, 0.125, 0.5, 0.75, 1e-7], dtype=np.float32), size=(U, n))
+    scores[1] = rng.random(n).astype(np.float32)
+    lengths = rng.integers(0, n + 1, size=U).astype(np.int32)
+    lengths[0] = n
+    got = H.token_topk(scores, k, lengths)
+    for u in range(U):
+        want = O.topk_blocks(scores[u, :lengths[u]], k)
+        assert np.array_equal(got[u], want), u
+    assert np.array_equal(H.token_topk(scores, k), np.stack([O.topk_blocks(s, k) for s in scores]))
+
+
+def test_token_topk_rejects_bad_scores(lib):
+    for bad in (np.nan, np.inf, -1.0):
+        s = np.zeros((2, 5), dtype=np.float32)
+        s[1, 3] = bad
+        with pytest.raises(H.HylraError):
+            H.token_topk(s, 2)
+    with pytest.raises(H.HylraError):
+        H.token_topk(np.zeros((1, 5), dtype=np.float32), 2, lengths=np.array([6], dtype=np.int32))
