@@ -428,7 +428,7 @@ def offload_measure(m: Model, H, policy, steps, warmup, dist_on):
         else:
             Ko.append(m.Ks[l])
             Vo.append(m.Vs[l])
-    n = H.stage_bytes(m.shape) // 2
+    n = H.stage_bytes(m.shape)  # bytes of one slot = bf16 elements of the two slots
     Ks = torch.empty(n, dtype=torch.bfloat16, device="cuda")
     Vs = torch.empty(n, dtype=torch.bfloat16, device="cuda")
     s = torch.cuda.Stream()

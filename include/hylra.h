@@ -179,10 +179,19 @@ int hylra_decode_reuse_staged(const hylra_shape_t* shape, const void* q, const v
                               size_t workspace_bytes, hylra_stream_t stream);
 
 /* hylra_decode_step where offloaded[l] == 1 marks a reuse layer whose K[l],
- * V[l] are host-resident: the layer gathers its reused blocks into K_stage /
- * V_stage (one pair, reused layer after layer) and runs on them.  Reset
- * layers must be device-resident (HYLRA_ERR_INVALID otherwise).  offloaded:
- * HOST uint8 [num_layers]. */
+ * V[l] are host-resident.  K_stage and V_stage (device) each hold TWO
+ * staging slots of hylra_stage_bytes; the offloaded layers use them in turn.
+ * A second stream owned by the library (one per host thread and device,
+ * created by the thread's first call, which should therefore not be inside a
+ * stream capture) prefetches: each offloaded layer's reused blocks cross the
+ * host link as soon as the indices it reuses exist (its reset layer is done)
+ * and its slot is free (the offloaded layer two before it is done), while
+ * the layers run.  The block holding each sequence's newest token is copied
+ * again after the preceding layer (in a model that layer writes the newest
+ * row), then the layer runs on its slot.  `stream` waits for the second
+ * stream at the end; capturable in a CUDA graph.  Reset layers must be
+ * device-resident (HYLRA_ERR_INVALID otherwise).  offloaded: HOST uint8
+ * [num_layers].  bf16 only. */
 int hylra_decode_step_offload(const hylra_shape_t* shape, int32_t num_layers,
                               const uint8_t* policy, const void* const* q,
                               const void* const* K, const void* const* V,

@@ -427,7 +427,8 @@ int check_stage_rows(const hylra_shape_t* s) {
 
 // Copy the listed blocks of a host-resident cache into a staging cache.
 int gather(const hylra_shape_t* s, const void* Kh, const void* Vh, const int32_t* seqlens,
-           const int32_t* topk_in, void* Ks, void* Vs, cudaStream_t stream, bool pdl) {
+           const int32_t* topk_in, void* Ks, void* Vs, cudaStream_t stream, bool pdl,
+           bool newest_only = false) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (s->dtype != HYLRA_BF16) return HYLRA_ERR_UNSUPPORTED;
@@ -452,6 +453,7 @@ int gather(const hylra_shape_t* s, const void* Kh, const void* Vh, const int32_t
   p.max_seqlen = s->max_seqlen;
   // status bits of a bad length are left to the reuse kernel that follows
   p.status = nullptr;
+  p.newest_only = newest_only ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s->batch * s->num_kv_heads, s->topk);
   cfg.blockDim = dim3(NT_GATHER);
@@ -475,6 +477,9 @@ struct LayerHooks {
   int (*before)(void* ctx, int layer);
   int (*after)(void* ctx, int layer);
   void* ctx;
+  // an offloaded reuse layer (index-guided offloading), given the layer of
+  // the indices it reuses; sets *prev_ctas like launch()
+  int (*offloaded)(void* ctx, int layer, int reset_layer, int* prev_ctas) = nullptr;
 };
 
 int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,
@@ -504,13 +509,8 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
                   workspace, workspace_bytes, stream, l > 0, true, l & 63, prev_ctas,
                   &prev_ctas);
     } else if (offloaded && offloaded[l]) {
-      // index-guided offloading: only the reused blocks cross the host link
-      const int32_t* idx = topk + last_reset * per_layer;
-      rc = gather(shape, K[l], V[l], seqlens, idx, K_stage, V_stage, stream, true);
-      if (!rc)
-        rc = launch(shape, false, q[l], K_stage, V_stage, seqlens, idx, out[l], nullptr,
-                    workspace, workspace_bytes, stream, true, true, l & 63, 0, &prev_ctas,
-                    true);
+      rc = hooks && hooks->offloaded ? hooks->offloaded(hooks->ctx, l, last_reset, &prev_ctas)
+                                     : HYLRA_ERR_INVALID;
     } else {
       rc = launch(shape, false, q[l], K[l], V[l], seqlens, topk + last_reset * per_layer, out[l],
                   nullptr, workspace, workspace_bytes, stream, l > 0, last_reset == l - 1,
@@ -617,6 +617,115 @@ int host_pipe_after(void* ctx, int layer) {
 }
 
 
+
+// Index-guided offloading with prefetch.  A second stream (one per host
+// thread and device) gathers each offloaded layer's reused blocks from host
+// memory into one of two staging slots as soon as the indices it reuses exist
+// (its reset layer is done) and the slot is free (the layer that used it two
+// offloaded layers earlier is done), so the link works while the layers run.
+// The block holding each sequence's newest token is written by the preceding
+// layer in a model: after that layer the caller's stream copies only those
+// blocks again, then runs the reuse layer on the slot.
+struct OffloadPipe {
+  const hylra_shape_t* shape = nullptr;
+  cudaStream_t main = nullptr, copy = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_reset = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_used[2] = {nullptr, nullptr}, ev_gathered[2] = {nullptr, nullptr};
+  const uint8_t* policy = nullptr;
+  const void* const* q = nullptr;
+  const void* const* K = nullptr;
+  const void* const* V = nullptr;
+  const int32_t* seqlens = nullptr;
+  float* const* out = nullptr;
+  const int32_t* topk = nullptr;
+  uint8_t* K_stage = nullptr;
+  uint8_t* V_stage = nullptr;
+  size_t slot_bytes = 0, per_layer = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  std::vector<int> order;     // offloaded layers in order
+  std::vector<int> pos_of;    // layer -> its place in `order` (-1: not offloaded)
+  std::vector<int> reset_of;  // layer -> the reset layer whose indices it reuses
+  int next = 0;               // next entry of `order` to gather
+};
+
+int offload_pipe_resources(OffloadPipe* op) {
+  struct Res {
+    cudaStream_t copy = nullptr;
+    cudaEvent_t ev[7] = {};
+  };
+  thread_local std::vector<Res> per_dev;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HYLRA_ERR_CUDA;
+  if ((int)per_dev.size() <= dev) per_dev.resize(dev + 1);
+  Res& r = per_dev[dev];
+  if (!r.copy) {
+    if (cudaStreamCreateWithFlags(&r.copy, cudaStreamNonBlocking) != cudaSuccess) {
+      r.copy = nullptr;
+      return HYLRA_ERR_CUDA;
+    }
+    for (auto& e : r.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return HYLRA_ERR_CUDA;
+  }
+  op->copy = r.copy;
+  op->ev_fork = r.ev[0];
+  op->ev_reset = r.ev[1];
+  op->ev_join = r.ev[2];
+  op->ev_used[0] = r.ev[3];
+  op->ev_used[1] = r.ev[4];
+  op->ev_gathered[0] = r.ev[5];
+  op->ev_gathered[1] = r.ev[6];
+  return HYLRA_OK;
+}
+
+// Gather every offloaded layer that can go now: layers < enq have been
+// enqueued on the caller's stream.
+int offload_pump(OffloadPipe* op, int enq) {
+  while (op->next < (int)op->order.size()) {
+    const int pos = op->next, j = op->order[pos], slot = pos & 1;
+    const int i = op->reset_of[j];
+    if (i >= enq) break;                                      // indices not enqueued yet
+    if (pos >= 2 && op->order[pos - 2] >= enq) break;         // slot's last user not enqueued
+    if (pos >= 2 && cudaStreamWaitEvent(op->copy, op->ev_used[slot], 0) != cudaSuccess)
+      return HYLRA_ERR_CUDA;
+    // ev_reset holds the record of reset layer i: a later reset would lie
+    // between i and j, and j would reuse its indices instead
+    if (cudaStreamWaitEvent(op->copy, op->ev_reset, 0) != cudaSuccess) return HYLRA_ERR_CUDA;
+    int rc = gather(op->shape, op->K[j], op->V[j], op->seqlens, op->topk + i * op->per_layer,
+                    op->K_stage + slot * op->slot_bytes, op->V_stage + slot * op->slot_bytes,
+                    op->copy, false);
+    if (rc) return rc;
+    if (cudaEventRecord(op->ev_gathered[slot], op->copy) != cudaSuccess) return HYLRA_ERR_CUDA;
+    ++op->next;
+  }
+  return HYLRA_OK;
+}
+
+int offload_before(void* ctx, int layer) { return offload_pump(static_cast<OffloadPipe*>(ctx), layer); }
+
+int offload_after(void* ctx, int layer) {
+  OffloadPipe* op = static_cast<OffloadPipe*>(ctx);
+  if (op->policy[layer] && cudaEventRecord(op->ev_reset, op->main) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return offload_pump(op, layer + 1);
+}
+
+int offload_layer(void* ctx, int l, int reset_layer, int* prev_ctas) {
+  OffloadPipe* op = static_cast<OffloadPipe*>(ctx);
+  const int pos = op->pos_of[l], slot = pos & 1;
+  if (pos < 0 || pos >= op->next) return HYLRA_ERR_INVALID;  // not gathered (cannot happen)
+  const int32_t* idx = op->topk + reset_layer * op->per_layer;
+  uint8_t* Ks = op->K_stage + slot * op->slot_bytes;
+  uint8_t* Vs = op->V_stage + slot * op->slot_bytes;
+  if (cudaStreamWaitEvent(op->main, op->ev_gathered[slot], 0) != cudaSuccess) return HYLRA_ERR_CUDA;
+  // the newest token's block, after the preceding layer
+  int rc = gather(op->shape, op->K[l], op->V[l], op->seqlens, idx, Ks, Vs, op->main, true, true);
+  if (!rc)
+    rc = launch(op->shape, false, op->q[l], Ks, Vs, op->seqlens, idx, op->out[l], nullptr, op->ws,
+                op->ws_bytes, op->main, true, true, l & 63, 0, prev_ctas, true);
+  if (rc) return rc;
+  return cudaEventRecord(op->ev_used[slot], op->main) == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -756,9 +865,52 @@ int hylra_decode_step_offload(const hylra_shape_t* shape, int32_t num_layers,
                               const uint8_t* offloaded, const int32_t* seqlens,
                               float* const* out, int32_t* topk, void* K_stage, void* V_stage,
                               void* workspace, size_t workspace_bytes, hylra_stream_t stream) {
-  if (!offloaded || !K_stage || !V_stage) return HYLRA_ERR_INVALID;
-  return run_step(shape, num_layers, policy, q, K, V, offloaded, seqlens, out, topk, K_stage,
-                  V_stage, workspace, workspace_bytes, (cudaStream_t)stream);
+  if (!offloaded || !K_stage || !V_stage || !policy || !K || !V || num_layers < 1)
+    return HYLRA_ERR_INVALID;
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (shape->dtype != HYLRA_BF16) return HYLRA_ERR_UNSUPPORTED;
+  if ((rc = check_stage_rows(shape))) return rc;
+  if (!aligned(K_stage, 16) || !aligned(V_stage, 16)) return HYLRA_ERR_INVALID;
+  OffloadPipe op;
+  if ((rc = offload_pipe_resources(&op))) return rc;
+  op.shape = shape;
+  op.main = (cudaStream_t)stream;
+  op.policy = policy;
+  op.q = q;
+  op.K = K;
+  op.V = V;
+  op.seqlens = seqlens;
+  op.out = out;
+  op.topk = topk;
+  op.K_stage = static_cast<uint8_t*>(K_stage);
+  op.V_stage = static_cast<uint8_t*>(V_stage);
+  op.slot_bytes = stage_bytes(shape);
+  op.per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
+  op.ws = workspace;
+  op.ws_bytes = workspace_bytes;
+  op.pos_of.assign(num_layers, -1);
+  op.reset_of.assign(num_layers, 0);
+  for (int l = 0, last = 0; l < num_layers; ++l) {
+    if (policy[l] == 1) last = l;
+    op.reset_of[l] = last;
+    if (offloaded[l] == 1 && policy[l] == 0) {
+      op.pos_of[l] = (int)op.order.size();
+      op.order.push_back(l);
+    }
+  }
+  // the copy stream starts after the caller's earlier work and rejoins it
+  if (cudaEventRecord(op.ev_fork, op.main) != cudaSuccess ||
+      cudaStreamWaitEvent(op.copy, op.ev_fork, 0) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  LayerHooks hooks{offload_before, offload_after, &op};
+  hooks.offloaded = offload_layer;
+  rc = run_step(shape, num_layers, policy, q, K, V, offloaded, seqlens, out, topk, K_stage,
+                V_stage, workspace, workspace_bytes, op.main, &hooks);
+  if (cudaEventRecord(op.ev_join, op.copy) != cudaSuccess ||
+      cudaStreamWaitEvent(op.main, op.ev_join, 0) != cudaSuccess)
+    return HYLRA_ERR_CUDA;
+  return rc;
 }
 
 int hylra_decode_step_host(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* policy,

@@ -125,6 +125,7 @@ struct Params {
   long long total;  // packed rows per KV-head plane
   int B, Hq, Hkv, r, k, max_seqlen, nbmax;
   int idx_wait;      // reuse: topk_in is written by the immediately preceding kernel
+  int newest_only;   // block gather: copy only the block holding each sequence's newest token
   int staged;        // reuse: K/V are a staging cache [B][Hkv][k][128][d] whose slot e holds
                      // block topk_in[b][h][e] (written by gather_blocks_kernel)
   int late_from;     // bf16 streaming kernel: CTAs >= late_from start late (their SM is
@@ -2268,6 +2269,7 @@ __global__ void __launch_bounds__(NT_GATHER) gather_blocks_kernel(const __grid_c
   if (e >= min(p.k, nb)) return;
   const int blk = __ldcg(p.topk_in + (size_t)bh * p.k + e);
   if (blk < 0 || blk >= nb) return;  // flagged by the reuse kernel
+  if (p.newest_only && blk != nb - 1) return;
   const int rows = min(BLK, seqlen - blk * BLK);
   const long long src_row = row_base(p, b, h) + (long long)blk * BLK;
   const long long dst_row = ((long long)bh * p.k + e) * BLK;

@@ -88,13 +88,34 @@ def test_staged_reuse_skips_unused_and_invalid_slots():
     assert torch.equal(out, ref)
 
 
-def test_offloaded_step_equals_device_step():
-    w = W.custom("off_step", batch=2, layers=7, seqlens=(6000, 2600), num_q_heads=32,
+def _stage2(run):
+    """Two staging slots each for K and V (the offloaded step's prefetch)."""
+    n = H.stage_bytes(run.shape)  # bytes of one slot = elements of two bf16 slots
+    return (torch.empty(n, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(n, dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.parametrize("policy,offloaded", [
+    ((1, 0, 0, 1, 0, 0, 0), (0, 1, 1, 0, 1, 1, 1)),
+    # slots reused several times, a device-resident reuse layer between
+    # offloaded ones, two reset layers in a row
+    ((1, 0, 0, 0, 1, 1, 0, 0, 0, 0), (0, 1, 0, 1, 0, 0, 1, 1, 1, 1)),
+])
+def test_offloaded_step_equals_device_step(policy, offloaded):
+    """The prefetching offloaded step equals the device-resident step bit for
+    bit, eagerly and replayed from a CUDA graph.  Layer 0 makes each
+    sequence's newest block rank first, so the offloaded layers copy it again
+    after their preceding layer."""
+    L = len(policy)
+    w = W.custom("off_step", batch=2, layers=L, seqlens=(6000, 2600 - 31), num_q_heads=32,
                  num_kv_heads=8, topk=16, seed=45)
-    policy = (1, 0, 0, 1, 0, 0, 0)
-    offloaded = tuple(0 if p else 1 for p in policy)
     run = T.Runner(w)
-    layers = [W.layer_inputs(w, l, "cpu") for l in range(w.layers)]
+    layers = [list(W.layer_inputs(w, l, "cpu")) for l in range(w.layers)]
+    u = W.structure(w).u
+    for b, n in enumerate(w.seqlens):
+        last = (n - 1) // 128 * 128
+        K0 = layers[0][1]
+        K0[b, :, last:n] = (K0[b, :, last:n].float() + 9.0 * u[b][:, None, :]).to(K0.dtype)
     qs = [l[0].cuda() for l in layers]
     Kd = [l[1].cuda() for l in layers]
     Vd = [l[2].cuda() for l in layers]
@@ -107,13 +128,31 @@ def test_offloaded_step_equals_device_step():
     Vo = [Vd[l] if not offloaded[l] else _pinned(layers[l][2]) for l in range(w.layers)]
     outs_o = [run.new_out() for _ in range(w.layers)]
     topk_o = torch.full_like(topk_d, -7)
-    Ks, Vs = _stage(run)
+    Ks, Vs = _stage2(run)
     H.decode_step_offload(run.shape, policy, qs, Ko, Vo, offloaded, run.seqlens, outs_o,
                           topk_o, Ks, Vs, run.ws)
     assert run.status() == 0
     assert torch.equal(topk_o, topk_d)
+    assert np.all(topk_d[0, :, :, 0].cpu().numpy() == np.array([[(n - 1) // 128] * 8
+                                                                for n in w.seqlens]))
     for l in range(w.layers):
         assert torch.equal(outs_o[l], outs_d[l]), f"layer {l}"
+    # replayed from a CUDA graph (the copy stream's work becomes graph nodes)
+    for o in outs_o:
+        o.fill_(float("nan"))
+    topk_o.fill_(-7)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        H.decode_step_offload(run.shape, policy, qs, Ko, Vo, offloaded, run.seqlens, outs_o,
+                              topk_o, Ks, Vs, run.ws, stream=torch.cuda.current_stream())
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    assert torch.equal(topk_o, topk_d)
+    for l in range(w.layers):
+        assert torch.equal(outs_o[l], outs_d[l]), f"graph layer {l}"
 
 
 def test_offloaded_reset_layer_is_rejected():
@@ -121,7 +160,7 @@ def test_offloaded_reset_layer_is_rejected():
                  topk=4, seed=46)
     run = T.Runner(w)
     layers = [_ for _ in (W.layer_inputs(w, l, "cuda") for l in range(2))]
-    Ks, Vs = _stage(run)
+    Ks, Vs = _stage2(run)
     outs = [run.new_out() for _ in range(2)]
     topk = torch.full((2, 1, 2, 4), -1, dtype=torch.int32, device="cuda")
     with pytest.raises(H.HylraError) as e:
