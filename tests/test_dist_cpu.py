@@ -111,3 +111,27 @@ def test_single_process_fallbacks():
     assert D.max_over_ranks(2.0) == 2.0
     assert list(D.shard(5, 0, 1)) == list(range(5))
     assert [len(D.shard(10, r, 4)) for r in range(4)] == [2, 3, 2, 3]
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_head_shards_hold_the_whole_layers_values(packed):
+    """A rank's KV-head shard of a layer (and of a later step's query) is the
+    same slice of values as in the whole layer, so sharded ranks compute
+    exactly what one GPU computes for those heads."""
+    from kv_cache_sparsity_b200 import workloads as W
+    w = W.custom("shard", batch=2, layers=2, seqlens=(300, 129), num_q_heads=8,
+                 num_kv_heads=4, topk=2, packed=packed, seed=9)
+    q, K, V = W.layer_inputs(w, 1)
+    for world in (2, 4):
+        for rank in range(world):
+            heads = D.shard(w.num_kv_heads, rank, world)
+            qs, Ks, Vs = W.layer_inputs(w, 1, heads=heads)
+            sl = slice(heads.start * w.group, heads.stop * w.group)
+            assert torch.equal(qs, q[:, sl])
+            if packed:
+                assert torch.equal(Ks, K[heads.start:heads.stop])
+                assert torch.equal(Vs, V[heads.start:heads.stop])
+            else:
+                assert torch.equal(Ks, K[:, heads.start:heads.stop])
+                assert torch.equal(Vs, V[:, heads.start:heads.stop])
+            assert torch.equal(W.step_query(w, 1, 2, heads=heads), W.step_query(w, 1, 2)[:, sl])
