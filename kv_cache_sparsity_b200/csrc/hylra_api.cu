@@ -261,6 +261,11 @@ bool plan_reuse_cluster(const hylra_shape_t* s, RCPlan* out) {
     if (pl.nst < 1) continue;
     const int n = rc_max_active(pl);
     if (n >= nbh || (cs == 1 && n > 0)) {
+      // A large layer (8 or more blocks per SM) whose clusters would leave
+      // more than a tenth of the SMs idle (one CTA per SM) streams faster
+      // over every SM with the cross-CTA merge kernel (B200: 8 x 64K and
+      // the ragged 16-sequence batch, 3-6 % per reuse layer).
+      if ((long long)nbh * kmax >= 8LL * sms && 10LL * pl.cs * nbh < 9LL * sms) return false;
       *out = pl;
       return true;
     }

@@ -51,8 +51,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (mbarrier.try_wait instead may suspend the
+// thread inside the instruction until the phase completes or a hardware time
+// limit passes).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Default limit of a bounded wait: ~2^31 SM clocks (about a second).
 constexpr long long WAIT_LIMIT_DEFAULT = 1ll << 31;
+// Limits below this (a watchdog set short, as tests do) poll with test_wait
+// and read the clock on every poll, so the limit holds to a few clocks.
+constexpr long long WAIT_LIMIT_POLL = 1ll << 16;
 // Limit of a drain (waiting for a CTA's own copies in flight before it exits).
 constexpr long long DRAIN_LIMIT = 1ll << 31;
 
@@ -65,6 +83,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
                                                   volatile int* abort,
                                                   long long limit = WAIT_LIMIT_DEFAULT) {
   if (*abort) return false;
+  if (limit < WAIT_LIMIT_POLL) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        *abort = 1;
+        return false;
+      }
+    }
+    return true;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
@@ -294,9 +323,32 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0u;
 }
 
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
                                                           volatile int* abort,
                                                           long long limit = WAIT_LIMIT_DEFAULT) {
+  if (limit < WAIT_LIMIT_POLL) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait_cluster(bar, parity)) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        *abort = 1;
+        return false;
+      }
+    }
+    return true;
+  }
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
