@@ -11,11 +11,14 @@ step streams more bytes than the 126 MB L2 holds.  The default workload is
 the largest one that fits one GPU (ragged16: 16 sequences of 8K-128K tokens,
 all 32 layer caches resident).
 
-With N GPUs (torchrun), rank r holds the KV heads shard(Hkv, r, N) of every
-sequence: one fixed workload split N ways ("scaling": "strong"), no
-collective in the step; the profiled overlap matrix is pooled exactly over
-the ranks (integer counts, one all-reduce), so every rank runs the policy a
-single GPU derives.
+With N GPUs (torchrun) there is no collective in the step.  Default
+(--shard batch, "scaling": "weak"): one global batch of N x B sequences,
+rank r running its own B (the configured workload's shapes, its own seed;
+rank 0's is the configured workload) under the policy rank 0 derives, which
+every rank receives.  --shard heads ("scaling": "strong"): rank r holds the
+KV heads shard(Hkv, r, N) of every sequence of the one workload, and the
+profiled overlap matrix is pooled exactly over the ranks (integer counts, one
+all-reduce), so every rank runs the policy a single GPU derives.
 
 value        = device time per hybrid decode step (us), max over ranks
 e2e          = the same step through the C-ABI host-buffer entry point
@@ -269,6 +272,12 @@ def step_bytes(w: W.Workload, policy) -> int:
     return R * w.kv_bytes_per_layer() + (w.layers - R) * w.kv_bytes_reuse_layer()
 
 
+def parallelism(args, world: int) -> str:
+    if args.shard == "heads":
+        return f"kv-head shards x{world}"
+    return f"sequence shards x{world} (each GPU its own batch of the workload)"
+
+
 def config_of(w: W.Workload, policy, args, world: int) -> dict:
     """The workload as both arms name it (the same keys and values)."""
     return {
@@ -277,7 +286,7 @@ def config_of(w: W.Workload, policy, args, world: int) -> dict:
         "policy_rule": policy_rule(args, w),
         "resets": int(sum(policy)),
         "l2": "inputs larger than L2: a step streams %.2f GB" % (step_bytes(w, policy) / 1e9),
-        "parallelism": f"kv-head shards x{world}",
+        "parallelism": parallelism(args, world),
     }
 
 
@@ -299,7 +308,7 @@ def profile_layer_sets(m: Model, H, q, K, V, token_topk: int) -> np.ndarray:
 
 
 def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int = 1,
-                  profile_seeds: int = 1, token_topk: int = 0):
+                  profile_seeds: int = 1, token_topk: int = 0, pooled: bool = True):
     """The step's reset/reuse policy.
 
     dp: profiling run(s) with every layer full -> overlap matrix -> DP policy
@@ -340,7 +349,8 @@ def derive_policy(m: Model, H, rule: str = "dp", theta=None, profile_steps: int 
             del q, K, V
         sets.append(np.stack(per_layer))
         torch.cuda.empty_cache()
-    M = D.pooled_similarity(H, np.concatenate(sets, axis=1), device="cuda")
+    sets = np.concatenate(sets, axis=1)
+    M = D.pooled_similarity(H, sets, device="cuda") if pooled else H.similarity(sets)
     pol, R, S = H.dp_policy(M, w.theta if theta is None else theta)
     return pol, M
 
@@ -521,18 +531,31 @@ def run_ours(args, rank, world, dist_on):
     from kv_cache_sparsity_b200 import hylra as H
     hbuild.build()
     H.load()
-    w = W.config(args.config)
-    heads = D.shard(w.num_kv_heads, rank, world)
-    if len(heads) == 0:
-        raise SystemExit(f"{world} ranks for {w.num_kv_heads} KV heads: a rank would hold none")
+    w0 = W.config(args.config)
+    if args.shard == "heads":
+        w, heads = w0, D.shard(w0.num_kv_heads, rank, world)
+        if len(heads) == 0:
+            raise SystemExit(f"{world} ranks for {w0.num_kv_heads} KV heads: a rank would hold none")
+    else:
+        # rank r: its own batch of the global batch (rank 0: the configured workload)
+        w, heads = seed_variant(w0, rank), range(w0.num_kv_heads)
     free = torch.cuda.mem_get_info()[0]
     per_layer = w.kv_bytes_per_layer() * len(heads) // w.num_kv_heads  # K and V on this GPU
     resident = w.layers
     if per_layer * w.layers > free * 0.85:
         resident = max(1, int(free * 0.85 // per_layer))
     m = Model(w, H, resident, heads)
-    policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps,
-                              args.profile_seeds, args.token_topk)
+    if args.shard == "heads":
+        # every rank profiles its heads; the counts are pooled over the ranks
+        policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps,
+                                  args.profile_seeds, args.token_topk)
+    else:
+        # the configured workload's policy (rank 0's), the same on every rank
+        policy = None
+        if rank == 0:
+            policy, M = derive_policy(m, H, args.policy, args.theta, args.profile_steps,
+                                      args.profile_seeds, args.token_topk, pooled=False)
+        policy = D.broadcast_policy(policy, device="cuda")
     L = w.layers
     allfull = (1,) * L
     one_then_reuse = (1,) + (0,) * (L - 1)
@@ -580,7 +603,9 @@ def run_ours(args, rank, world, dist_on):
                if args.offload else None)
 
     peak, peak_kind = measured_hbm_peak()
-    job_bytes = step_bytes(w, policy)
+    # the whole job: every rank's batch (sequence shards) or the one workload
+    job_batches = world if args.shard == "batch" else 1
+    job_bytes = step_bytes(w, policy) * job_batches
     us_h = ms_h * 1000.0
     kv_gbs = job_bytes / (ms_h * 1e-3) / 1e9
     full_b, reuse_b = m.full_bytes(), m.reuse_bytes()
@@ -603,7 +628,7 @@ def run_ours(args, rank, world, dist_on):
         "warmup": args.warmup,
         "ms_per_step": round(ms_h, 6),
         "higher_is_better": False,
-        "scaling": "strong",
+        "scaling": "weak" if args.shard == "batch" else "strong",
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
@@ -615,7 +640,7 @@ def run_ours(args, rank, world, dist_on):
         "kv_frac_of_8tbs": round(kv_gbs / NOMINAL_HBM_GBS, 4),
         "full_us_per_step": round(ms_f * 1000.0, 3),
         "speedup_vs_full": round(ms_f / ms_h, 4),
-        "sequences_per_s": round(w.batch / (ms_h * 1e-3), 1),
+        "sequences_per_s": round(job_batches * w.batch / (ms_h * 1e-3), 1),
         "reset_layer": layer_rate(full_b, reset_us),
         "reuse_layer": dict(layer_rate(reuse_b, reuse_us),
                             how="(one reset + %d reuse layers) - (one reset layer), per reuse "
@@ -725,7 +750,7 @@ def run_reference(args, world):
         "warmup": args.warmup,
         "ms_per_step": round(us / 1000.0, 3),
         "higher_is_better": False,
-        "scaling": "strong",
+        "scaling": "weak" if args.shard == "batch" else "strong",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded salient-block K, iid V; see workloads.py)",
@@ -758,6 +783,9 @@ def main():
                     help="decode steps pooled into the profiled overlap matrix")
     ap.add_argument("--profile-seeds", type=int, default=1,
                     help="synthetic workloads (seeds) pooled into the profiled overlap matrix")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="N GPUs: batch = each GPU its own batch (weak), heads = KV heads of one "
+                         "workload split over the GPUs (strong)")
     ap.add_argument("--token-topk", type=int, default=0,
                     help="profile top-k tokens (this many per head) instead of top-k blocks")
     ap.add_argument("--no-clock-fill", action="store_true",

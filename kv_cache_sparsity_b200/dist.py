@@ -1,14 +1,19 @@
 """Host-side helpers for running one process per GPU.
 
-The decode path splits by KV head with no exchange step in the data path:
-every (sequence, KV head) pair is independent through full attention, block
-scoring, top-k and reuse attention, so rank r holds the KV heads
-``shard(Hkv, r, world)`` of every sequence (and their query heads) and runs
-the whole step on them.  The only data crossing ranks is in the offline
-profiling: the overlap matrix is a ratio of two integer sums over index sets
-(hylra_overlap_counts), so the ranks add their counts with one integer
-all-reduce and every rank derives the same matrix, and the same policy, as a
-single GPU holding every head.  Timing is max-reduced over ranks.
+Every (sequence, KV head) pair is independent through full attention, block
+scoring, top-k and reuse attention, so the decode path splits across GPUs
+with no exchange step in the data path, in either of two ways:
+
+* by sequence (weak scaling): rank r runs its own batch of sequences of one
+  global batch, every KV head of them; the policy of the configured workload
+  (rank 0's) is broadcast, so every rank runs the same layers;
+* by KV head (strong scaling): rank r holds the KV heads ``shard(Hkv, r,
+  world)`` of every sequence of one workload.  The overlap matrix is a ratio
+  of two integer sums over index sets (hylra_overlap_counts), so the ranks add
+  their counts with one integer all-reduce and every rank derives the same
+  matrix, and the same policy, as a single GPU holding every head.
+
+Timing is max-reduced over ranks.
 """
 
 from __future__ import annotations
@@ -79,3 +84,17 @@ def pooled_similarity(H, sets: np.ndarray, device="cpu") -> np.ndarray:
     inter, total = H.overlap_counts(sets)
     inter, total = sum_over_ranks(inter, total, device=device)
     return H.similarity_from_counts(inter, total)
+
+
+def broadcast_policy(policy, device="cpu"):
+    """Rank 0's policy on every rank (the policy itself when not distributed).
+    Every rank calls this once; ranks other than 0 may pass None."""
+    if not dist_on():
+        return tuple(int(x) for x in policy)
+    n = torch.tensor([len(policy) if policy is not None else 0], dtype=torch.int64, device=device)
+    torch.distributed.broadcast(n, src=0)
+    t = torch.zeros(int(n.item()), dtype=torch.int64, device=device)
+    if torch.distributed.get_rank() == 0:
+        t.copy_(torch.tensor([int(x) for x in policy], dtype=torch.int64))
+    torch.distributed.broadcast(t, src=0)
+    return tuple(int(x) for x in t.cpu().tolist())

@@ -34,6 +34,9 @@ def _worker(rank, world, port, q):
         got = D.max_over_ranks(1.5 + rank * 2.25)
         D.barrier()
         shard = list(D.shard(7, rank, world))
+        # rank 0's policy reaches every rank (sequence shards run the same layers)
+        pol = D.broadcast_policy((1, 0, 0, 1, 0) if rank == 0 else None)
+        assert pol == (1, 0, 0, 1, 0)
         q.put((rank, got, shard))
     finally:
         torch.distributed.destroy_process_group()
@@ -108,6 +111,7 @@ def test_two_ranks_pool_the_overlap_matrix_exactly():
 
 def test_single_process_fallbacks():
     assert not D.dist_on()
+    assert D.broadcast_policy([1, 0, 1]) == (1, 0, 1)
     assert D.max_over_ranks(2.0) == 2.0
     assert list(D.shard(5, 0, 1)) == list(range(5))
     assert [len(D.shard(10, r, 4)) for r in range(4)] == [2, 3, 2, 3]
