@@ -315,9 +315,9 @@ int hylra_decode_full_noalloc(const hylra_shape_t* shape, const void* q, const v
  * 2^31 (about a second) by default; the kernel then stops issuing copies,
  * waits (bounded) for the copies it already issued, finishes without trusting
  * the data it did not get, and sets HYLRA_STATUS_TIMEOUT in the workspace
- * status word (hylra_read_status).  Its outputs are then meaningless, and so
- * may be the workspace's per-(sequence, KV head) tickets: re-initialize the
- * workspace (hylra_workspace_init) before its next use.  This sets the limit for launches made after the call
+ * status word (hylra_read_status).  Its outputs are then meaningless; the
+ * workspace, cleared with hylra_read_status(..., clear = 1), serves the next
+ * call as before.  This sets the limit for launches made after the call
  * (process-wide; a CUDA graph keeps the limit it was captured with);
  * cycles <= 0 restores the default.  A short limit makes a watchdog fire on a
  * healthy GPU: tests use that to exercise the path.  Always HYLRA_OK. */

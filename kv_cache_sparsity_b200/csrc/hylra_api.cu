@@ -395,12 +395,7 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     const cudaError_t e = full ? cudaLaunchKernelEx(&cfg, decode_bf16_kernel<true>, tmK, tmV, p)
                                : cudaLaunchKernelEx(&cfg, decode_bf16_kernel<false>, tmK, tmV, p);
     if (e != cudaSuccess) return HYLRA_ERR_CUDA;
-    if (!full) {
-      // reuse layers merge inside the streaming kernel (last contributor)
-      if (last_ctas) *last_ctas = G;
-      return cudaGetLastError() == cudaSuccess ? HYLRA_OK : HYLRA_ERR_CUDA;
-    }
-    // the cross-CTA merge and top-k as the streaming kernel's dependent
+    // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
     const int nout = merge_out_ctas(s->num_q_heads / s->num_kv_heads,
                                     (long long)s->batch * s->num_kv_heads, G_sms);
@@ -411,7 +406,9 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     mcfg.attrs = attr;
     mcfg.numAttrs = 1;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    if (cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G) != cudaSuccess) return HYLRA_ERR_CUDA;
+    const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
+                                : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
+    if (em != cudaSuccess) return HYLRA_ERR_CUDA;
     if (last_ctas) *last_ctas = s->batch * s->num_kv_heads * (1 + nout);
   } else {
     if (full)

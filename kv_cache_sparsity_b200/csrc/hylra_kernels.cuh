@@ -252,19 +252,6 @@ __device__ __forceinline__ int part_owner(long long u, long long T, int G, int E
   return lo;
 }
 
-// The contributors of the (b, h) of a stage description under the split
-// part_lo (late CTAs take fewer units): first partial slot and count.
-__device__ __forceinline__ void set_contributors(const Params& p, const SmemCommon& c, int T,
-                                                 int G, int E, int D, StageMeta& m) {
-  if (m.b < 0 || m.b >= p.B || m.h < 0 || m.h >= p.Hkv) return;  // rejected by meta_sane
-  const int U = (c.prefix[m.b + 1] - c.prefix[m.b]) / p.Hkv;
-  if (U <= 0) return;
-  const long long start = c.prefix[m.b] + (long long)m.h * U;
-  const int first = part_owner(start, T, G, E, D);
-  m.first_slot = first + m.b * p.Hkv + m.h;
-  m.ncontrib = part_owner(start + U - 1, T, G, E, D) - first + 1;
-}
-
 // CTA that owns linear unit u when CTA c holds [floor(c*T/G), floor((c+1)*T/G));
 // with G <= T every such range is non-empty.
 __device__ __forceinline__ int owner_cta(long long u, long long T, int G) {
@@ -679,9 +666,7 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
 // through shared memory.
 template <bool FULL, int NT>
 __device__ void merge_bh(const Params& p, SmemCommon& c, const StageMeta& m, int ct) {
-  // contributors per thread and batch of loads (the bf16 streaming kernel merges
-  // few contributors per (b, h) and keeps its registers for the hot loop)
-  constexpr int CB = NT >= 256 ? 4 : 10;
+  constexpr int CB = NT >= 512 ? 6 : 10;  // contributors per thread and batch of loads
   const int bh = m.b * p.Hkv + m.h;
   const int nc = m.ncontrib;
   const int r = p.r;
@@ -1451,16 +1436,6 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
   // the same barriers even after a failed wait left a description unwritten.
   UnitIter cit;
   if (n > 0) cit.seek(c, p, lo);
-  if (!FULL) {
-    // Reuse layers merge in this kernel (the last contributor of each (b, h),
-    // by ticket), so sequences without units get their zero output here.
-    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-      if (c.prefix[b + 1] != c.prefix[b]) continue;
-      ensure_waited();
-      float* o = p.out + (size_t)b * p.Hq * HD;
-      for (int i = ct; i < p.Hq * HD; i += NT_BF16) o[i] = 0.f;
-    }
-  }
 
   for (int i = 0; i < n; ++i) {
     const int s = i % NSTAGE;
@@ -1518,22 +1493,13 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 5 << 8);
       ensure_waited();
       wa.to_comb(c.comb_o, c.comb_m, c.comb_z, cw);  // eight warp states -> four
-      if (FULL) {
-        store_partial<NT_BF16, false>(p, c, m, ct);  // merged by merge_kernel
-      } else {
-        // the last contributor of (b, h) merges its partials (flush_segments)
-        StageMeta mm = m;
-        set_contributors(p, c, T, G, E, D, mm);
-        store_partial<NT_BF16, true>(p, c, mm, ct);
-        if (c.nseg == MAX_SEGS) flush_segments<false, NT_BF16>(p, c, ct);
-      }
+      store_partial<NT_BF16, false>(p, c, m, ct);  // merged by merge_kernel
       if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 6 << 8);
     }
   }
   // every CTA waits once, so that this kernel completes only after its
   // predecessor (later kernels rely on that ordering without waiting)
   ensure_waited();
-  if (!FULL) flush_segments<false, NT_BF16>(p, c, ct);
   if (ct == 0) HYLRA_TRACE_EV(c.trace_n, 0, 9 << 8);
   if (*abort_flag && ct == 0) atomicOr(p.status, HYLRA_STATUS_TIMEOUT);
 }
