@@ -397,8 +397,11 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     if (e != cudaSuccess) return HYLRA_ERR_CUDA;
     // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
-    const int nout = merge_out_ctas(s->num_q_heads / s->num_kv_heads,
-                                    (long long)s->batch * s->num_kv_heads, G_sms);
+    // reset layers: per (b, h) a selection CTA and 1-4 output CTAs; reuse
+    // layers: one CTA per (b, h) (output merge, then the index-list check)
+    const int nout = full ? merge_out_ctas(s->num_q_heads / s->num_kv_heads,
+                                           (long long)s->batch * s->num_kv_heads, G_sms)
+                          : 0;
     mcfg.gridDim = dim3(s->batch * s->num_kv_heads, 1 + nout);
     mcfg.blockDim = dim3(NT_MERGE);
     mcfg.dynamicSmemBytes = 0;

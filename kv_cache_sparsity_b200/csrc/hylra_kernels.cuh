@@ -1551,10 +1551,16 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int part = (int)blockIdx.y;  // 0: statistics and top-k; 1..: output heads
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int r = p.r;
+  // output CTAs: y >= 1 on reset layers; on reuse layers the grid has one
+  // CTA per (b, h), which merges every head and then checks the index list
+  // (two CTAs would hold SMs that the next layer's CTAs need whole)
+  const bool outcta = FULL ? part > 0 : true;
   int g0 = 0, g1 = 0;
   if (part > 0) {
     merge_out_heads(r, (int)gridDim.y - 1, part, g0, g1);
     if (g0 >= g1) return;  // no heads left for this part (not launched so)
+  } else if (!FULL) {
+    g1 = r;
   }
   // The next layer's kernel may launch now: it reads nothing of this layer
   // and writes nothing before its own wait, which returns only after this
@@ -1593,7 +1599,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     // returns (values discarded: nothing is used before the wait).
     const int32_t* idx_row = (FULL ? p.topk_out : p.topk_in) + (size_t)bh * p.k;
     const void* ptr;
-    if (part == 0) {
+    if (!outcta) {
       const float* bs0 = FULL ? p.bstat + bstat_at(p, bh, 0, 0) : pbase;
       const float* bs1 = FULL ? p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1 : pbase;
       ptr = tid == 0 ? (const void*)bs0
@@ -1616,14 +1622,14 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 31 << 8);
   if (U == 0) {
     // a sequence without units: zero output (and no indices)
-    if (part > 0)
+    if (outcta)
       for (int i = g0 * HD + tid; i < g1 * HD; i += NT_MERGE) out_bh[i] = 0.f;
-    else if (FULL)
+    else
       for (int i = tid; i < p.k; i += NT_MERGE) p.topk_out[(size_t)bh * p.k + i] = -1;
     return;
   }
 
-  if (part > 0) {
+  if (outcta) {
     // ------------------------------------------ output rows g0..g1-1 (LSE merge)
     constexpr int CB = 10;  // contributors per thread and batch of loads
     const int ncol = (g1 - g0) * (HD / 4);  // float4 columns
@@ -1702,7 +1708,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       *reinterpret_cast<float4*>(out_bh + g * HD + 4 * d4) = o;
     }
     if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 17 << 8);
-    return;
+    if (FULL) return;  // reuse layers go on to the index-list check
   }
 
   const int tb = tid;  // 0..NT_MERGE-1

@@ -629,3 +629,36 @@ def test_token_scores_match_oracle(w):
             left = np.delete(S32[h], got[h][:kp]).astype(np.float64)
             if left.size:
                 assert chosen.min() >= left.max() * (1 - 2 * TOKEN_RTOL)
+
+
+def test_large_reuse_layer_stream_split_parity_and_index_flags():
+    """A reuse layer large enough for the stream-K split over every SM (16 x
+    8 heads x 16 blocks, clusters would leave SMs idle): outputs against the
+    oracle, and a duplicated, an out-of-range and a -1 entry handled as on the
+    cluster path (duplicate counted twice and flagged, out-of-range skipped
+    and flagged, -1 skipped)."""
+    w = W.custom("reuse_streamk", batch=16, seqlens=(2176,) * 15 + (2000,), num_q_heads=32,
+                 num_kv_heads=8, topk=16, seed=71)
+    run = T.Runner(w)
+    q0, K0, V0 = _layer(w, 0)
+    q1, K1, V1 = _layer(w, 1)
+    _, tk = run.full(q0, K0, V0)
+    assert run.status() == 0
+    out = run.reuse(q1, K1, V1, tk)
+    assert run.status() == 0
+    out, tkn = out.cpu().numpy(), tk.cpu().numpy()
+    for b in (0, 15):
+        T.check_out(out[b], T.oracle_reuse(w, q1, K1, V1, b, tkn[b]), "bf16", f"stream-K b={b}")
+    bad = tkn.copy()
+    bad[3, 2, 5] = bad[3, 2, 1]          # duplicate
+    bad[5, 1, 0] = 17 + 999              # out of range
+    bad[7, 0, 4] = -1                    # skipped
+    out2 = run.reuse(q1, K1, V1, torch.from_numpy(bad).cuda())
+    st = run.status()
+    assert st & H.STATUS_DUP_INDEX and st & H.STATUS_BAD_INDEX
+    out2 = out2.cpu().numpy()
+    ref_lists = bad.copy()
+    ref_lists[5, 1, 0] = -1              # the kernel skips an out-of-range block
+    for b in (3, 5, 7, 0):
+        T.check_out(out2[b], T.oracle_reuse(w, q1, K1, V1, b, ref_lists[b]), "bf16",
+                    f"stream-K flagged b={b}")
