@@ -637,8 +637,8 @@ def test_large_reuse_layer_stream_split_parity_and_index_flags():
     oracle, and a duplicated, an out-of-range and a -1 entry handled as on the
     cluster path (duplicate counted twice and flagged, out-of-range skipped
     and flagged, -1 skipped)."""
-    w = W.custom("reuse_streamk", batch=16, seqlens=(2176,) * 15 + (2000,), num_q_heads=32,
-                 num_kv_heads=8, topk=16, seed=71)
+    w = W.custom("reuse_streamk", batch=16, layers=2, seqlens=(2176,) * 15 + (2000,),
+                 num_q_heads=32, num_kv_heads=8, topk=16, seed=71)
     run = T.Runner(w)
     q0, K0, V0 = _layer(w, 0)
     q1, K1, V1 = _layer(w, 1)
