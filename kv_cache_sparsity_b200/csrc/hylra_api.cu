@@ -124,6 +124,27 @@ int make_tmap(CUtensorMap* tm, const void* base, long long rows) {
   return r == CUDA_SUCCESS ? HYLRA_OK : HYLRA_ERR_CUDA;
 }
 
+// CTAs of the merge kernel one SM holds at once (registers decide), per
+// device and template; 1 if the query fails.
+int merge_ctas_per_sm(bool full) {
+  static std::mutex mu;
+  static std::vector<int> cache;  // [dev * 2 + full]
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)cache.size() <= 2 * dev + 1) cache.resize(2 * dev + 2, 0);
+  int& v = cache[2 * dev + (full ? 1 : 0)];
+  if (v == 0) {
+    int n = 0;
+    const cudaError_t e =
+        full ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel<true>, NT_MERGE, 0)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel<false>, NT_MERGE, 0);
+    if (e != cudaSuccess) cudaGetLastError();
+    v = e == cudaSuccess ? std::max(1, n) : 1;
+  }
+  return v;
+}
+
 // Opt the bf16 kernels in to their dynamic shared memory once per device.
 int prepare_bf16_kernels() {
   static std::mutex mu;
@@ -332,7 +353,8 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
   p.idx_wait = (idx_from_prev || staged) ? 1 : 0;
   p.staged = staged ? 1 : 0;
   // CTAs launched early beside the preceding kernel stage their first blocks
-  // before it ends; the last late_ctas of the grid find their SMs still held
+  // before it ends; the last late_ctas of the grid (as many as the SMs the
+  // preceding kernel holds) find their SMs still held
   // and start after it: they take LATE_DEFICIT units fewer (bf16 streaming)
   p.late_from = G - std::min(G, std::max(0, late_ctas));
   p.late_deficit = pdl && late_ctas > 0 ? LATE_DEFICIT : 0;
@@ -412,7 +434,12 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
                                 : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
     if (em != cudaSuccess) return HYLRA_ERR_CUDA;
-    if (last_ctas) *last_ctas = s->batch * s->num_kv_heads * (1 + nout);
+    // SMs the merge kernel holds while the next layer's CTAs arrive (several
+    // of its CTAs share an SM)
+    if (last_ctas) {
+      const int per_sm = merge_ctas_per_sm(full);
+      *last_ctas = std::min(G_sms, (s->batch * s->num_kv_heads * (1 + nout) + per_sm - 1) / per_sm);
+    }
   } else {
     if (full)
       decode_f32_kernel<true><<<G, NT_F32, 0, stream>>>(p);
@@ -508,7 +535,7 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
   }
   const size_t per_layer = (size_t)shape->batch * shape->num_kv_heads * shape->topk;
   int last_reset = 0;
-  int prev_ctas = 0;  // CTAs of the kernel launched last (each holds an SM)
+  int prev_ctas = 0;  // SMs the kernel launched last holds (the next one's late CTAs)
   for (int l = 0; l < num_layers; ++l) {
     if (hooks && hooks->before && (rc = hooks->before(hooks->ctx, l))) return rc;
     if (policy[l]) {
