@@ -662,3 +662,46 @@ def test_large_reuse_layer_stream_split_parity_and_index_flags():
     for b in (3, 5, 7, 0):
         T.check_out(out2[b], T.oracle_reuse(w, q1, K1, V1, b, ref_lists[b]), "bf16",
                     f"stream-K flagged b={b}")
+
+
+def test_maximum_topk_reset_and_reuse():
+    """k = HYLRA_MAX_TOPK (1024) of 1500 blocks: the radix selection at its
+    largest k, and a reuse layer over 1024 blocks per head."""
+    w = W.custom("maxk", batch=1, layers=2, seqlens=(128 * 1500 - 9,), num_q_heads=8,
+                 num_kv_heads=2, topk=H.MAX_TOPK, structure="iid", seed=81)
+    run, (q, K, V), out, tk, swaps = _full_and_check(w)
+    assert np.all(tk[0] >= 0)  # k' = 1024 <= 1500 blocks: no padding
+    q1, K1, V1 = _layer(w, 1)
+    out1 = run.reuse(q1, K1, V1, torch.from_numpy(tk).cuda())
+    assert run.status() == 0
+    ref = T.oracle_reuse(w, q1, K1, V1, 0, tk[0])
+    T.check_out(out1.cpu().numpy()[0], ref, "bf16", "maxk reuse")
+
+
+def test_maximum_batch():
+    """B = HYLRA_MAX_BATCH (1024) sequences of mixed small lengths (0 .. 300
+    tokens, packed): the per-sequence prefix sums and splits at their widest;
+    sampled sequences against the oracle, empty ones zero with -1 indices."""
+    rng = np.random.default_rng(82)
+    lens = [int(x) for x in rng.integers(0, 301, size=H.MAX_BATCH)]
+    lens[5] = 0
+    w = W.custom("maxbatch", batch=H.MAX_BATCH, layers=2, seqlens=lens, num_q_heads=4,
+                 num_kv_heads=2, topk=2, packed=True, seed=83)
+    run = T.Runner(w)
+    q, K, V = _layer(w, 0)
+    out, tk = run.full(q, K, V)
+    assert run.status() == 0
+    out, tk = out.cpu().numpy(), tk.cpu().numpy()
+    assert np.all(out[5] == 0.0) and np.all(tk[5] == -1)
+    for b in (0, 1, 511, 1023):
+        o_ref, S32, tk_ref = T.oracle_full(w, q, K, V, b)
+        T.check_out(out[b], o_ref, "bf16", f"maxbatch b={b}")
+        for h in range(w.num_kv_heads):
+            T.check_topk_certified("maxbatch", tk[b, h], tk_ref[h], S32[h], w.topk,
+                                   f"maxbatch b={b} h={h}")
+    q1, K1, V1 = _layer(w, 1)
+    out1 = run.reuse(q1, K1, V1, torch.from_numpy(tk).cuda()).cpu().numpy()
+    assert run.status() == 0
+    assert np.all(out1[5] == 0.0)
+    for b in (0, 1023):
+        T.check_out(out1[b], T.oracle_reuse(w, q1, K1, V1, b, tk[b]), "bf16", f"maxbatch reuse {b}")
