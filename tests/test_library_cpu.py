@@ -262,3 +262,18 @@ def test_token_topk_rejects_bad_scores(lib):
             H.token_topk(s, 2)
     with pytest.raises(H.HylraError):
         H.token_topk(np.zeros((1, 5), dtype=np.float32), 2, lengths=np.array([6], dtype=np.int32))
+
+
+@pytest.mark.parametrize("field,limit,extra", [
+    ("batch", 1024, {}), ("topk", 1024, {}),
+    ("max_seqlen", 262144, {"kv_capacity": 262144 + 1}),
+])
+def test_limits_are_exact(lib, field, limit, extra):
+    """Each documented limit is accepted and the next value rejected as
+    unsupported, before anything touches a device."""
+    n = ctypes.c_size_t(0)
+    ok = _shape(**{field: limit, **extra})
+    # accepted: past validation (without a GPU the device query then fails)
+    assert lib.hylra_workspace_bytes(ctypes.byref(ok), ctypes.byref(n)) in (0, -3)
+    over = _shape(**{field: limit + 1, **extra})
+    assert lib.hylra_workspace_bytes(ctypes.byref(over), ctypes.byref(n)) == -2
