@@ -319,7 +319,8 @@ def decode_reuse_staged(shape: Shape, q, K_stage, V_stage, seqlens, topk_in, out
 
 def decode_step_offload(shape: Shape, policy: Sequence[int], qs, Ks, Vs, offloaded, seqlens,
                         outs, topk, K_stage, V_stage, ws, stream=None):
-    """Ks[l] / Vs[l] of layers with offloaded[l] = 1 are pinned torch CPU tensors."""
+    """Ks[l] / Vs[l] of layers with offloaded[l] = 1 are pinned torch CPU tensors;
+    K_stage / V_stage each hold two staging slots (2 x stage_bytes bytes)."""
     L = len(policy)
     pol = (ctypes.c_uint8 * L)(*[int(x) for x in policy])
     off = (ctypes.c_uint8 * L)(*[int(x) for x in offloaded])
