@@ -233,18 +233,10 @@ __device__ __forceinline__ long long row_base(const Params& p, int b, int h) {
 // [part_lo(c), part_lo(c+1)).  The CTAs from E on start late (inside a decode
 // step their SMs are still held by the preceding kernel while the others
 // already stage their first blocks), so each takes D units fewer than the
-// rest; D applies only when every late CTA still gets a unit.  The host
-// passes the least D (p.late_deficit, 0: none); the late CTAs' delay grows
-// with the layer (the preceding layer's tail and merge), so D grows with the
-// units per CTA, a fifth of them, up to LATE_DEFICIT_MAX (B200 traces: late
-// CTAs ~3 us behind at 14 units per CTA, ~8 us at 28).
-constexpr int LATE_DEFICIT_MAX = 6;
+// rest; D applies only when every late CTA still gets a unit.
 __device__ __forceinline__ int late_deficit(const Params& p, long long T, int G) {
-  const long long E = min(max(p.late_from, 0), G), L = G - E;
-  if (p.late_deficit <= 0 || L <= 0) return 0;
-  const long long D = max((long long)p.late_deficit,
-                          min((long long)LATE_DEFICIT_MAX, T / (5ll * G)));
-  return T + L * D >= (long long)G * (D + 1) ? (int)D : 0;
+  const long long E = min(max(p.late_from, 0), G), L = G - E, D = p.late_deficit;
+  return (D > 0 && L > 0 && T + L * D >= (long long)G * (D + 1)) ? (int)D : 0;
 }
 __device__ __forceinline__ long long part_lo(long long c, long long T, int G, int E, int D) {
   const long long L = G - E;
