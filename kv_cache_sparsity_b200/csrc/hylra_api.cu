@@ -124,8 +124,8 @@ int make_tmap(CUtensorMap* tm, const void* base, long long rows) {
   return r == CUDA_SUCCESS ? HYLRA_OK : HYLRA_ERR_CUDA;
 }
 
-// CTAs of the merge kernel one SM holds at once (registers decide), per
-// device and template; 1 if the query fails.
+// CTAs of a merge kernel one SM holds at once (registers decide), per
+// device and kernel (reset layers' or reuse layers'); 1 if the query fails.
 int merge_ctas_per_sm(bool full) {
   static std::mutex mu;
   static std::vector<int> cache;  // [dev * 2 + full]
@@ -137,8 +137,8 @@ int merge_ctas_per_sm(bool full) {
   if (v == 0) {
     int n = 0;
     const cudaError_t e =
-        full ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel<true>, NT_MERGE, 0)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel<false>, NT_MERGE, 0);
+        full ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel, NT_MERGE, 0)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_reuse_kernel, NT_RMERGE, 0);
     if (e != cudaSuccess) cudaGetLastError();
     v = e == cudaSuccess ? std::max(1, n) : 1;
   }
@@ -420,25 +420,26 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
     // reset layers: per (b, h) a selection CTA and 1-4 output CTAs; reuse
-    // layers: one CTA per (b, h) (output merge, then the index-list check)
-    const int nout = full ? merge_out_ctas(s->num_q_heads / s->num_kv_heads,
-                                           (long long)s->batch * s->num_kv_heads, G_sms)
-                          : 0;
-    mcfg.gridDim = dim3(s->batch * s->num_kv_heads, 1 + nout);
-    mcfg.blockDim = dim3(NT_MERGE);
+    // layers: one small CTA per (b, h) (output merge and index-list check)
+    // that fits beside a streaming CTA
+    const int nbh = s->batch * s->num_kv_heads;
+    const int nout =
+        full ? merge_out_ctas(s->num_q_heads / s->num_kv_heads, (long long)nbh, G_sms) : 0;
+    mcfg.gridDim = dim3(nbh, 1 + nout);
+    mcfg.blockDim = dim3(full ? NT_MERGE : NT_RMERGE);
     mcfg.dynamicSmemBytes = 0;
     mcfg.stream = stream;
     mcfg.attrs = attr;
     mcfg.numAttrs = 1;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel<true>, p, G)
-                                : cudaLaunchKernelEx(&mcfg, merge_kernel<false>, p, G);
+    const cudaError_t em = full ? cudaLaunchKernelEx(&mcfg, merge_kernel, p, G)
+                                : cudaLaunchKernelEx(&mcfg, merge_reuse_kernel, p, G);
     if (em != cudaSuccess) return HYLRA_ERR_CUDA;
     // SMs the merge kernel holds while the next layer's CTAs arrive (several
     // of its CTAs share an SM)
     if (last_ctas) {
       const int per_sm = merge_ctas_per_sm(full);
-      *last_ctas = std::min(G_sms, (s->batch * s->num_kv_heads * (1 + nout) + per_sm - 1) / per_sm);
+      *last_ctas = std::min(G_sms, (nbh * (1 + nout) + per_sm - 1) / per_sm);
     }
   } else {
     if (full)

@@ -24,9 +24,11 @@
 //     block's local max and probability sum relative to it: the exact
 //     ingredients of the block's attention mass once the global max and sum
 //     are known.
-//   * merge_kernel: the streaming kernel's programmatic dependent, one CTA
-//     per (b, h): LSE merge of the segments' partials into the output and,
-//     on reset layers, the block masses and the top-k (topk_select).
+//   * merge_kernel (reset layers) and merge_reuse_kernel (reuse layers): the
+//     streaming kernel's programmatic dependent, per (b, h): LSE merge of the
+//     segments' partials into the output and, on reset layers, the block
+//     masses and the top-k (topk_select); on reuse layers the index-list
+//     check.
 //   * decode_reuse_cluster_kernel: a reuse layer as one thread-block
 //     cluster per (b, h); the CTAs' states meet in CTA 0's shared memory
 //     (st.async), which writes the output.
@@ -1506,16 +1508,17 @@ __global__ void __launch_bounds__(NTHR_BF16, 1)
 
 // ------------------------------------------------------------ merge kernel
 //
-// Runs after decode_bf16_kernel (as its programmatic dependent).  The kernel
-// boundary makes the streaming kernel's partials visible; no fence or ticket
-// is needed.  Grid (B*Hkv, 1 + merge_out_ctas(..)): for each (sequence, KV
-// head) independent CTAs run side by side so that none waits for another and
-// each SM loads only its share of the partials:
-//   y = 0      (reset layers) derives each head's max and sum straight from
-//              the contributors' (m, Z) pairs, scores the blocks and selects
-//              the top-k; (reuse layers) checks the index list for repeats;
+// Reset layers: runs after decode_bf16_kernel (as its programmatic
+// dependent).  The kernel boundary makes the streaming kernel's partials
+// visible; no fence or ticket is needed.  Grid (B*Hkv, 1 + merge_out_ctas(..)):
+// for each (sequence, KV head) independent CTAs run side by side so that none
+// waits for another and each SM loads only its share of the partials:
+//   y = 0      derives each head's max and sum straight from the
+//              contributors' (m, Z) pairs, scores the blocks and selects the
+//              top-k;
 //   y = 1..    each merges the contributors' partial rows of its heads into
 //              the output.
+// (Reuse layers merge in merge_reuse_kernel.)
 constexpr int BAR_TOPK = 3;           // named barrier of the selection CTA
 
 // Output CTAs per (b, h): one per head up to four when the grid stays
@@ -1541,7 +1544,6 @@ struct SmemMerge {
   SmemCommon c;            // prefix sums; head statistics, keys and top-k scratch
 };
 
-template <bool FULL>
 __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constant__ Params p,
                                                             int grid_stream) {
   __shared__ SmemMerge sm;
@@ -1551,16 +1553,11 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
   const int part = (int)blockIdx.y;  // 0: statistics and top-k; 1..: output heads
   const int b = bh / p.Hkv, h = bh - b * p.Hkv;
   const int r = p.r;
-  // output CTAs: y >= 1 on reset layers; on reuse layers the grid has one
-  // CTA per (b, h), which merges every head and then checks the index list
-  // (two CTAs would hold SMs that the next layer's CTAs need whole)
-  const bool outcta = FULL ? part > 0 : true;
+  const bool outcta = part > 0;  // output rows; else statistics and top-k
   int g0 = 0, g1 = 0;
-  if (part > 0) {
+  if (outcta) {
     merge_out_heads(r, (int)gridDim.y - 1, part, g0, g1);
     if (g0 >= g1) return;  // no heads left for this part (not launched so)
-  } else if (!FULL) {
-    g1 = r;
   }
   // The next layer's kernel may launch now: it reads nothing of this layer
   // and writes nothing before its own wait, which returns only after this
@@ -1573,7 +1570,7 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 30 << 8);
   }
   // everything that does not depend on the streaming kernel's output first
-  build_prefix(p, c, FULL);
+  build_prefix(p, c, true);
   const int seqlen = valid_seqlen(p, b, false);
   __syncthreads();
   const int T = c.prefix[p.B];
@@ -1590,18 +1587,17 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
     first += bh;  // partial slot of contributor c is c + bh
   }
   const int nb = (seqlen + BLK - 1) / BLK;
-  const int kp = min(p.k, nb);
   const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
   float* out_bh = p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD;
   if (U > 0 && tid < 6) {
     // Before the wait: a line at each end of every range read or written
     // after it, so that their address translations are cached when it
     // returns (values discarded: nothing is used before the wait).
-    const int32_t* idx_row = (FULL ? p.topk_out : p.topk_in) + (size_t)bh * p.k;
+    const int32_t* idx_row = p.topk_out + (size_t)bh * p.k;
     const void* ptr;
     if (!outcta) {
-      const float* bs0 = FULL ? p.bstat + bstat_at(p, bh, 0, 0) : pbase;
-      const float* bs1 = FULL ? p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1 : pbase;
+      const float* bs0 = p.bstat + bstat_at(p, bh, 0, 0);
+      const float* bs1 = p.bstat + bstat_at(p, bh, r - 1, max(nb - 1, 0)) + 1;
       ptr = tid == 0 ? (const void*)bs0
           : tid == 1 ? (const void*)bs1
           : tid == 2 ? (const void*)idx_row
@@ -1708,12 +1704,12 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       *reinterpret_cast<float4*>(out_bh + g * HD + 4 * d4) = o;
     }
     if (tid == 0) HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 17 << 8);
-    if (FULL) return;  // reuse layers go on to the index-list check
+    return;
   }
 
   const int tb = tid;  // 0..NT_MERGE-1
   const int wb = tb >> 5, lane = tb & 31;
-  if (FULL) {
+  {
     // --------------------------------------------- block scores and top-k
     // block records of this thread's first SPT blocks (tb, tb + 256, ...),
     // all loaded up front, together with the head statistics below
@@ -1817,22 +1813,168 @@ __global__ void __launch_bounds__(NT_MERGE, 1) merge_kernel(const __grid_constan
       HYLRA_TRACE_VAL(c.trace_n, c.trace_cta, 44 << 8, HYLRA_CLOCK());
       HYLRA_TRACE_CTA(c.trace_n, c.trace_cta, 13 << 8);
     }
-
-  } else {
-    // a reused list naming one block twice counts that block twice: flag it
-    const int32_t* idx = p.topk_in + (size_t)bh * p.k;
-    int32_t* sidx = reinterpret_cast<int32_t*>(&c.comb_o[0][0][0]);
-    for (int e = tb; e < kp; e += NT_MERGE) sidx[e] = __ldcg(idx + e);
-    named_bar_sync(BAR_TOPK, NT_MERGE);
-    bool dup = false;
-    for (int e = tb; e < kp; e += NT_MERGE) {
-      const int32_t v = sidx[e];
-      if (v < 0) continue;
-      for (int j = 0; j < e; ++j) dup |= sidx[j] == v;
-    }
-    if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
   }
-  (void)wb;
+}
+
+// ------------------------------------------------------ reuse merge kernel
+//
+// Reuse layers on the bf16 streaming kernel: its programmatic dependent, one
+// CTA of NT_RMERGE threads per (b, h) that LSE-merges the contributors'
+// partial rows into the output and checks the index list for repeats.  Its
+// CTAs start on SMs that this layer's streaming CTAs leave and wait there for
+// the layer to end; an SM that holds one cannot take a streaming CTA of the
+// next layer (the nine warps of a streaming CTA leave too few registers in
+// one SM sub-partition for any other CTA beside them, and too little shared
+// memory beside a larger one).  So the CTA is small (four warps, under 100
+// registers a thread, 272 bytes of shared memory: five share an SM) and
+// holds as few of the SMs that the next layer's CTAs wait for as it can.
+constexpr int NT_RMERGE = 128;
+
+__global__ void __launch_bounds__(NT_RMERGE, 4) merge_reuse_kernel(const __grid_constant__ Params p,
+                                                                  int grid_stream) {
+  __shared__ uint32_t seen[MAX_NB / 32];  // blocks named so far in the index list
+  __shared__ int units[2];                // units before sequence b (all heads), all units
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int bh = (int)blockIdx.x;
+  const int b = bh / p.Hkv, h = bh - b * p.Hkv;
+  const int r = p.r;
+  // the next layer's kernel may launch now (as in merge_kernel)
+  griddep_launch_dependents();
+#ifdef HYLRA_TRACE
+  int tn = 0;
+  const int tcta = 160 + bh;
+  if (tid == 0) HYLRA_TRACE_CTA(tn, tcta, 30 << 8);
+#endif
+  // everything that does not depend on the streaming kernel's output first:
+  // the unit counts (warp 0, no per-sequence array) and the split
+  if (tid < 32) {
+    int before = 0, total = 0;
+    for (int s = lane; s < p.B; s += 32) {
+      const int n = units_of(p, valid_seqlen(p, s, false), false) * p.Hkv;
+      total += n;
+      if (s < b) before += n;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, off);
+      total += __shfl_xor_sync(0xffffffffu, total, off);
+    }
+    if (lane == 0) {
+      units[0] = before;
+      units[1] = total;
+    }
+  }
+  for (int i = tid; i < MAX_NB / 32; i += NT_RMERGE) seen[i] = 0u;
+  const int seqlen = valid_seqlen(p, b, false);
+  __syncthreads();
+  const int T = units[1];
+  const int nb = (seqlen + BLK - 1) / BLK;
+  const int U = units_of(p, seqlen, false);
+  const int kp = min(p.k, nb);
+  const int G = min(grid_stream, max(T, 1));
+  const int E = min(max(p.late_from, 0), G), D = late_deficit(p, T, G);
+  const int start = units[0] + h * U;
+  int first = 0, nc = 0;
+  if (U > 0) {
+    // the streaming kernel's static split (part_lo): every CTA of it owns
+    // at least one unit, so the owners of (b, h) are contiguous
+    first = part_owner(start, T, G, E, D);
+    nc = part_owner((long long)start + U - 1, T, G, E, D) - first + 1;
+    first += bh;  // partial slot of contributor c is c + bh
+  }
+  const float* pbase = p.partials + (size_t)first * SLOT_FLOATS;
+  float* out_bh = p.out + ((size_t)b * p.Hq + (size_t)h * r) * HD;
+  const int32_t* idx = p.topk_in + (size_t)bh * p.k;
+  if (U > 0 && tid < 4) {
+    // before the wait: a line at each end of the ranges read or written after
+    // it (address translations; values discarded)
+    const void* ptr = tid == 0 ? (const void*)pbase
+                    : tid == 1 ? (const void*)(pbase + (size_t)nc * SLOT_FLOATS - 1)
+                    : tid == 2 ? (const void*)out_bh
+                               : (const void*)(out_bh + r * HD - 1);
+    touch_line(ptr);
+  }
+  griddep_wait();  // the streaming kernel has completed: partials are visible
+#ifdef HYLRA_TRACE
+  if (tid == 0) HYLRA_TRACE_CTA(tn, tcta, 31 << 8);
+#endif
+  if (U == 0) {
+    // a sequence without units: zero output
+    for (int i = tid; i < r * HD; i += NT_RMERGE) out_bh[i] = 0.f;
+    return;
+  }
+  // this thread's entries of the index list, loaded together with the partials
+  constexpr int EPT = HYLRA_MAX_TOPK / NT_RMERGE;
+  int32_t ent[EPT];
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const int e = tid + u * NT_RMERGE;
+    ent[u] = e < kp ? __ldcg(idx + e) : -1;
+  }
+  // output rows: thread t merges float4 column t (and t + 128 when r > 4)
+  // over every contributor, online, in batches of CB loads
+  constexpr int CB = 8;
+  for (int col = tid; col < r * (HD / 4); col += NT_RMERGE) {
+    const int g = col / (HD / 4), d4 = col % (HD / 4);
+    float M = -INFINITY, Z = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < nc; j0 += CB) {
+      float mv[CB], zv[CB];
+      float4 ov[CB];
+#pragma unroll
+      for (int u = 0; u < CB; ++u) {
+        const int j = j0 + u;  // the same in every thread
+        mv[u] = -INFINITY;
+        if (j < nc) {
+          const float* sl = pbase + (size_t)j * SLOT_FLOATS;
+          mv[u] = __ldcg(sl + GMAX * HD + g);
+          zv[u] = __ldcg(sl + GMAX * HD + GMAX + g);
+          ov[u] = __ldcg(reinterpret_cast<const float4*>(sl + g * HD + 4 * d4));
+        }
+      }
+      float mb = M;
+#pragma unroll
+      for (int u = 0; u < CB; ++u) mb = fmaxf(mb, mv[u]);
+      if (mb != -INFINITY) {
+        const float fo = M == -INFINITY ? 0.f : ex2_approx(M - mb);
+        acc.x *= fo;
+        acc.y *= fo;
+        acc.z *= fo;
+        acc.w *= fo;
+        Z *= fo;
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+          if (mv[u] == -INFINITY) continue;
+          const float f = ex2_approx(mv[u] - mb);
+          acc.x = fmaf(ov[u].x, f, acc.x);
+          acc.y = fmaf(ov[u].y, f, acc.y);
+          acc.z = fmaf(ov[u].z, f, acc.z);
+          acc.w = fmaf(ov[u].w, f, acc.w);
+          Z = fmaf(zv[u], f, Z);
+        }
+        M = mb;
+      }
+    }
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (Z > 0.f) o = make_float4(acc.x / Z, acc.y / Z, acc.z / Z, acc.w / Z);
+    *reinterpret_cast<float4*>(out_bh + g * HD + 4 * d4) = o;
+  }
+  // a reused list naming one block twice counts that block twice: flag it
+  // (entries outside the sequence are skipped and flagged by the streaming
+  // kernel)
+  bool dup = false;
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const int32_t v = ent[u];
+    if (v >= 0 && v < nb) {
+      const uint32_t bit = 1u << (v & 31);
+      dup |= (atomicOr(&seen[v >> 5], bit) & bit) != 0u;
+    }
+  }
+  if (dup) atomicOr(p.status, HYLRA_STATUS_DUP_INDEX);
+#ifdef HYLRA_TRACE
+  if (tid == 0) HYLRA_TRACE_CTA(tn, tcta, 17 << 8);
+#endif
 }
 
 // ------------------------------------------------- cluster reuse kernel
