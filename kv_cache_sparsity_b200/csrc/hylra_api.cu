@@ -124,21 +124,20 @@ int make_tmap(CUtensorMap* tm, const void* base, long long rows) {
   return r == CUDA_SUCCESS ? HYLRA_OK : HYLRA_ERR_CUDA;
 }
 
-// CTAs of a merge kernel one SM holds at once (registers decide), per
-// device and kernel (reset layers' or reuse layers'); 1 if the query fails.
-int merge_ctas_per_sm(bool full) {
+// CTAs of the reset layers' merge kernel one SM holds at once (registers
+// decide), per device; 1 if the query fails.
+int merge_ctas_per_sm() {
   static std::mutex mu;
-  static std::vector<int> cache;  // [dev * 2 + full]
+  static std::vector<int> cache;  // [dev]
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   std::lock_guard<std::mutex> lock(mu);
-  if ((int)cache.size() <= 2 * dev + 1) cache.resize(2 * dev + 2, 0);
-  int& v = cache[2 * dev + (full ? 1 : 0)];
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  int& v = cache[dev];
   if (v == 0) {
     int n = 0;
     const cudaError_t e =
-        full ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel, NT_MERGE, 0)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_reuse_kernel, NT_RMERGE, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel, NT_MERGE, 0);
     if (e != cudaSuccess) cudaGetLastError();
     v = e == cudaSuccess ? std::max(1, n) : 1;
   }
@@ -436,9 +435,12 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
                                 : cudaLaunchKernelEx(&mcfg, merge_reuse_kernel, p, G);
     if (em != cudaSuccess) return HYLRA_ERR_CUDA;
     // SMs the merge kernel holds while the next layer's CTAs arrive (several
-    // of its CTAs share an SM)
+    // of its CTAs share an SM).  The reuse merge's CTAs could share an SM
+    // five at a time, but they arrive as the streaming CTAs leave and spread
+    // over the SMs freed first: a trace of the ragged16 step found its 128
+    // CTAs on 42-57 SMs, so count three to an SM.
     if (last_ctas) {
-      const int per_sm = merge_ctas_per_sm(full);
+      const int per_sm = full ? merge_ctas_per_sm() : 3;
       *last_ctas = std::min(G_sms, (nbh * (1 + nout) + per_sm - 1) / per_sm);
     }
   } else {

@@ -527,19 +527,22 @@ __device__ void topk_select(const Params& p, SmemCommon& c, int bh, int nb, int 
     if (rw < kp) lists[wid * 32 + rw] = v;
     named_bar_sync(BAR, NT);
     if (rw < kp && v != 0ull) {
-      // the NW searches advance in lock step (independent loads in flight);
-      // in its own warp's list an entry finds exactly `rw` predecessors
+      // how many entries of each list exceed v: a binary search over the 32
+      // places (a list past its kp entries holds zeros, below every key), the
+      // NW searches in lock step, each step a select (independent loads in
+      // flight, no branch); in its own warp's list an entry finds exactly
+      // `rw` predecessors
       int pos[NW];
 #pragma unroll
       for (int w = 0; w < NW; ++w) pos[w] = 0;
 #pragma unroll
-      for (int step = 32; step > 0; step >>= 1) {
+      for (int step = 16; step > 0; step >>= 1) {
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const int t = pos[w] + step;
-          if (t <= kp && lists[w * 32 + t - 1] > v) pos[w] = t;
-        }
+        for (int w = 0; w < NW; ++w)
+          pos[w] += lists[w * 32 + pos[w] + step - 1] > v ? step : 0;
       }
+#pragma unroll
+      for (int w = 0; w < NW; ++w) pos[w] += lists[w * 32 + pos[w]] > v ? 1 : 0;
       int rank = 0;
 #pragma unroll
       for (int w = 0; w < NW; ++w) rank += pos[w];
