@@ -564,8 +564,9 @@ int run_step(const hylra_shape_t* shape, int32_t num_layers, const uint8_t* poli
 // overlap the step.  Layer 0's query goes first on the caller's stream, the
 // other layers' queries on the copy stream (layer 1 waits for them), the
 // outputs of every OUT_CHUNK layers go back as soon as those layers are done
-// and the indices once the last reset layer is; the caller's stream joins
-// the copy stream at the end.
+// (towards the end in halving chunks, so that the copy left after the last
+// layer is one layer's) and the indices once the last reset layer is; the
+// caller's stream joins the copy stream at the end.
 // The stream and events are per host thread and device.
 constexpr int OUT_CHUNK = 8;
 
@@ -647,8 +648,10 @@ int host_pipe_before(void* ctx, int layer) {
 
 int host_pipe_after(void* ctx, int layer) {
   HostPipe* hp = static_cast<HostPipe*>(ctx);
-  const int done = layer + 1;
-  const bool chunk = done % OUT_CHUNK == 0 && done < hp->num_layers;
+  const int done = layer + 1, left = hp->num_layers - done;
+  // every OUT_CHUNK layers, and where the layers left halve below that
+  const bool chunk = left > 0 && (done % OUT_CHUNK == 0 ||
+                                  (left < OUT_CHUNK && (left & (left - 1)) == 0));
   if (chunk || layer == hp->last_reset)
     return host_pipe_copy_out(hp, chunk ? done : hp->copied, layer == hp->last_reset);
   return HYLRA_OK;

@@ -664,6 +664,38 @@ def test_large_reuse_layer_stream_split_parity_and_index_flags():
                     f"stream-K flagged b={b}")
 
 
+def test_large_reuse_layer_group8_empty_sequence_and_repeat():
+    """The reuse merge of the stream-K path with r = 8 q-heads per KV head
+    (two float4 columns per merge thread), a sequence without tokens (no
+    units: zero output) and a repeated index (counted twice, flagged): 16
+    sequences x 4 KV heads x 24 reused blocks, large enough for the split
+    over every SM."""
+    lens = (3840, 4000, 3300, 3968, 3100, 0, 4096, 3500, 3072, 3900, 3700, 3200, 4000, 3333, 3999,
+            3600)
+    w = W.custom("reuse_streamk_r8", batch=16, layers=2, seqlens=lens, num_q_heads=32,
+                 num_kv_heads=4, topk=24, seed=92)
+    run = T.Runner(w)
+    q0, K0, V0 = _layer(w, 0)
+    q1, K1, V1 = _layer(w, 1)
+    _, tk = run.full(q0, K0, V0)
+    assert run.status() == 0
+    tkn = tk.cpu().numpy()
+    assert np.all(tkn[5] == -1)
+    out = run.reuse(q1, K1, V1, tk)
+    assert run.status() == 0
+    out = out.cpu().numpy()
+    assert np.all(out[5] == 0.0)
+    for b in (0, 6, 15):
+        T.check_out(out[b], T.oracle_reuse(w, q1, K1, V1, b, tkn[b]), "bf16", f"r8 b={b}")
+    bad = tkn.copy()
+    bad[6, 3, 10] = bad[6, 3, 2]  # repeated: counted twice, flagged
+    out2 = run.reuse(q1, K1, V1, torch.from_numpy(bad).cuda())
+    assert run.status() & H.STATUS_DUP_INDEX
+    out2 = out2.cpu().numpy()
+    for b in (6, 0):
+        T.check_out(out2[b], T.oracle_reuse(w, q1, K1, V1, b, bad[b]), "bf16", f"r8 repeat b={b}")
+
+
 def test_maximum_topk_reset_and_reuse():
     """k = HYLRA_MAX_TOPK (1024) of 1500 blocks: the radix selection at its
     largest k, and a reuse layer over 1024 blocks per head."""
