@@ -46,7 +46,9 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
     """Compile libhylra.so if a source changed (or ``force``); return its path."""
     if not force and not ptxas_info and not needs_build():
         return LIB
-    tmp = LIB + ".tmp"
+    # one temporary file per process: several ranks may build at once, and
+    # each then installs a complete library with one atomic rename
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = [nvcc_path(), "-gencode", GENCODE, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC,-O3", "-shared", "-I", INCLUDE, "-I", CSRC,
            "-o", tmp] + SOURCES
@@ -56,6 +58,8 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
+        if os.path.exists(tmp):
+            os.remove(tmp)
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if ptxas_info or verbose:
         sys.stdout.write(res.stdout + res.stderr)
