@@ -34,3 +34,46 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
+
+
+def test_algorithmic_bytes_follow_the_shapes():
+    """The roofline's algorithmic bytes: K and V (bf16, d = 128) of every
+    cached token of every KV head for a reset layer, of the k' selected
+    128-token blocks per head for a reuse layer; a step adds them by policy."""
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    from kv_cache_sparsity_b200 import workloads as W
+    kv = 2 * 2 * 128  # K and V, bf16, per token and KV head
+    expect = {
+        "llama8b_32k": (8 * 32768 * kv, 8 * 16 * 128 * kv),
+        "llama8b_b8_64k": (8 * 8 * 65536 * kv, 8 * 8 * 32 * 128 * kv),
+        "llama8b_128k": (8 * 131072 * kv, 8 * 64 * 128 * kv),
+    }
+    for name, (full, reuse) in expect.items():
+        w = W.config(name)
+        assert w.kv_bytes_per_layer() == full, name
+        assert w.kv_bytes_reuse_layer() == reuse, name
+    w = W.config("ragged16")
+    assert w.kv_bytes_per_layer() == 8 * sum(w.seqlens) * kv
+    assert min(w.seqlens) >= 32 * 128  # every sequence has k = 32 blocks to reuse
+    assert w.kv_bytes_reuse_layer() == 16 * 8 * 32 * 128 * kv
+    policy = (1, 0, 0, 1) + (0,) * (w.layers - 4)
+    assert bench.step_bytes(w, policy) == 2 * w.kv_bytes_per_layer() + (w.layers - 2) * \
+        w.kv_bytes_reuse_layer()
+    args = argparse.Namespace(policy="dp", theta=None, profile_steps=1, profile_seeds=1,
+                              token_topk=0, shard="batch")
+    cfg = bench.config_of(w, policy, args, 1)
+    assert cfg["policy"] == "RUUR" + "U" * (w.layers - 4) and cfg["resets"] == 2
+    assert set(cfg) == {"workload", "policy", "policy_rule", "resets", "l2", "parallelism"}
+
+
+def test_seed_variant_keeps_shapes_and_changes_the_draw():
+    sys.path.insert(0, ROOT)
+    import bench
+    from kv_cache_sparsity_b200 import workloads as W
+    w = W.config("ragged16")
+    assert bench.seed_variant(w, 0) is w
+    v = bench.seed_variant(w, 3)
+    assert v.seed != w.seed and v.seqlens == w.seqlens and v.layers == w.layers
+    assert (v.num_q_heads, v.num_kv_heads, v.topk) == (w.num_q_heads, w.num_kv_heads, w.topk)
