@@ -419,8 +419,8 @@ int launch(const hylra_shape_t* s, bool full, const void* q, const void* K, cons
     // the cross-CTA merge (and top-k) as the streaming kernel's dependent
     cudaLaunchConfig_t mcfg = {};
     // reset layers: per (b, h) a selection CTA and 1-4 output CTAs; reuse
-    // layers: one small CTA per (b, h) (output merge and index-list check)
-    // that fits beside a streaming CTA
+    // layers: one small CTA per (b, h) (output merge and index-list check),
+    // so that its CTAs hold few of the SMs the next layer's CTAs wait for
     const int nbh = s->batch * s->num_kv_heads;
     const int nout =
         full ? merge_out_ctas(s->num_q_heads / s->num_kv_heads, (long long)nbh, G_sms) : 0;
